@@ -1,0 +1,500 @@
+"""Pins of the CPU oracle to facts the pages and the mathematics fix.
+
+None of these re-types an oracle formula: each compares the oracle with a
+different route to the same answer (brute force, a library routine the
+oracle does not use, a closed form, an invariant, or numbers printed on the
+pages, stored under tests/golden/ with their citation).
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from draft_tree_build_ddtree_b200 import datagen
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _cfg1():
+    w = datagen.workload(1)
+    z = datagen.drafter_logits(w).to(torch.float64).numpy()
+    ids, lp32, lse32, lp64 = oracle.topk(z, w.K)
+    return w, z, ids, lp32, lse32, lp64
+
+
+# ---------------------------------------------------------------- log-softmax
+
+def test_log_softmax_normalises_and_matches_torch():
+    g = torch.Generator().manual_seed(7)
+    z = (torch.randn(6, 1000, generator=g, dtype=torch.float64) * 5).numpy()
+    z[0, :10] = -np.inf
+    lp, lse = oracle.log_softmax(z)
+    assert np.all(np.abs(np.exp(lp).sum(-1) - 1.0) < 1e-12)
+    ref = torch.log_softmax(torch.from_numpy(z), dim=-1).numpy()
+    fin = np.isfinite(ref)
+    assert np.array_equal(fin, np.isfinite(lp))
+    assert np.max(np.abs(lp[fin] - ref[fin])) < 1e-12
+    ref_lse = torch.logsumexp(torch.from_numpy(z), dim=-1).numpy()
+    assert np.max(np.abs(lse - ref_lse)) < 1e-12
+
+
+def test_log_softmax_rejects_nan():
+    z = np.zeros((2, 8))
+    z[1, 3] = np.nan
+    with pytest.raises(ValueError):
+        oracle.log_softmax(z)
+
+
+# ---------------------------------------------------------------- top-K
+
+def _rank_by_counting(row, i):
+    """Position of token i in (value desc, id asc): count who beats it."""
+    v = row[i]
+    return int(np.sum(row > v) + np.sum((row == v) & (np.arange(row.size) < i)))
+
+
+@pytest.mark.parametrize("V,K", [(50, 7), (64, 64), (300, 33)])
+def test_topk_ranks_by_counting_with_ties(V, K):
+    g = torch.Generator().manual_seed(V * 31 + K)
+    z = torch.randint(-4, 5, (5, V), generator=g).to(torch.float64).numpy()
+    z[0, 3] = -0.0
+    z[0, 4] = 0.0
+    z[1, :5] = -np.inf
+    ids, lp32, lse32, lp64 = oracle.topk(z, K)
+    for r in range(z.shape[0]):
+        ranks = [_rank_by_counting(z[r], int(i)) for i in ids[r]]
+        assert ranks == list(range(K))
+        assert lp32.dtype == np.float32
+        assert np.all(lp32[r] == lp64[r, ids[r]].astype(np.float32))
+
+
+def test_topk_signed_zero_and_neg_inf():
+    z = np.array([[-0.0, 0.0, -np.inf, -1.0, -0.0]])
+    ids, *_ = oracle.topk(z, 5)
+    assert ids[0].tolist() == [0, 1, 4, 3, 2]
+
+
+# ---------------------------------------------------------------- heap (Prop. 2, 3)
+
+def test_prop2_heap_equals_bruteforce_config1():
+    w, z, ids, lp32, *_ = _cfg1()
+    t = oracle.build_tree(ids[0], lp32[0], 0, w.B)
+    brute = oracle.bruteforce_top_prefixes(lp32[0], w.B)
+    assert t.tuples[1:] == brute
+    assert t.n_nodes == w.B + 1
+    # prefix-closed, and parent indices point at the tuple's prefix
+    index = {tup: i for i, tup in enumerate(t.tuples)}
+    for i in range(1, t.n_nodes):
+        tup = t.tuples[i]
+        assert tup[:-1] in index
+        assert index[tup[:-1]] == t.parent[i] < i
+        assert t.depth[i] == len(tup)
+        assert t.node_rank[i] == tup[-1]
+        assert t.node_token[i] == ids[0, len(tup) - 1, tup[-1]]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_prop2_heap_equals_bruteforce_with_exact_ties(seed):
+    # A coarse table makes many prefixes tie exactly in fp32, so the
+    # tuple tie-break decides the order.
+    g = torch.Generator().manual_seed(100 + seed)
+    L, K, B = 3, 4, 30
+    lp = -torch.randint(0, 3, (L, K), generator=g).to(torch.float32).numpy()
+    lp = -np.sort(-lp, axis=1)          # ranks sorted best-first like a top-K table
+    ids = np.arange(L * K, dtype=np.int32).reshape(L, K)
+    t = oracle.build_tree(ids, lp, 0, B)
+    assert t.tuples[1:] == oracle.bruteforce_top_prefixes(lp, B)
+
+
+def test_budget_larger_than_tree_space():
+    lp = np.log(np.array([[0.5, 0.3], [0.6, 0.2]], dtype=np.float64)).astype(np.float32)
+    ids = np.array([[5, 6], [7, 8]], dtype=np.int32)
+    t = oracle.build_tree(ids, lp, 9, 100)
+    assert t.n_nodes == 1 + 2 + 4
+    assert np.all(t.parent[t.n_nodes:] == -1)
+    assert np.all(t.anc[t.n_nodes:] == 0)
+
+
+def test_prop1_expected_acceptance_config1():
+    w, z, ids, lp32, lse32, lp64 = _cfg1()
+    t = oracle.build_tree(ids[0], lp32[0], 0, w.B)
+    lp64_topk = np.take_along_axis(lp64[0], ids[0].astype(np.int64), axis=-1)
+    p_topk = np.exp(lp64_topk)
+    lhs = oracle.expected_acceptance_enumerated(t, p_topk)
+    rhs = oracle.surrogate_value(t.tuples, lp64_topk)
+    assert abs(lhs - rhs) < 1e-9
+
+
+def test_beam_and_chain_never_beat_heap():
+    w, z, ids, lp32, lse32, lp64 = _cfg1()
+    lp64_topk = np.take_along_axis(lp64[0], ids[0].astype(np.int64), axis=-1)
+    heap = oracle.build_tree(ids[0], lp32[0], 0, w.B)
+    v_heap = oracle.surrogate_value(heap.tuples, lp64_topk)
+    for width in (1, 2, 3, 4):
+        beam = oracle.beam_tree(lp32[0], width)
+        assert len(beam) <= w.B
+        assert oracle.surrogate_value(beam, lp64_topk) <= v_heap + 1e-15
+    chain = oracle.chain_tree(w.L)
+    assert oracle.surrogate_value(chain, lp64_topk) <= v_heap + 1e-15
+
+
+def test_lemma1_topk_min_b_v_suffices():
+    g = torch.Generator().manual_seed(3)
+    V, L = 9, 3
+    z = (torch.randn(L, V, generator=g, dtype=torch.float64) * 2).numpy()
+    for B in (2, 5, 8):
+        K = min(B, V)
+        ids_k, lp_k, *_ = oracle.topk(z, K)
+        ids_v, lp_v, *_ = oracle.topk(z, V)
+        tk = oracle.build_tree(ids_k, lp_k, 0, B)
+        tv = oracle.build_tree(ids_v, lp_v, 0, B)
+        assert tk.tuples == tv.tuples
+        assert np.array_equal(tk.node_token, tv.node_token)
+
+
+# ---------------------------------------------------------------- pages' examples
+
+def test_worked_example_deep_dive():
+    gold = _golden("worked_marginals_deep_dive.json")
+    p = gold["position1"]
+    toks = list(p)
+    probs = np.array([p[t] for t in toks] + [1.0 - sum(p.values())])
+    lp = np.log(probs)[None, :].astype(np.float32)          # L = 1
+    ids = np.arange(probs.size, dtype=np.int32)[None, :]
+    lp64 = np.log(probs)[None, :]
+    greedy = oracle.build_tree(ids, lp, -1, 1)
+    assert toks[greedy.node_token[1]] == gold["greedy_token"]
+    three = oracle.build_tree(ids, lp, -1, 3)
+    v1 = oracle.surrogate_value(greedy.tuples, lp64)
+    v3 = oracle.surrogate_value(three.tuples, lp64)
+    assert abs((v3 - v1) - gold["discarded_by_greedy"]) < 1e-6
+    assert sorted(toks[i] for i in three.node_token[1:4]) == sorted(toks)
+
+
+def test_example_marginals_llm_wiki_products():
+    gold = _golden("example_marginals_llm_wiki.json")
+    pos = gold["positions"]
+    names = [list(d) for d in pos]
+    probs = [np.array(list(d.values())) for d in pos]
+    K = max(len(p) for p in probs)
+    lp64 = np.full((2, K), -np.inf)
+    for d in range(2):
+        lp64[d, :len(probs[d])] = np.log(probs[d])
+    # expected order from plain products, enumerated directly
+    prods = []
+    for d in (1, 2):
+        for tup in itertools.product(*[range(len(probs[i])) for i in range(d)]):
+            prods.append((-math.prod(probs[i][r] for i, r in enumerate(tup)), tup))
+    prods.sort()
+    for B in range(1, len(prods) + 1):
+        t = oracle.build_tree(np.zeros((2, K), np.int32), lp64.astype(np.float32), 0, B)
+        assert t.tuples[1:] == [tup for _, tup in prods[:B]]
+    t = oracle.build_tree(np.zeros((2, K), np.int32), lp64.astype(np.float32), 0, 4)
+    got = [names[len(u) - 1][u[-1]] for u in t.tuples[1:]]
+    assert got == ["token_a", "token_b", "token_c", "token_x"]
+
+
+def test_hand_tree_mask_block_diffusion_drafters():
+    gold = _golden("hand_tree_block_diffusion_drafters.json")
+    names = gold["nodes"]
+    idx = {n: i for i, n in enumerate(names)}
+    parent = np.array([-1] + [idx[gold["parent"][n]] for n in names[1:]], dtype=np.int32)
+    anc = oracle.ancestor_mask(parent, len(names), len(names))
+    row = int(anc[idx["D"], 0])
+    seen = {n for n in names if (row >> idx[n]) & 1}
+    assert seen == set(gold["attends"]["D"])
+    assert not seen & set(gold["not_attends"]["D"])
+
+
+def _walk_mask(parent, n_nodes, n):
+    W = (n + 31) // 32
+    m = np.zeros((n, W), np.uint32)
+    for i in range(n_nodes):
+        j = i
+        while j >= 0:
+            m[i, j // 32] |= np.uint32(1 << (j % 32))
+            j = int(parent[j])
+    return m
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_mask_equals_explicit_parent_walks(seed):
+    g = torch.Generator().manual_seed(seed)
+    L, V, B = 6, 40, 70
+    z = (torch.randn(L, V, generator=g, dtype=torch.float64) * (1 + seed)).numpy()
+    ids, lp32, *_ = oracle.topk(z, min(B, V))
+    t = oracle.build_tree(ids, lp32, 1, B)
+    assert np.array_equal(t.anc, _walk_mask(t.parent, t.n_nodes, B + 1))
+
+
+# ---------------------------------------------------------------- attention
+
+def _random_case(seed, N=2, layers=2, Hq=4, Hkv=2, D=16, L=4, V=30, B=9, paged=False):
+    g = torch.Generator().manual_seed(seed)
+    trees = []
+    for r in range(N):
+        z = (torch.randn(L, V, generator=g, dtype=torch.float64) * 2).numpy()
+        ids, lp32, *_ = oracle.topk(z, min(B, V))
+        trees.append(oracle.build_tree(ids, lp32, 0, B))
+    st = oracle.stack_trees(trees)
+    n = B + 1
+    P = torch.randint(3, 12, (N,), generator=g).numpy().astype(np.int32)
+    S = int(P.max()) + n
+    q = torch.randn(layers, N, n, Hq, D, generator=g, dtype=torch.float64).numpy()
+    k = torch.randn(layers, N, S, Hkv, D, generator=g, dtype=torch.float64).numpy()
+    v = torch.randn(layers, N, S, Hkv, D, generator=g, dtype=torch.float64).numpy()
+    return st, P, q, k, v
+
+
+def _sdpa_reference(q, k, v, P, parent, n_nodes, scale, l, r):
+    """torch SDPA (float64) with the boolean mask from explicit parent walks."""
+    nn = int(n_nodes[r])
+    Hq, Hkv = q.shape[3], k.shape[3]
+    Pr = int(P[r])
+    mask = torch.zeros(nn, Pr + nn, dtype=torch.bool)
+    mask[:, :Pr] = True
+    for i in range(nn):
+        j = i
+        while j >= 0:
+            mask[i, Pr + j] = True
+            j = int(parent[r, j])
+    qq = torch.from_numpy(q[l, r, :nn]).permute(1, 0, 2)                 # [Hq, nn, D]
+    kk = torch.from_numpy(k[l, r, :Pr + nn]).permute(1, 0, 2)
+    vv = torch.from_numpy(v[l, r, :Pr + nn]).permute(1, 0, 2)
+    kk = kk.repeat_interleave(Hq // Hkv, dim=0)
+    vv = vv.repeat_interleave(Hq // Hkv, dim=0)
+    o = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=mask, scale=scale)
+    return o.permute(1, 0, 2).numpy()                                     # [nn, Hq, D]
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_attention_equals_sdpa_with_mask(seed):
+    st, P, q, k, v = _random_case(seed)
+    scale = 1 / math.sqrt(q.shape[-1])
+    out, _ = oracle.tree_attention(q, k, v, P, st["anc"], st["n_nodes"], scale)
+    for l in range(q.shape[0]):
+        for r in range(q.shape[1]):
+            ref = _sdpa_reference(q, k, v, P, st["parent"], st["n_nodes"], scale, l, r)
+            for i in range(int(st["n_nodes"][r])):
+                for h in range(q.shape[3]):
+                    assert np.max(np.abs(out[(l, r, i, h)] - ref[i, h])) < 1e-12
+
+
+def test_attention_paged_equals_contiguous():
+    st, P, q, k, v = _random_case(11)
+    layers, N, S, Hkv, D = k.shape
+    page = oracle.PAGE
+    nb = (S + page - 1) // page
+    perm = np.random.RandomState(0).permutation(N * nb)
+    table = perm.reshape(N, nb).astype(np.int32)
+    kp = np.zeros((layers, N * nb, page, Hkv, D))
+    vp = np.zeros_like(kp)
+    for r in range(N):
+        for s in range(S):
+            kp[:, table[r, s // page], s % page] = k[:, r, s]
+            vp[:, table[r, s // page], s % page] = v[:, r, s]
+    scale = 0.3
+    a, _ = oracle.tree_attention(q, k, v, P, st["anc"], st["n_nodes"], scale)
+    b, _ = oracle.tree_attention(q, kp, vp, P, st["anc"], st["n_nodes"], scale, block_table=table)
+    for key in a:
+        assert np.array_equal(a[key], b[key])
+
+
+def test_attention_chain_is_causal():
+    # chain tree: node i's ancestors are 0..i, so the tree part is causal
+    n, P, H, D = 7, 5, 2, 8
+    g = torch.Generator().manual_seed(5)
+    parent = np.arange(-1, n - 1, dtype=np.int32)
+    anc = oracle.ancestor_mask(parent, n, n)[None]
+    q = torch.randn(1, 1, n, H, D, generator=g, dtype=torch.float64)
+    k = torch.randn(1, 1, P + n, H, D, generator=g, dtype=torch.float64)
+    v = torch.randn(1, 1, P + n, H, D, generator=g, dtype=torch.float64)
+    out, _ = oracle.tree_attention(q.numpy(), k.numpy(), v.numpy(), np.array([P]), anc,
+                                   np.array([n]), 0.5)
+    # causal SDPA over the P+n sequence; the tree queries are its last n rows
+    qs = torch.cat([torch.zeros(1, 1, P, H, D, dtype=torch.float64), q], dim=2)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qs[0, 0].permute(1, 0, 2), k[0, 0].permute(1, 0, 2), v[0, 0].permute(1, 0, 2),
+        is_causal=True, scale=0.5).permute(1, 0, 2)[P:]
+    for i in range(n):
+        for h in range(H):
+            assert np.max(np.abs(out[(0, 0, i, h)] - ref[i, h].numpy())) < 1e-12
+
+
+def test_attention_budget_zero_is_decode():
+    P, H, D = 9, 3, 8
+    g = torch.Generator().manual_seed(9)
+    q = torch.randn(1, 1, 1, H, D, generator=g, dtype=torch.float64)
+    k = torch.randn(1, 1, P + 1, H, D, generator=g, dtype=torch.float64)
+    v = torch.randn(1, 1, P + 1, H, D, generator=g, dtype=torch.float64)
+    anc = np.ones((1, 1, 1), np.uint32)
+    out, _ = oracle.tree_attention(q.numpy(), k.numpy(), v.numpy(), np.array([P]), anc,
+                                   np.array([1]), 0.25)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q[0, 0].permute(1, 0, 2), k[0, 0].permute(1, 0, 2), v[0, 0].permute(1, 0, 2),
+        scale=0.25).permute(1, 0, 2)
+    for h in range(H):
+        assert np.max(np.abs(out[(0, 0, 0, h)] - ref[0, h].numpy())) < 1e-12
+
+
+def test_attention_uniform_keys_reveal_visible_set():
+    # With all keys equal the softmax is uniform over the visible slots, so
+    # one-hot values read the visible set back exactly.
+    st, P, q, _, _ = _random_case(21, N=1, layers=1, Hq=2, Hkv=1, D=4, B=12)
+    n = 13
+    S = int(P[0]) + n
+    k = np.zeros((1, 1, S, 1, 4))
+    v = np.zeros((1, 1, S, 1, S))
+    v[0, 0, np.arange(S), 0, np.arange(S)] = 1.0
+    q2 = np.zeros((1, 1, n, 2, S))
+    out, _ = oracle.tree_attention(q2, np.concatenate([k, np.zeros((1, 1, S, 1, S - 4))], -1),
+                                   v, P, st["anc"], st["n_nodes"], 1.0)
+    walk = _walk_mask(st["parent"][0], int(st["n_nodes"][0]), n)
+    for i in range(int(st["n_nodes"][0])):
+        vis = [j for j in range(n) if (int(walk[i, j // 32]) >> (j % 32)) & 1]
+        expect = np.zeros(S)
+        expect[:P[0]] = 1.0
+        expect[P[0] + np.array(vis)] = 1.0
+        expect /= expect.sum()
+        assert np.max(np.abs(out[(0, 0, i, 0)] - expect)) < 1e-15
+
+
+# ---------------------------------------------------------------- walk + compaction
+
+def _deepest_consistent(t_arg, parent, node_token, n_nodes):
+    """Brute force: the deepest node whose every edge matches the argmax above it."""
+    best, best_depth = 0, 0
+    for i in range(1, n_nodes):
+        j, ok, d = i, True, 0
+        while j > 0:
+            p = int(parent[j])
+            if node_token[j] != t_arg[p]:
+                ok = False
+                break
+            j, d = p, d + 1
+        if ok and d > best_depth:
+            best, best_depth = i, d
+    return best, best_depth
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_accept_equals_deepest_consistent_node(seed):
+    g = torch.Generator().manual_seed(40 + seed)
+    L, V, B = 5, 12, 25
+    z = (torch.randn(L, V, generator=g, dtype=torch.float64) * 1.5).numpy()
+    ids, lp32, *_ = oracle.topk(z, min(B, V))
+    t = oracle.build_tree(ids, lp32, 3, B)
+    n = B + 1
+    target = torch.randn(n, V, generator=g, dtype=torch.float64).numpy()
+    # plant matches along a random branch so long walks happen
+    for i in range(1, t.n_nodes):
+        if torch.rand(1, generator=g).item() < 0.5:
+            target[t.parent[i], t.node_token[i]] = 10.0 + torch.rand(1, generator=g).item()
+    acc = oracle.accept(target, t.node_token, t.parent, t.n_nodes, L, 100)
+    tgt = np.argmax(target, axis=-1)
+    last, depth = _deepest_consistent(tgt, t.parent, t.node_token, t.n_nodes)
+    assert acc.accept_len == depth + 1
+    assert acc.path[acc.accept_len - 1] == last
+    assert acc.next_bonus == tgt[last]
+    # the path is the ancestor chain of the last node
+    chain = []
+    j = last
+    while j >= 0:
+        chain.append(j)
+        j = int(t.parent[j])
+    assert acc.path[:acc.accept_len].tolist() == chain[::-1]
+    assert acc.new_prefix_len == 100 + acc.accept_len
+    assert acc.src_slot[:acc.accept_len].tolist() == [100 + j for j in chain[::-1]]
+
+
+def test_accept_k1_chain_is_single_line():
+    # K = 1, B = L: the tree is the single drafted line; acceptance is the
+    # number of leading positions where the target argmax equals the draft.
+    L, V = 6, 10
+    g = torch.Generator().manual_seed(77)
+    z = torch.randn(L, V, generator=g, dtype=torch.float64).numpy()
+    ids, lp32, *_ = oracle.topk(z, 1)
+    t = oracle.build_tree(ids, lp32, 4, L)
+    assert list(t.parent[1:]) == list(range(L))
+    draft = ids[:, 0]
+    for n_match in range(L + 1):
+        target = np.zeros((L + 1, V))
+        for i in range(L + 1):
+            target[i, (draft[i] + 1) % V if i < L else 0] = 1.0
+        for i in range(n_match):
+            target[i] = 0.0
+            target[i, draft[i]] = 1.0
+        acc = oracle.accept(target, t.node_token, t.parent, t.n_nodes, L, 0)
+        lead = 0
+        while lead < L and np.argmax(target[lead]) == draft[lead]:
+            lead += 1
+        assert acc.accept_len == lead + 1 == n_match + 1
+
+
+def test_argmax_lowest_id_on_ties():
+    x = np.array([[1.0, 3.0, 3.0, -1.0], [-0.0, 0.0, -1.0, 0.0]])
+    assert oracle.argmax_rows(x).tolist() == [1, 0]
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_compaction_equals_index_select(paged):
+    g = torch.Generator().manual_seed(8)
+    layers, N, S, Hkv, D = 2, 2, 40, 2, 4
+    k = torch.randn(layers, N, S, Hkv, D, generator=g, dtype=torch.float64).numpy()
+    v = torch.randn(layers, N, S, Hkv, D, generator=g, dtype=torch.float64).numpy()
+    P = 7
+    path = np.array([0, 2, 5, 9, 10, -1, -1], dtype=np.int32)
+    acc = oracle.Acceptance(path, 5, 0, np.where(path >= 0, P + path, -1).astype(np.int32),
+                            np.where(path >= 0, P + np.arange(7), -1).astype(np.int32),
+                            P + 5, np.zeros(1, np.int32))
+    src = torch.tensor([P + j for j in path[:5]])
+    if not paged:
+        k0, v0 = k.copy(), v.copy()
+        oracle.compact(k, v, 1, acc)
+        for c, c0 in ((k, k0), (v, v0)):
+            expect = torch.index_select(torch.from_numpy(c0[:, 1]), 1, src).numpy()
+            assert np.array_equal(c[:, 1, P:P + 5], expect)
+            assert np.array_equal(c[:, 1, :P], c0[:, 1, :P])
+            assert np.array_equal(c[:, 1, P + 5:], c0[:, 1, P + 5:])
+            assert np.array_equal(c[:, 0], c0[:, 0])
+    else:
+        page = oracle.PAGE
+        table = np.array([[1, 0], [3, 2]], dtype=np.int32)   # one page per request is enough here
+        kp = torch.randn(layers, 4, page, Hkv, D, generator=g, dtype=torch.float64).numpy()
+        vp = torch.randn(layers, 4, page, Hkv, D, generator=g, dtype=torch.float64).numpy()
+        k0 = kp.copy()
+        oracle.compact(kp, vp, 1, acc, block_table=table)
+        logical = k0[:, table[1, 0]]                 # slots 0..63 of request 1
+        expect = torch.index_select(torch.from_numpy(logical), 1, src).numpy()
+        assert np.array_equal(kp[:, table[1, 0], P:P + 5], expect)
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+def test_pins_catch_a_dropped_sibling_push():
+    """A heap that never pushes siblings must fail the brute-force pin.
+
+    Feeding the heap a one-column table is exactly a heap without sibling
+    pushes: every popped entry then has only its child to push.
+    """
+    w, z, ids, lp32, *_ = _cfg1()
+    t = oracle.build_tree(ids[0][:, :1], lp32[0][:, :1], 0, w.B)
+    assert t.tuples[1:] != oracle.bruteforce_top_prefixes(lp32[0], w.B)
+
+
+def test_pins_catch_a_wrong_scale_in_attention():
+    st, P, q, k, v = _random_case(2)
+    scale = 1 / math.sqrt(q.shape[-1])
+    out, _ = oracle.tree_attention(q, k, v, P, st["anc"], st["n_nodes"], scale * 1.01)
+    ref = _sdpa_reference(q, k, v, P, st["parent"], st["n_nodes"], scale, 0, 0)
+    assert np.max(np.abs(out[(0, 0, 1, 0)] - ref[1, 0])) > 1e-6

@@ -1,0 +1,81 @@
+// Shared device helpers of the DDTree round library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ddtree.h"
+
+namespace ddt {
+
+// Device status word read by ddtree_device_status(); bits DDTREE_STATUS_*.
+__device__ unsigned int g_status;
+
+__device__ __forceinline__ void flag_status(unsigned int bits) { atomicOr(&g_status, bits); }
+
+// ---------------------------------------------------------------------------
+// Order-preserving integer keys: a > b as reals  <=>  key(a) > key(b).
+// -0.0 maps to the key of +0.0; -inf is the smallest key of a real value.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t key16_of_bf16(uint16_t bits) {
+  if (bits == 0x8000u) bits = 0;                       // -0.0 -> +0.0
+  return (bits & 0x8000u) ? (uint32_t)(~bits & 0xFFFFu) : (uint32_t)(bits | 0x8000u);
+}
+__device__ __forceinline__ float bf16_of_key16(uint32_t key) {
+  uint16_t bits = (key & 0x8000u) ? (uint16_t)(key & 0x7FFFu) : (uint16_t)(~key & 0xFFFFu);
+  return __uint_as_float(((uint32_t)bits) << 16);
+}
+__device__ __forceinline__ uint32_t key32_of_f32(float x) {
+  uint32_t bits = __float_as_uint(x);
+  if (bits == 0x80000000u) bits = 0;                   // -0.0 -> +0.0
+  return (bits & 0x80000000u) ? ~bits : (bits | 0x80000000u);
+}
+__device__ __forceinline__ float f32_of_key32(uint32_t key) {
+  uint32_t bits = (key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key;
+  return __uint_as_float(bits);
+}
+__device__ __forceinline__ bool bf16_is_nan(uint16_t bits) {
+  return (bits & 0x7F80u) == 0x7F80u && (bits & 0x007Fu) != 0;
+}
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t bits) {
+  return __uint_as_float(((uint32_t)bits) << 16);
+}
+
+// 16-byte read-only global load that does not allocate in L1 (streamed once).
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// Word k (0..3) of a 16-byte vector; k is a compile-time constant after
+// unrolling, so this is a register select, not a memory access.
+__device__ __forceinline__ uint32_t u32_at(const uint4& v, int k) {
+  return k == 0 ? v.x : (k == 1 ? v.y : (k == 2 ? v.z : v.w));
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = w > v ? w : v;
+  }
+  return v;
+}
+
+inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+}  // namespace ddt

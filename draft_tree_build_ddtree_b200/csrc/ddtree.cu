@@ -1,0 +1,413 @@
+// libddtree.so: the C ABI of include/ddtree.h.
+//
+// One translation unit: the kernels of every stage are included here so the
+// device status word is a single symbol without relocatable device code.
+// Host code validates every argument before launching anything; kernels
+// never trap, assert or wait on another CTA.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "ddtree.h"
+#include "common.cuh"
+#include "topk.cuh"
+#include "build.cuh"
+#include "accept.cuh"
+#include "attn_simt.cuh"
+#include "attn_tc.cuh"
+
+using namespace ddt;
+
+namespace {
+
+constexpr int MAX_L = 32;
+constexpr int MAX_K = 1024;
+constexpr int MAX_B = 1024;
+constexpr int MAX_REQ = 4096;
+constexpr int MAX_V = 1 << TOPK_ID_BITS;
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+int max_smem_optin() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  return n > 0 ? n : 227 * 1024;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int esize_of(int dtype) { return dtype == DDTREE_BF16 ? 2 : 4; }
+
+bool dtype_ok(int dtype) { return dtype == DDTREE_BF16 || dtype == DDTREE_F32; }
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DDTREE_OK : DDTREE_ERR_CUDA;
+}
+
+template <typename F>
+int set_smem(F* kernel, size_t bytes) {
+  if (bytes > (size_t)max_smem_optin()) return DDTREE_ERR_UNSUPPORTED;
+  if (bytes > 48 * 1024) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+      return DDTREE_ERR_CUDA;
+  }
+  return DDTREE_OK;
+}
+
+// ------------------------------------------------------------------ topk
+int topk_check(const void* logits, int dtype, int rows, int V, long long row_stride, int K,
+               const void* ids, const void* lp) {
+  if (!logits || !ids || !lp) return DDTREE_ERR_INVALID_ARG;
+  if (!dtype_ok(dtype)) return DDTREE_ERR_INVALID_ARG;
+  if (rows < 1 || V < 1 || V > MAX_V || K < 1 || K > MAX_K || K > V) return DDTREE_ERR_INVALID_ARG;
+  if (row_stride < V || (row_stride * esize_of(dtype)) % 16 != 0) return DDTREE_ERR_INVALID_ARG;
+  if (!aligned16(logits)) return DDTREE_ERR_INVALID_ARG;
+  return DDTREE_OK;
+}
+
+size_t topk_ws(int rows, int V, int K, int dtype) {
+  TopkPlan p = topk_plan(rows, V, K, esize_of(dtype), num_sms());
+  return topk_ws_bytes(rows, p);
+}
+
+int topk_launch(const void* logits, int dtype, int rows, int V, long long row_stride, int K,
+                int32_t* ids, float* lp, float* lse, void* ws, size_t ws_bytes, cudaStream_t s) {
+  int st = topk_check(logits, dtype, rows, V, row_stride, K, ids, lp);
+  if (st) return st;
+  TopkPlan p = topk_plan(rows, V, K, esize_of(dtype), num_sms());
+  if (p.cand > TOPK_MAX_CAND) return DDTREE_ERR_UNSUPPORTED;
+  if (!ws || !aligned16(ws) || ws_bytes < topk_ws_bytes(rows, p)) return DDTREE_ERR_INVALID_ARG;
+  TopkWs w = topk_ws_carve(ws, rows, p);
+  const size_t smem = topk_smem_bytes(p, K);
+  const long long grid = (long long)rows * p.cpr;
+  if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
+  if (dtype == DDTREE_BF16) {
+    if ((st = set_smem(topk_kernel<DDTREE_BF16>, smem))) return st;
+    topk_kernel<DDTREE_BF16><<<(unsigned)grid, TOPK_THREADS, smem, s>>>(logits, rows, V, row_stride, K, p, w,
+                                                                       ids, lp, lse);
+  } else {
+    if ((st = set_smem(topk_kernel<DDTREE_F32>, smem))) return st;
+    topk_kernel<DDTREE_F32><<<(unsigned)grid, TOPK_THREADS, smem, s>>>(logits, rows, V, row_stride, K, p, w,
+                                                                      ids, lp, lse);
+  }
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ build
+int build_launch(const int32_t* ids, const float* lp, const int32_t* root_token, int n_req, int L, int K,
+                 int B, int32_t* node_token, int32_t* parent, int32_t* depth, int32_t* node_rank,
+                 float* score, uint32_t* anc, int32_t* n_nodes, cudaStream_t s) {
+  if (!ids || !lp || !root_token || !parent || !anc || !n_nodes) return DDTREE_ERR_INVALID_ARG;
+  if (n_req < 1 || n_req > MAX_REQ || L < 1 || L > MAX_L || K < 1 || K > MAX_K || B < 0 || B > MAX_B)
+    return DDTREE_ERR_INVALID_ARG;
+  const int kc = B < K ? B : K;
+  const size_t smem = build_smem_bytes(L, kc, B);
+  int st = set_smem(build_kernel, smem);
+  if (st) return st;
+  build_kernel<<<n_req, BUILD_THREADS, smem, s>>>(ids, lp, root_token, L, K, B, kc, node_token, parent, depth,
+                                                   node_rank, score, anc, n_nodes);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ attention
+int kv_check(const ddtree_kv_desc* kv) {
+  if (!kv) return DDTREE_ERR_INVALID_ARG;
+  if (kv->layers < 1 || kv->n_req < 1 || kv->n_req > MAX_REQ || kv->Hq < 1 || kv->Hkv < 1 ||
+      kv->Hq % kv->Hkv != 0)
+    return DDTREE_ERR_INVALID_ARG;
+  if (kv->D != 64 && kv->D != 128) return DDTREE_ERR_UNSUPPORTED;
+  if (kv->paged) {
+    if (kv->num_blocks < 1 || kv->max_blocks < 1) return DDTREE_ERR_INVALID_ARG;
+  } else if (kv->s_max < 1) {
+    return DDTREE_ERR_INVALID_ARG;
+  }
+  return DDTREE_OK;
+}
+
+AttnGeom geom_of(const ddtree_kv_desc* kv, int B) {
+  AttnGeom g;
+  g.layers = kv->layers;
+  g.n_req = kv->n_req;
+  g.n = B + 1;
+  g.Hq = kv->Hq;
+  g.Hkv = kv->Hkv;
+  g.D = kv->D;
+  g.W = (B + 1 + 31) / 32;
+  g.scale = kv->scale > 0.f ? kv->scale : 1.0f / sqrtf((float)kv->D);
+  g.paged = kv->paged;
+  g.s_max = kv->s_max;
+  g.num_blocks = kv->num_blocks;
+  g.max_blocks = kv->max_blocks;
+  return g;
+}
+
+bool use_tc_attn(int dtype, const ddtree_kv_desc* kv) {
+  return dtype == DDTREE_BF16 && kv->D == 128 && tc_attn_supported(kv->Hq / kv->Hkv);
+}
+
+size_t attn_ws(const ddtree_kv_desc* kv, int B, int dtype) {
+  if (!use_tc_attn(dtype, kv)) return 0;
+  return tc_attn_ws_bytes(geom_of(kv, B), num_sms());
+}
+
+int attn_launch(const void* q, const void* k_cache, const void* v_cache, int dtype, const ddtree_kv_desc* kv,
+                const int32_t* block_table, const int32_t* prefix_len, const uint32_t* anc,
+                const int32_t* n_nodes, int B, void* out, float* out_lse, void* ws, size_t ws_bytes,
+                cudaStream_t s) {
+  int st = kv_check(kv);
+  if (st) return st;
+  if (!dtype_ok(dtype) || B < 0 || B > MAX_B) return DDTREE_ERR_INVALID_ARG;
+  if (!q || !k_cache || !v_cache || !prefix_len || !anc || !n_nodes || !out) return DDTREE_ERR_INVALID_ARG;
+  if (kv->paged && !block_table) return DDTREE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return DDTREE_ERR_INVALID_ARG;
+  AttnGeom g = geom_of(kv, B);
+  if (use_tc_attn(dtype, kv)) {
+    const size_t need = tc_attn_ws_bytes(g, num_sms());
+    if (need && (!ws || !aligned16(ws) || ws_bytes < need)) return DDTREE_ERR_INVALID_ARG;
+    return tc_attn_launch(q, k_cache, v_cache, block_table, prefix_len, anc, n_nodes, g, out, out_lse, ws,
+                          num_sms(), s);
+  }
+  const long long grid =
+      (long long)g.layers * g.n_req * g.n * ((g.Hq + ATTN_SIMT_WARPS - 1) / ATTN_SIMT_WARPS);
+  if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
+  const dim3 blk(ATTN_SIMT_WARPS * 32);
+  if (dtype == DDTREE_BF16) {
+    typedef __nv_bfloat16 T;
+    if (g.D == 64)
+      tree_attn_simt_kernel<T, 64><<<(unsigned)grid, blk, 0, s>>>((const T*)q, (const T*)k_cache,
+                                                                  (const T*)v_cache, block_table, prefix_len,
+                                                                  anc, n_nodes, g, (T*)out, out_lse);
+    else
+      tree_attn_simt_kernel<T, 128><<<(unsigned)grid, blk, 0, s>>>((const T*)q, (const T*)k_cache,
+                                                                   (const T*)v_cache, block_table, prefix_len,
+                                                                   anc, n_nodes, g, (T*)out, out_lse);
+  } else {
+    typedef float T;
+    if (g.D == 64)
+      tree_attn_simt_kernel<T, 64><<<(unsigned)grid, blk, 0, s>>>((const T*)q, (const T*)k_cache,
+                                                                  (const T*)v_cache, block_table, prefix_len,
+                                                                  anc, n_nodes, g, (T*)out, out_lse);
+    else
+      tree_attn_simt_kernel<T, 128><<<(unsigned)grid, blk, 0, s>>>((const T*)q, (const T*)k_cache,
+                                                                   (const T*)v_cache, block_table, prefix_len,
+                                                                   anc, n_nodes, g, (T*)out, out_lse);
+  }
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ accept
+struct AcceptPlan {
+  int cpr, chunk;
+};
+
+AcceptPlan accept_plan(int rows, int V, int esize) {
+  const int epv = 16 / esize;
+  const int max_chunk = ARGMAX_THREADS * TOPK_MAX_VPT * epv;
+  int cpr_min = ceil_div(V, max_chunk);
+  int cpr_fill = num_sms() * 2 / (rows > 0 ? rows : 1);
+  int cpr_small = ceil_div(V, 4096);
+  int cpr = cpr_fill < cpr_small ? cpr_fill : cpr_small;
+  if (cpr < cpr_min) cpr = cpr_min;
+  if (cpr < 1) cpr = 1;
+  AcceptPlan p;
+  p.chunk = ceil_div(ceil_div(V, cpr), epv) * epv;
+  p.cpr = ceil_div(V, p.chunk);
+  return p;
+}
+
+size_t accept_ws(int n_req, int B) { return argmax_ws_bytes(n_req * (B + 1)); }
+
+int accept_launch(const void* target_logits, int dtype, int V, long long row_stride, const int32_t* node_token,
+                  const int32_t* parent, const int32_t* n_nodes, int n_req, int L, int B,
+                  const int32_t* prefix_len, int32_t* new_prefix_len, void* k_cache, void* v_cache,
+                  const ddtree_kv_desc* kv, const int32_t* block_table, int32_t* target_argmax, int32_t* path,
+                  int32_t* accept_len, int32_t* next_bonus, int32_t* src_slot, int32_t* dst_slot, void* ws,
+                  size_t ws_bytes, cudaStream_t s) {
+  if (!target_logits || !node_token || !parent || !n_nodes || !prefix_len || !new_prefix_len)
+    return DDTREE_ERR_INVALID_ARG;
+  if (new_prefix_len == prefix_len) return DDTREE_ERR_INVALID_ARG;
+  if (!dtype_ok(dtype) || V < 1 || V > MAX_V || n_req < 1 || n_req > MAX_REQ || L < 1 || L > MAX_L || B < 0 ||
+      B > MAX_B)
+    return DDTREE_ERR_INVALID_ARG;
+  if (row_stride < V || (row_stride * esize_of(dtype)) % 16 != 0 || !aligned16(target_logits))
+    return DDTREE_ERR_INVALID_ARG;
+  const int n = B + 1;
+  const int rows = n_req * n;
+  if (!ws || !aligned16(ws) || ws_bytes < argmax_ws_bytes(rows)) return DDTREE_ERR_INVALID_ARG;
+  int row_bytes = 0;
+  if (k_cache) {
+    int st = kv_check(kv);
+    if (st) return st;
+    if (!v_cache || kv->n_req != n_req || (kv->paged && !block_table)) return DDTREE_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache)) return DDTREE_ERR_INVALID_ARG;
+    row_bytes = kv->Hkv * kv->D * esize_of(dtype);
+    if (row_bytes % 16 != 0) return DDTREE_ERR_UNSUPPORTED;
+  }
+  AcceptPlan p = accept_plan(rows, V, esize_of(dtype));
+  ArgmaxWs w = argmax_ws_carve(ws, rows);
+  const long long grid = (long long)rows * p.cpr;
+  if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
+  if (dtype == DDTREE_BF16)
+    argmax_kernel<DDTREE_BF16><<<(unsigned)grid, ARGMAX_THREADS, 0, s>>>(target_logits, n, V, row_stride,
+                                                                        n_nodes, p.cpr, p.chunk, w);
+  else
+    argmax_kernel<DDTREE_F32><<<(unsigned)grid, ARGMAX_THREADS, 0, s>>>(target_logits, n, V, row_stride,
+                                                                       n_nodes, p.cpr, p.chunk, w);
+  int st = launch_status();
+  if (st) return st;
+  WalkArgs a;
+  a.node_token = node_token;
+  a.parent = parent;
+  a.n_nodes = n_nodes;
+  a.prefix_len = prefix_len;
+  a.argmax_ws = w.argmax;
+  a.n = n;
+  a.L = L;
+  a.new_prefix_len = new_prefix_len;
+  a.target_argmax = target_argmax;
+  a.path = path;
+  a.accept_len = accept_len;
+  a.next_bonus = next_bonus;
+  a.src_slot = src_slot;
+  a.dst_slot = dst_slot;
+  a.k_cache = (unsigned char*)k_cache;
+  a.v_cache = (unsigned char*)v_cache;
+  a.block_table = block_table;
+  a.layers = k_cache ? kv->layers : 1;
+  a.n_req = n_req;
+  a.paged = k_cache ? kv->paged : 0;
+  a.s_max = k_cache ? kv->s_max : 0;
+  a.num_blocks = k_cache ? kv->num_blocks : 0;
+  a.max_blocks = k_cache ? kv->max_blocks : 0;
+  a.row_bytes = row_bytes;
+  const size_t smem = (size_t)n * 8;
+  dim3 grid2(n_req, a.layers * 2);
+  walk_compact_kernel<<<grid2, WALK_THREADS, smem, s>>>(a);
+  return launch_status();
+}
+
+}  // namespace
+
+// ======================================================================
+// C ABI
+// ======================================================================
+extern "C" {
+
+size_t ddtree_topk_workspace_bytes(int rows, int V, int K) {
+  if (rows < 1 || V < 1 || K < 1) return 0;
+  size_t a = topk_ws(rows, V, K, DDTREE_BF16), b = topk_ws(rows, V, K, DDTREE_F32);
+  return a > b ? a : b;
+}
+
+int ddtree_topk(const void* logits, int dtype, int rows, int V, long long row_stride, int K, int32_t* ids,
+                float* lp, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return topk_launch(logits, dtype, rows, V, row_stride, K, ids, lp, lse, ws, ws_bytes, stream);
+}
+
+int ddtree_build(const int32_t* ids, const float* lp, const int32_t* root_token, int n_req, int L, int K, int B,
+                 int32_t* node_token, int32_t* parent, int32_t* depth, int32_t* node_rank, float* score,
+                 uint32_t* anc, int32_t* n_nodes, cudaStream_t stream) {
+  return build_launch(ids, lp, root_token, n_req, L, K, B, node_token, parent, depth, node_rank, score, anc,
+                      n_nodes, stream);
+}
+
+size_t ddtree_attn_workspace_bytes(const ddtree_kv_desc* kv, int B) {
+  if (kv_check(kv) || B < 0 || B > MAX_B) return 0;
+  return attn_ws(kv, B, DDTREE_BF16);
+}
+
+int ddtree_tree_attn(const void* q, const void* k_cache, const void* v_cache, int dtype, const ddtree_kv_desc* kv,
+                     const int32_t* block_table, const int32_t* prefix_len, const uint32_t* anc,
+                     const int32_t* n_nodes, int B, void* out, float* out_lse, void* ws, size_t ws_bytes,
+                     cudaStream_t stream) {
+  return attn_launch(q, k_cache, v_cache, dtype, kv, block_table, prefix_len, anc, n_nodes, B, out, out_lse,
+                     ws, ws_bytes, stream);
+}
+
+size_t ddtree_accept_workspace_bytes(int n_req, int B, int V) {
+  (void)V;
+  if (n_req < 1 || B < 0) return 0;
+  return accept_ws(n_req, B);
+}
+
+int ddtree_accept(const void* target_logits, int dtype, int V, long long row_stride, const int32_t* node_token,
+                  const int32_t* parent, const int32_t* n_nodes, int n_req, int L, int B,
+                  const int32_t* prefix_len, int32_t* new_prefix_len, void* k_cache, void* v_cache,
+                  const ddtree_kv_desc* kv, const int32_t* block_table, int32_t* target_argmax, int32_t* path,
+                  int32_t* accept_len, int32_t* next_bonus, int32_t* src_slot, int32_t* dst_slot, void* ws,
+                  size_t ws_bytes, cudaStream_t stream) {
+  return accept_launch(target_logits, dtype, V, row_stride, node_token, parent, n_nodes, n_req, L, B,
+                       prefix_len, new_prefix_len, k_cache, v_cache, kv, block_table, target_argmax, path,
+                       accept_len, next_bonus, src_slot, dst_slot, ws, ws_bytes, stream);
+}
+
+static size_t round_parts(const ddtree_round_args* a, size_t* off_attn, size_t* off_acc) {
+  const size_t t = align256(topk_ws(a->n_req * a->L, a->V, a->K, a->dtype));
+  const size_t at = align256(attn_ws(&a->kv, a->B, a->dtype));
+  const size_t ac = align256(accept_ws(a->n_req, a->B));
+  if (off_attn) *off_attn = t;
+  if (off_acc) *off_acc = t + at;
+  return t + at + ac;
+}
+
+size_t ddtree_round_workspace_bytes(const ddtree_round_args* a) {
+  if (!a || a->n_req < 1 || a->L < 1 || a->V < 1 || a->K < 1 || a->B < 0 || kv_check(&a->kv)) return 0;
+  return round_parts(a, nullptr, nullptr);
+}
+
+int ddtree_round(const ddtree_round_args* a, cudaStream_t stream) {
+  if (!a) return DDTREE_ERR_INVALID_ARG;
+  if (kv_check(&a->kv)) return DDTREE_ERR_INVALID_ARG;
+  if (a->kv.n_req != a->n_req) return DDTREE_ERR_INVALID_ARG;
+  size_t off_attn = 0, off_acc = 0;
+  const size_t need = round_parts(a, &off_attn, &off_acc);
+  if (!a->ws || a->ws_bytes < need) return DDTREE_ERR_INVALID_ARG;
+  char* ws = (char*)a->ws;
+  int st = topk_launch(a->drafter_logits, a->dtype, a->n_req * a->L, a->V, a->drafter_stride, a->K, a->ids, a->lp,
+                       a->lse, ws, off_attn, stream);
+  if (st) return st;
+  st = build_launch(a->ids, a->lp, a->root_token, a->n_req, a->L, a->K, a->B, a->node_token, a->parent, a->depth,
+                    a->node_rank, a->score, a->anc, a->n_nodes, stream);
+  if (st) return st;
+  st = attn_launch(a->q, a->k_cache, a->v_cache, a->dtype, &a->kv, a->block_table, a->prefix_len, a->anc,
+                   a->n_nodes, a->B, a->attn_out, a->attn_lse, ws + off_attn, off_acc - off_attn, stream);
+  if (st) return st;
+  return accept_launch(a->target_logits, a->dtype, a->V, a->target_stride, a->node_token, a->parent, a->n_nodes,
+                       a->n_req, a->L, a->B, a->prefix_len, a->new_prefix_len, a->k_cache, a->v_cache, &a->kv,
+                       a->block_table, a->target_argmax, a->path, a->accept_len, a->next_bonus, a->src_slot,
+                       a->dst_slot, ws + off_acc, need - off_acc, stream);
+}
+
+const char* ddtree_status_string(int status) {
+  switch (status) {
+    case DDTREE_OK: return "ok";
+    case DDTREE_ERR_INVALID_ARG: return "invalid argument";
+    case DDTREE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case DDTREE_ERR_CUDA: return "CUDA error";
+    case DDTREE_ERR_NONFINITE: return "non-finite logits";
+    case DDTREE_ERR_TIMEOUT: return "bounded wait timed out";
+    case DDTREE_ERR_CAPACITY: return "prefix plus tree exceeds the KV cache";
+    default: return "unknown status";
+  }
+}
+
+int ddtree_device_status(cudaStream_t stream, unsigned int* bits) {
+  if (!bits) return DDTREE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return DDTREE_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return DDTREE_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return DDTREE_ERR_CUDA;
+  *bits = v;
+  return DDTREE_OK;
+}
+
+int ddtree_version(void) { return 100; }
+
+}  // extern "C"

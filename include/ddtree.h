@@ -1,0 +1,265 @@
+/*
+ * ddtree.h - C ABI of the DDTree round library (libddtree.so), sm_100a.
+ *
+ * One DDTree draft-and-verify round, as described in "DDTree Deep Dive:
+ * Algorithm, Code, and Engineering Philosophy of Block Diffusion Draft
+ * Trees" (zhichai.net; below "Deep Dive") and "DDTree: Turning Block
+ * Diffusion Drafters into Tree-Based Speculative Decoders" (alanhou.org):
+ *
+ *   ddtree_topk       per-position log-softmax and top-K of the drafter's
+ *                     block logits                    (Deep Dive §1, §2 Lemma 1)
+ *   ddtree_build      best-first heap over rank tuples -> prefix-closed tree
+ *                     with parents, depths and ancestor bitmasks
+ *                                                     (Deep Dive §2 Props. 2-3, §3)
+ *   ddtree_tree_attn  ancestor-only attention of the B+1 tree nodes over
+ *                     the committed KV prefix         (Deep Dive §4)
+ *   ddtree_accept     greedy verifier walk + in-place KV compaction
+ *                                                     (Deep Dive §5, §6)
+ *   ddtree_round      the four stages in stream order, no host sync
+ *
+ * Conventions (all entry points):
+ *  - Every pointer argument named as device memory must point to memory of
+ *    the current CUDA device.  The caller owns every buffer; the library
+ *    allocates nothing.  Scratch memory is the caller's workspace `ws` of at
+ *    least the matching *_workspace_bytes(); it must be zero-filled once
+ *    before its first use, and every call leaves its counters at zero again.
+ *    Distinct calls that run concurrently need distinct workspaces.
+ *  - Device pointers must be 16-byte aligned; logits rows must start on
+ *    16-byte boundaries (row_stride * element size a multiple of 16).
+ *  - Every call is asynchronous on `stream`.  The return value reports
+ *    argument and launch errors synchronously (ddtree_status).  Data errors
+ *    found on the device (NaN logits, a prefix that does not fit the cache)
+ *    are OR-ed into a device status word that ddtree_device_status() reads.
+ *  - Integer outputs are bit-exact functions of the inputs.  Ties are broken
+ *    by lower token id (top-K, argmax) and lower rank tuple (tree order).
+ *  - Limits: 1 <= L <= 32, 1 <= K <= min(V, 1024), 0 <= B <= 1024,
+ *    1 <= n_req <= 4096, V <= 1048576, D in {64, 128}, Hq % Hkv == 0,
+ *    page size 64.
+ */
+#ifndef DDTREE_H
+#define DDTREE_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DDTREE_OK = 0,
+  DDTREE_ERR_INVALID_ARG = 1,  /* bad size, null or misaligned pointer */
+  DDTREE_ERR_UNSUPPORTED = 2,  /* valid request outside what is built */
+  DDTREE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  DDTREE_ERR_NONFINITE = 4,    /* device status bit: NaN in logits */
+  DDTREE_ERR_TIMEOUT = 5,      /* device status bit: a bounded wait gave up */
+  DDTREE_ERR_CAPACITY = 6      /* device status bit: prefix + tree exceeds the cache */
+} ddtree_status;
+
+/* Device status word bits (ddtree_device_status). */
+#define DDTREE_STATUS_NONFINITE 0x1u
+#define DDTREE_STATUS_TIMEOUT   0x2u
+#define DDTREE_STATUS_CAPACITY  0x4u
+
+typedef enum { DDTREE_BF16 = 0, DDTREE_F32 = 1 } ddtree_dtype;
+
+#define DDTREE_PAGE 64
+
+/*
+ * KV cache geometry (Deep Dive §5: tree K/V sit in the cache tail).
+ * Request r's committed prefix occupies logical slots 0..P_r-1 and its tree
+ * node j occupies slot P_r + j.
+ *   paged == 0: k/v are contiguous [layers][n_req][s_max][Hkv][D].
+ *   paged == 1: k/v are pools [layers][num_blocks][64][Hkv][D]; logical slot
+ *               s of request r is row s % 64 of block block_table[r][s / 64];
+ *               block_table is int32 [n_req][max_blocks] in device memory.
+ * Element type is the call's dtype.
+ */
+typedef struct {
+  int layers;
+  int n_req;
+  int Hq;
+  int Hkv;
+  int D;
+  float scale;       /* softmax scale; <= 0 selects 1/sqrt(D) */
+  int paged;
+  int s_max;         /* contiguous: slots per request */
+  int num_blocks;    /* paged: pool blocks per layer */
+  int max_blocks;    /* paged: block_table row length (logical capacity 64*max_blocks) */
+} ddtree_kv_desc;
+
+/* ---------------------------------------------------------------------- */
+/* Stage 1: top-K + log-softmax (Deep Dive §1 and §2 Lemma 1).            */
+/* ---------------------------------------------------------------------- */
+
+size_t ddtree_topk_workspace_bytes(int rows, int V, int K);
+
+/*
+ * logits     device, [rows][row_stride] of dtype; only the first V entries
+ *            of a row are read (rows = n_req * L block positions).
+ * K          tokens kept per row, 1 <= K <= min(V, 1024).
+ * ids        device int32 [rows][K]: token ids by (logit desc, id asc).
+ * lp         device float [rows][K]: log q of those tokens, (z - max) - log S
+ *            in fp32, where S = sum exp(z - max).
+ * lse        device float [rows] (may be NULL): max + log S.
+ * NaN logits set DDTREE_STATUS_NONFINITE; -inf is allowed and ranks last;
+ * -0.0 ranks equal to +0.0.
+ */
+int ddtree_topk(const void* logits, int dtype, int rows, int V, long long row_stride,
+                int K, int32_t* ids, float* lp, float* lse,
+                void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Stage 2: tree build (Deep Dive §2 Propositions 2 and 3, §3, §4).       */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * ids, lp    device [n_req][L][K] as written by ddtree_topk (lp sorted
+ *            non-increasing within a row).
+ * root_token device int32 [n_req]: the bonus token b of each request.
+ * B          node budget: non-root nodes, 0 <= B <= 1024.
+ * Outputs, n = B + 1 rows per request, node 0 = root, nodes 1.. in pop
+ * order (so parent[i] < i); rows at or past n_nodes[r] are filled with
+ * token/parent/depth/rank -1, score -inf and an all-zero mask:
+ *   node_token int32 [n_req][n]   token of the node (root: root_token)
+ *   parent     int32 [n_req][n]   parent node (root: -1)
+ *   depth      int32 [n_req][n]   block position of the node (root: 0)
+ *   node_rank  int32 [n_req][n]   rank of the token within its position's top-K
+ *   score      float [n_req][n]   fp32 sum of lp along the path, one add per
+ *                                 depth in root-to-leaf order (root: 0)
+ *   anc        uint32 [n_req][n][W], W = ceil(n/32): bit j of row i (word
+ *              j/32, bit j%32) is set iff node j is i or an ancestor of i
+ *   n_nodes    int32 [n_req]: 1 + number of popped prefixes
+ * The popped set is the top-B of all prefixes of length <= L under the order
+ * (score desc, rank tuple lexicographically asc).  Any output pointer other
+ * than parent, anc and n_nodes may be NULL.
+ */
+int ddtree_build(const int32_t* ids, const float* lp, const int32_t* root_token,
+                 int n_req, int L, int K, int B,
+                 int32_t* node_token, int32_t* parent, int32_t* depth,
+                 int32_t* node_rank, float* score, uint32_t* anc, int32_t* n_nodes,
+                 cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Stage 3: ancestor-only tree attention (Deep Dive §4).                  */
+/* ---------------------------------------------------------------------- */
+
+size_t ddtree_attn_workspace_bytes(const ddtree_kv_desc* kv, int B);
+
+/*
+ * q          device [layers][n_req][B+1][Hq][D] of dtype: tree-node queries
+ *            (already rotated).
+ * k_cache, v_cache  device, geometry `kv` (see ddtree_kv_desc).
+ * prefix_len device int32 [n_req]: committed prefix P_r; P_r + n_nodes[r]
+ *            must fit the request's capacity, else the request is skipped
+ *            and DDTREE_STATUS_CAPACITY is set.
+ * anc, n_nodes  device, as written by ddtree_build for budget B.
+ * out        device [layers][n_req][B+1][Hq][D] of dtype: for node i < n_nodes
+ *            and query head h (KV head h / (Hq/Hkv)), softmax(q k^T * scale) v
+ *            over the prefix slots 0..P-1 and the tree slots P+j of every j set
+ *            in anc[i].  Rows of absent nodes are not written.
+ * out_lse    device float [layers][n_req][B+1][Hq] natural-log sum-exp of the
+ *            scaled scores (may be NULL).
+ * bf16: tcgen05 tensor-core path for D = 128 (fp32 accumulation, P rounded
+ * to bf16 for the PV product); fp32 and D = 64: CUDA-core fp32 path.
+ */
+int ddtree_tree_attn(const void* q, const void* k_cache, const void* v_cache, int dtype,
+                     const ddtree_kv_desc* kv, const int32_t* block_table,
+                     const int32_t* prefix_len, const uint32_t* anc, const int32_t* n_nodes,
+                     int B, void* out, float* out_lse,
+                     void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Stage 4: verifier walk + KV compaction (Deep Dive §5, §6).             */
+/* ---------------------------------------------------------------------- */
+
+size_t ddtree_accept_workspace_bytes(int n_req, int B, int V);
+
+/*
+ * target_logits device [n_req][B+1][row_stride] of dtype: the target's
+ *            logits at every tree node (rows past n_nodes are not read).
+ * node_token, parent, n_nodes  device, from ddtree_build.
+ * prefix_len device int32 [n_req] (read only); new_prefix_len device int32
+ *            [n_req] receives P + accept_len (must not alias prefix_len).
+ * k_cache, v_cache, kv, block_table  the cache to compact in place; k_cache
+ *            may be NULL to skip compaction.
+ * Outputs per request (temperature 0):
+ *   target_argmax int32 [n_req][B+1] (may be NULL): argmax of each live
+ *                 node's row, lowest id on ties (-0.0 equals +0.0)
+ *   path       int32 [n_req][L+1]: accepted node ids root first, -1 after
+ *   accept_len int32 [n_req]: accepted draft nodes + 1 (the new bonus)
+ *   next_bonus int32 [n_req]: target argmax at the last accepted node
+ *   src_slot, dst_slot int32 [n_req][L+1]: P+path[j] -> P+j, -1 after
+ * For every layer and both caches, slot P+path[j] is copied to slot P+j for
+ * j = 0..accept_len-1; all sources are read before any destination is
+ * written.  Any output pointer except new_prefix_len may be NULL.
+ */
+int ddtree_accept(const void* target_logits, int dtype, int V, long long row_stride,
+                  const int32_t* node_token, const int32_t* parent, const int32_t* n_nodes,
+                  int n_req, int L, int B,
+                  const int32_t* prefix_len, int32_t* new_prefix_len,
+                  void* k_cache, void* v_cache, const ddtree_kv_desc* kv,
+                  const int32_t* block_table,
+                  int32_t* target_argmax, int32_t* path, int32_t* accept_len,
+                  int32_t* next_bonus, int32_t* src_slot, int32_t* dst_slot,
+                  void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* The whole round (Deep Dive §3 stage pipeline: draft -> tree_build ->   */
+/* tree_compile -> verify -> commit; the draft and the target forward are */
+/* the caller's, their logits and Q/K/V are inputs here).                 */
+/* ---------------------------------------------------------------------- */
+
+typedef struct {
+  /* sizes */
+  int n_req, L, V, K, B;
+  int dtype;                       /* of drafter logits, q, caches, target logits */
+  ddtree_kv_desc kv;
+  /* inputs (device) */
+  const void* drafter_logits;      /* [n_req*L][drafter_stride] */
+  long long drafter_stride;
+  const int32_t* root_token;       /* [n_req] */
+  const void* q;                   /* [layers][n_req][B+1][Hq][D] */
+  void* k_cache;                   /* compacted in place */
+  void* v_cache;
+  const int32_t* block_table;      /* paged only */
+  const int32_t* prefix_len;       /* [n_req] */
+  const void* target_logits;       /* [n_req][B+1][target_stride] */
+  long long target_stride;
+  /* outputs (device) */
+  int32_t* ids; float* lp; float* lse;                        /* stage 1 */
+  int32_t* node_token; int32_t* parent; int32_t* depth;       /* stage 2 */
+  int32_t* node_rank; float* score; uint32_t* anc; int32_t* n_nodes;
+  void* attn_out; float* attn_lse;                            /* stage 3 */
+  int32_t* target_argmax; int32_t* path; int32_t* accept_len; /* stage 4 */
+  int32_t* next_bonus; int32_t* src_slot; int32_t* dst_slot;
+  int32_t* new_prefix_len;
+  /* scratch */
+  void* ws; size_t ws_bytes;
+} ddtree_round_args;
+
+size_t ddtree_round_workspace_bytes(const ddtree_round_args* a);
+
+/* Stage order topk -> build -> tree_attn -> accept on `stream`; ids, lp,
+ * node_token, parent, depth, anc, n_nodes and new_prefix_len are required,
+ * the other outputs may be NULL. */
+int ddtree_round(const ddtree_round_args* a, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Status                                                                 */
+/* ---------------------------------------------------------------------- */
+
+const char* ddtree_status_string(int status);
+
+/* Synchronises `stream`, returns the device status word's bits in *bits and
+ * clears it.  Returns DDTREE_OK or DDTREE_ERR_CUDA. */
+int ddtree_device_status(cudaStream_t stream, unsigned int* bits);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int ddtree_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DDTREE_H */

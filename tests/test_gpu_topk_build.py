@@ -1,0 +1,162 @@
+"""GPU parity: top-K/log-softmax and tree build against the oracle.
+
+The build stage is fed the oracle's fp32 log-prob table (and ids), so every
+tree array is compared bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import draft_tree_build_ddtree_b200 as dd
+from draft_tree_build_ddtree_b200 import datagen
+
+from parity import assert_topk, assert_tree, oracle_topk, oracle_trees, tree_inputs
+
+pytestmark = pytest.mark.gpu
+CUDA = "cuda:0"
+
+
+def _gpu_topk(z: torch.Tensor, K: int):
+    x = z.reshape(-1, z.shape[-1]).to(CUDA)
+    ids, lp, lse = dd.ddtree_topk(x, K)
+    torch.cuda.synchronize()
+    assert dd.device_status() == 0
+    return ids, lp, lse
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_topk_configs(cfg):
+    w = datagen.workload(cfg)
+    z = datagen.drafter_logits(w)
+    ids, lp32, lse32 = oracle_topk(z, w.K)
+    g = _gpu_topk(z, w.K)
+    assert_topk(*g, ids.reshape(-1, w.K), lp32.reshape(-1, w.K), lse32.reshape(-1))
+
+
+@pytest.mark.parametrize("sigma", [1.0, 8.0])
+def test_topk_k1024_sweep(sigma):
+    w = datagen.workload(5, B=1024, sigma=sigma)
+    z = datagen.drafter_logits(w)
+    ids, lp32, lse32 = oracle_topk(z, w.K)
+    g = _gpu_topk(z, w.K)
+    assert_topk(*g, ids.reshape(-1, w.K), lp32.reshape(-1, w.K), lse32.reshape(-1))
+
+
+@pytest.mark.parametrize("V,K,dtype", [(5000, 64, torch.bfloat16), (5000, 1024, torch.bfloat16),
+                                       (3000, 100, torch.float32), (151936, 256, torch.bfloat16)])
+def test_topk_heavy_ties(V, K, dtype):
+    g = torch.Generator().manual_seed(V + K)
+    z = torch.randint(-3, 4, (6, V), generator=g).to(dtype)
+    z[0, 5] = -0.0
+    z[0, 6] = 0.0
+    z[1, :100] = float("-inf")
+    ids, lp32, lse32 = oracle_topk(z, K)
+    assert_topk(*_gpu_topk(z, K), ids, lp32, lse32)
+
+
+def test_topk_dominant_token_uses_fallback_select():
+    # one logit far above the rest: the max-anchored window holds < K values
+    g = torch.Generator().manual_seed(4)
+    z = torch.randn(4, 151936, generator=g).to(torch.bfloat16)
+    z[:, 7] = 300.0
+    ids, lp32, lse32 = oracle_topk(z, 64)
+    assert_topk(*_gpu_topk(z, 64), ids, lp32, lse32)
+
+
+@pytest.mark.parametrize("V,K", [(1001, 17), (9, 9), (3, 1)])
+def test_topk_ragged_rows(V, K):
+    g = torch.Generator().manual_seed(V)
+    stride = (V + 7) // 8 * 8
+    full = torch.randn(5, stride, generator=g).to(torch.bfloat16)
+    ids, lp32, lse32 = oracle_topk(full[:, :V], K)
+    x = full.to(CUDA)[:, :V]
+    gi, gl, ge = dd.ddtree_topk(x, K)
+    assert_topk(gi, gl, ge, ids, lp32, lse32)
+
+
+def test_topk_many_rows_sampled():
+    w = datagen.workload(4)
+    z = datagen.drafter_logits(w)            # [32, 16, V]
+    gi, gl, ge = _gpu_topk(z, w.K)
+    rows = [0, 17, 255, 300, 511]
+    flat = z.reshape(-1, w.V)
+    ids, lp32, lse32 = oracle_topk(flat[rows], w.K)
+    assert_topk(gi[rows], gl[rows], ge[rows], ids, lp32, lse32)
+
+
+def test_topk_repeat_calls_reuse_workspace():
+    w = datagen.workload(2)
+    z = datagen.drafter_logits(w)
+    a = _gpu_topk(z, w.K)
+    b = _gpu_topk(z, w.K)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_topk_nan_sets_status():
+    z = torch.randn(2, 4096).to(torch.bfloat16)
+    z[1, 100] = float("nan")
+    dd.ddtree_topk(z.to(CUDA), 8)
+    assert dd.device_status() & dd.STATUS_NONFINITE
+    assert dd.device_status() == 0
+
+
+# ------------------------------------------------------------------ build
+
+def _gpu_build(ids, lp32, root, B):
+    t = dd.ddtree_build(torch.from_numpy(np.ascontiguousarray(ids)).to(CUDA),
+                        torch.from_numpy(np.ascontiguousarray(lp32)).to(CUDA),
+                        torch.from_numpy(np.ascontiguousarray(root).astype(np.int32)).to(CUDA), B)
+    torch.cuda.synchronize()
+    return t
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_build_configs(cfg):
+    w = datagen.workload(cfg)
+    z, ids, lp32, lse32, root, trees, st = tree_inputs(w)
+    assert_tree(_gpu_build(ids, lp32, root, w.B), st)
+
+
+@pytest.mark.parametrize("sigma", [1.0, 4.0, 8.0])
+def test_build_sweep_b1024(sigma):
+    w = datagen.workload(5, B=1024, sigma=sigma)
+    z, ids, lp32, lse32, root, trees, st = tree_inputs(w)
+    assert_tree(_gpu_build(ids, lp32, root, w.B), st)
+
+
+@pytest.mark.parametrize("B", [16, 128, 512])
+def test_build_sweep_budgets(B):
+    w = datagen.workload(5, B=B, sigma=4.0)
+    z, ids, lp32, lse32, root, trees, st = tree_inputs(w)
+    assert_tree(_gpu_build(ids, lp32, root, w.B), st)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_build_exact_score_ties(seed):
+    # coarse tables: many prefixes tie exactly in fp32 and the rank tuple decides
+    g = torch.Generator().manual_seed(seed)
+    N, L, K, B = 8, 6, 12, 200
+    lp = -torch.randint(0, 4, (N, L, K), generator=g).to(torch.float32) * 0.5
+    lp = -torch.sort(-lp, dim=-1).values
+    ids = torch.randint(0, 1000, (N, L, K), generator=g).to(torch.int32)
+    root = torch.arange(N, dtype=torch.int32)
+    trees, st = oracle_trees(ids.numpy(), lp.numpy(), root.numpy(), B)
+    assert_tree(_gpu_build(ids.numpy(), lp.numpy(), root.numpy(), B), st)
+
+
+@pytest.mark.parametrize("L,K,B", [(2, 2, 10), (4, 3, 0), (16, 1, 16), (32, 4, 300), (1, 7, 5)])
+def test_build_edge_shapes(L, K, B):
+    g = torch.Generator().manual_seed(L * 100 + K)
+    lp = -torch.rand(3, L, K, generator=g) * 5
+    lp = -torch.sort(-lp, dim=-1).values
+    ids = torch.randint(0, 5000, (3, L, K), generator=g).to(torch.int32)
+    root = torch.tensor([1, 2, 3], dtype=torch.int32)
+    trees, st = oracle_trees(ids.numpy(), lp.numpy(), root.numpy(), B)
+    assert_tree(_gpu_build(ids.numpy(), lp.numpy(), root.numpy(), B), st)
+
+
+def test_build_batched_config4():
+    w = datagen.workload(4)
+    z, ids, lp32, lse32, root, trees, st = tree_inputs(w)
+    assert_tree(_gpu_build(ids, lp32, root, w.B), st)

@@ -1,0 +1,89 @@
+"""The C-ABI library builds, loads and exports what include/ddtree.h declares.
+
+CPU only: no call here launches a kernel.  Argument checks run on the host
+before any CUDA call, so invalid arguments are rejected without a device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import draft_tree_build_ddtree_b200 as dd
+from draft_tree_build_ddtree_b200 import build_lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if f.endswith(".h")]
+
+
+def declared_functions():
+    names = []
+    for h in HEADERS:
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*[A-Za-z_][\w \*]*?\b(ddtree_\w+)\s*\(", src, flags=re.M):
+            names.append(m.group(1))
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_lib.build()
+    return dd.lib()
+
+
+def test_header_declares_the_round_entry_points():
+    names = declared_functions()
+    for n in ("ddtree_topk", "ddtree_build", "ddtree_tree_attn", "ddtree_accept", "ddtree_round"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_covers_every_declared_symbol():
+    assert set(declared_functions()) <= set(dd.exported_symbols())
+
+
+def test_status_strings(lib):
+    assert lib.ddtree_status_string(0) == b"ok"
+    assert lib.ddtree_status_string(1) == b"invalid argument"
+    assert lib.ddtree_version() >= 100
+
+
+def test_host_validation_rejects_bad_arguments(lib):
+    INVALID = 1
+    # null logits
+    assert lib.ddtree_topk(None, 0, 16, 1000, 1000, 8, None, None, None, None, 0, None) == INVALID
+    # K > V
+    p = ctypes.c_void_p(16)
+    assert lib.ddtree_topk(p, 0, 1, 8, 8, 9, p, p, None, p, 1 << 20, None) == INVALID
+    # row stride not a multiple of 16 bytes
+    assert lib.ddtree_topk(p, 0, 1, 1001, 1001, 8, p, p, None, p, 1 << 20, None) == INVALID
+    # misaligned logits pointer
+    assert lib.ddtree_topk(ctypes.c_void_p(18), 0, 1, 1000, 1000, 8, p, p, None, p, 1 << 20,
+                           None) == INVALID
+    # budget above the limit; L above the limit
+    assert lib.ddtree_build(p, p, p, 1, 16, 64, 1025, p, p, p, p, p, p, p, None) == INVALID
+    assert lib.ddtree_build(p, p, p, 1, 33, 64, 64, p, p, p, p, p, p, p, None) == INVALID
+    # accept: output aliasing its input
+    kv = dd.kv_desc(1, 1, 32, 4, 128, s_max=4096)
+    assert lib.ddtree_accept(p, 0, 1000, 1000, p, p, p, 1, 16, 64, p, p, None, None,
+                             ctypes.byref(kv), None, None, None, None, None, None, None, p,
+                             1 << 20, None) == INVALID
+    # attention: Hq not a multiple of Hkv; unsupported head dim
+    bad = dd.kv_desc(1, 1, 30, 4, 128, s_max=4096)
+    assert lib.ddtree_tree_attn(p, p, p, 0, ctypes.byref(bad), None, p, p, p, 64, p, None, p,
+                                1 << 20, None) == INVALID
+    odd = dd.kv_desc(1, 1, 32, 4, 96, s_max=4096)
+    assert lib.ddtree_tree_attn(p, p, p, 0, ctypes.byref(odd), None, p, p, p, 64, p, None, p,
+                                1 << 20, None) == 2
+
+
+def test_cpu_tensors_are_refused():
+    import torch
+    with pytest.raises(dd.DDTreeError):
+        dd.ddtree_topk(torch.zeros(2, 64), 4)

@@ -194,6 +194,17 @@ __global__ void __launch_bounds__(WALK_THREADS) walk_compact_kernel(WalkArgs a) 
     s_ok = (P >= 0 && (long long)P + nn <= cap) ? 1 : 0;
   }
   __syncthreads();
+  if (a.paged && a.k_cache != nullptr && s_ok) {   // blocks holding slots [0, P + nn) must be pool blocks
+    const int nb = (P + nn + DDTREE_PAGE - 1) / DDTREE_PAGE;
+    int bad = 0;
+    for (int b = tid; b < nb; b += WALK_THREADS) {
+      const int blk = a.block_table[(size_t)r * a.max_blocks + b];
+      bad |= (blk < 0 || blk >= a.num_blocks);
+    }
+    bad = __syncthreads_or(bad);
+    if (tid == 0 && bad) s_ok = 0;
+    __syncthreads();
+  }
   const int k = s_k;
   if (lk == 0) {
     for (int i = tid; i <= a.L; i += WALK_THREADS) {

@@ -73,6 +73,18 @@ tree_attn_simt_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T
     if (threadIdx.x == 0 && i == 0 && hg == 0) flag_status(DDTREE_STATUS_CAPACITY);
     return;
   }
+  if (g.paged) {   // every block the request reads must be a pool block
+    const int nb = (P + nn + DDTREE_PAGE - 1) / DDTREE_PAGE;
+    int bad = 0;
+    for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+      const int blk = block_table[(size_t)r * g.max_blocks + b];
+      bad |= (blk < 0 || blk >= g.num_blocks);
+    }
+    if (__syncthreads_or(bad)) {
+      if (threadIdx.x == 0 && i == 0 && hg == 0) flag_status(DDTREE_STATUS_CAPACITY);
+      return;
+    }
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     int c = 0;

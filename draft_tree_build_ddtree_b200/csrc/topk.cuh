@@ -9,7 +9,12 @@
 //    6 vectors per thread), so one wave of CTAs keeps the whole input in
 //    flight.
 //  * Each CTA reduces its chunk to (max, sum exp(z - max)) and to its local
-//    top-K' (K' = min(K, chunk length)) by a radix select on a unique
+//    top-K' (K' = min(K, chunk length)).  The sum is taken in fp64 (fp64
+//    exp and adds) so that log q = z - lse, rounded once to fp32, is the
+//    correctly rounded value in all but vanishingly rare cases: bf16 logits
+//    sit on a coarse grid, many prefixes tie exactly in real arithmetic, and
+//    only a correctly rounded log-prob table orders them reproducibly.  The
+//    local top-K' comes from a radix select on a unique
 //    composite key (order key of the logit, then the complemented local
 //    index so that lower ids win ties).  For bf16 the first pass is a
 //    256-bin histogram anchored at the chunk maximum: each bin is one bf16
@@ -64,14 +69,14 @@ inline TopkPlan topk_plan(int rows, int V, int K, int esize, int num_sms) {
 // (max, sumexp) float2, then the candidates (u64).
 struct TopkWs {
   uint32_t* ticket;        // [rows]
-  float2* stats;           // [rows][cpr]
+  double2* stats;          // [rows][cpr]: (chunk max, sum of exp(z - max)) in fp64
   unsigned long long* cand;  // [rows][cand]
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 inline size_t topk_ws_bytes(int rows, const TopkPlan& p) {
-  return align256((size_t)rows * 4) + align256((size_t)rows * p.cpr * 8) +
+  return align256((size_t)rows * 4) + align256((size_t)rows * p.cpr * 16) +
          align256((size_t)rows * p.cand * 8);
 }
 
@@ -80,8 +85,8 @@ inline TopkWs topk_ws_carve(void* ws, int rows, const TopkPlan& p) {
   TopkWs w;
   w.ticket = (uint32_t*)b;
   b += align256((size_t)rows * 4);
-  w.stats = (float2*)b;
-  b += align256((size_t)rows * p.cpr * 8);
+  w.stats = (double2*)b;
+  b += align256((size_t)rows * p.cpr * 16);
   w.cand = (unsigned long long*)b;
   return w;
 }
@@ -185,7 +190,7 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ uint32_t hist[256];
   __shared__ int bcast[4];
-  __shared__ float red_f[TOPK_THREADS / 32];
+  __shared__ double red_d[TOPK_THREADS / 32];
   __shared__ LKey red_k[TOPK_THREADS / 32];
   __shared__ int s_count;
   __shared__ int s_last;
@@ -274,22 +279,24 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   // ---- sum of exp(z - m); for bf16 also the max-anchored window histogram ----
   for (int i = tid; i < 256; i += TOPK_THREADS) hist[i] = 0;
   __syncthreads();
-  float s = 0.f;
+  double s = 0.0;
   const bool m_finite = m > -INFINITY;
+  const double md = (double)m;
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     if (lid_at(e) < len) {
       uint32_t bits = raw_at(e);
       float z = (DT == DDTREE_BF16) ? bf16_bits_to_f32((uint16_t)bits) : __uint_as_float(bits);
-      if (m_finite) s += expf(z - m);
+      if (m_finite) s += exp((double)z - md);
       if (DT == DDTREE_BF16) {
         uint32_t d = vkey_max - key16_of_bf16((uint16_t)bits);
         if (d < 256u) atomicAdd(&hist[d], 1u);
       }
     }
   }
-  s = warp_sum(s);
-  if ((tid & 31) == 0) red_f[tid >> 5] = s;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((tid & 31) == 0) red_d[tid >> 5] = s;
   __syncthreads();
 
   // ---- local threshold ----
@@ -362,9 +369,9 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
     }
   }
   if (tid == 0) {
-    float tot = 0.f;
-    for (int i = 0; i < TOPK_THREADS / 32; ++i) tot += red_f[i];
-    ws.stats[(size_t)row * plan.cpr + c] = make_float2(m, tot);
+    double tot = 0.0;
+    for (int i = 0; i < TOPK_THREADS / 32; ++i) tot += red_d[i];
+    ws.stats[(size_t)row * plan.cpr + c] = make_double2(md, tot);
   }
   __threadfence();
   __syncthreads();
@@ -385,19 +392,18 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   for (int i = tid; i < ncand; i += TOPK_THREADS) sc[i] = __ldcg(cand_row + i);
   for (int i = tid; i < kpow; i += TOPK_THREADS) win[i] = 0ull;
   if (tid == 0) s_count = 0;
-  __shared__ float s_M, s_logS;
+  __shared__ double s_lse;
   if (tid == 0) {
-    float M = -INFINITY;
-    for (int i = 0; i < plan.cpr; ++i) M = fmaxf(M, __ldcg(&ws.stats[(size_t)row * plan.cpr + i].x));
-    float S = 0.f;
+    double M = -INFINITY;
+    for (int i = 0; i < plan.cpr; ++i) M = fmax(M, __ldcg(&ws.stats[(size_t)row * plan.cpr + i].x));
+    double S = 0.0;
     if (M > -INFINITY) {
       for (int i = 0; i < plan.cpr; ++i) {
-        float2 st = __ldcg(&ws.stats[(size_t)row * plan.cpr + i]);
-        if (st.x > -INFINITY) S += st.y * expf(st.x - M);
+        double2 st = __ldcg(&ws.stats[(size_t)row * plan.cpr + i]);
+        if (st.x > -INFINITY) S += st.y * exp(st.x - M);
       }
     }
-    s_M = M;
-    s_logS = logf(S);
+    s_lse = M + log(S);
     ws.ticket[row] = 0;   // leave the workspace ready for the next call
   }
   __syncthreads();
@@ -433,16 +439,16 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
       __syncthreads();
     }
   }
-  const float M = s_M, logS = s_logS;
+  const double lse = s_lse;
   for (int i = tid; i < K; i += TOPK_THREADS) {
     unsigned long long k = win[i];
     uint32_t vkey = (uint32_t)(k >> TOPK_ID_BITS);
     int id = (int)(TOPK_ID_MASK - (uint32_t)(k & TOPK_ID_MASK));
     float z = (DT == DDTREE_BF16) ? bf16_of_key16(vkey) : f32_of_key32(vkey);
     out_ids[(size_t)row * K + i] = id;
-    out_lp[(size_t)row * K + i] = (z - M) - logS;
+    out_lp[(size_t)row * K + i] = (float)((double)z - lse);   // one rounding of the fp64 value
   }
-  if (out_lse != nullptr && tid == 0) out_lse[row] = M + logS;
+  if (out_lse != nullptr && tid == 0) out_lse[row] = (float)lse;
 }
 
 inline size_t topk_smem_bytes(const TopkPlan& p, int K) {

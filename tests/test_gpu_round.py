@@ -1,9 +1,10 @@
 """GPU parity of the whole round (ddtree_round) against the oracle chain.
 
-The round feeds its own top-K table to its build, so the tree is compared
-bit-exactly only where the oracle's order margin exceeds what the log-prob
-tolerance can move (else the GPU tree is checked for validity); every
-downstream integer output is compared bit-exactly.
+The round feeds its own top-K table to its build.  Its log-probs are the
+fp64 log-softmax rounded once to fp32, like the oracle's, so the table is
+bit-identical in practice and every tree array is then compared bit for
+bit; every downstream integer output and the compacted cache are compared
+bit for bit, the attention output within tolerance.
 """
 import numpy as np
 import pytest
@@ -13,7 +14,7 @@ import draft_tree_build_ddtree_b200 as dd
 import oracle
 from draft_tree_build_ddtree_b200 import datagen
 
-from parity import LP_TOL, assert_topk, attn_close, np64, order_margin, tree_inputs
+from parity import assert_topk, attn_close, np64, tree_inputs
 
 pytestmark = pytest.mark.gpu
 CUDA = "cuda:0"
@@ -49,17 +50,21 @@ def check_round(w, rb, h, layers=None, nodes=None, heads=None):
     assert_topk(rb.ids.reshape(-1, w.K), rb.lp.reshape(-1, w.K), rb.lse, h["ids"].reshape(-1, w.K),
                 h["lp32"].reshape(-1, w.K), h["lse32"].reshape(-1))
     st = h["st"]
-    exact = all(order_margin(h["lp32"][r], w.B) > 2 * w.L * LP_TOL + 1e-4 for r in range(w.N))
+    # The tree is a deterministic function of the (ids, lp) table, and the
+    # build stage alone is bit-exact on identical tables; so when the round's
+    # lp table is bit-identical to the oracle's, every tree array must be too.
+    lp_same = np.array_equal(rb.lp.cpu().numpy().reshape(h["lp32"].shape).view(np.uint32),
+                             h["lp32"].view(np.uint32))
     t = rb.tree
-    if exact:
+    if lp_same:
         for name in ("node_token", "parent", "depth", "node_rank", "n_nodes"):
             assert np.array_equal(getattr(t, name).cpu().numpy(), st[name]), name
         assert np.array_equal(t.anc.cpu().numpy().view(np.uint32), st["anc"])
-        assert np.max(np.abs(t.score.cpu().numpy()[:, 1:] - st["score"][:, 1:])) <= w.L * LP_TOL
+        assert np.array_equal(t.score.cpu().numpy().view(np.uint32), st["score"].view(np.uint32))
     else:
         for r in range(w.N):
             _valid_tree(t.parent[r].cpu().numpy(), t.anc[r].cpu().numpy(), int(t.n_nodes[r]))
-        pytest.skip("order margin below the log-prob tolerance: tree validity checked only")
+        pytest.skip("an lp value differs from the oracle's in its last bit: tree validity checked only")
     # attention of the tree nodes
     table = None if h["cache"].block_table is None else h["cache"].block_table.numpy()
     ref, _ = oracle.tree_attention(np64(h["q"]), np64(h["cache"].k), np64(h["cache"].v), h["prefix"],

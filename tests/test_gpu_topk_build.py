@@ -24,13 +24,17 @@ def _gpu_topk(z: torch.Tensor, K: int):
     return ids, lp, lse
 
 
-@pytest.mark.parametrize("cfg", [1, 2])
+@pytest.mark.parametrize("cfg", [1, 2, 4])
 def test_topk_configs(cfg):
     w = datagen.workload(cfg)
     z = datagen.drafter_logits(w)
+    if cfg == 4:
+        z = z[:4]
     ids, lp32, lse32 = oracle_topk(z, w.K)
     g = _gpu_topk(z, w.K)
     assert_topk(*g, ids.reshape(-1, w.K), lp32.reshape(-1, w.K), lse32.reshape(-1))
+    # fp64 log-sum-exp: the fp32 log-probs round like the oracle's, bit for bit
+    assert np.array_equal(g[1].cpu().numpy().view(np.uint32), lp32.reshape(-1, w.K).view(np.uint32))
 
 
 @pytest.mark.parametrize("sigma", [1.0, 8.0])

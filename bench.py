@@ -459,7 +459,7 @@ def oracle_round_sample(w, z, root, q, cache, prefix, tgt, frac_rows=1, node_lim
     # and the compaction of the accepted path over every layer
     arows = min(tree.n_nodes, frac_rows if w.cfg == 1 else 2)
     t0 = time.perf_counter()
-    oracle.argmax_rows(tgt[0, :arows].numpy())
+    oracle.argmax_rows(tgt[0, :arows].to(torch.float32).numpy())
     t_arg = (time.perf_counter() - t0) * tree.n_nodes / arows
     tg = np.zeros((tree.n_nodes, 4))
     for i in range(1, tree.n_nodes):      # a target that follows the deepest branch

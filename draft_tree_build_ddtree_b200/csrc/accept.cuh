@@ -51,13 +51,16 @@ inline ArgmaxWs argmax_ws_carve(void* ws, int rows) {
   return w;
 }
 
-template <int DT>
+// The argmax of one chunk: bf16 keys are 32-bit composites (16-bit order key,
+// then the complemented 15-bit chunk-local index) reduced with redux.sync;
+// fp32 keys need 64 bits.  The chunk winner becomes a 64-bit composite with
+// the global token id for the row-wide atomicMax.
+template <int DT, int VPT>
 __global__ void __launch_bounds__(ARGMAX_THREADS)
 argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_stride,
               const int32_t* __restrict__ n_nodes, int cpr, int chunk, ArgmaxWs ws) {
   constexpr int EPV = (DT == DDTREE_BF16) ? 8 : 4;
   __shared__ unsigned long long red[ARGMAX_THREADS / 32];
-  __shared__ int s_last;
   const int tid = threadIdx.x;
   const int row = blockIdx.x / cpr;              // row = req * n + node
   const int c = blockIdx.x - row * cpr;
@@ -69,55 +72,63 @@ argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_strid
       (const unsigned char*)logits + ((long long)row * row_stride + c0) * (16 / EPV);
   const int nvec_full = len / EPV;
 
-  uint4 vec[TOPK_MAX_VPT];
+  uint4 vec[VPT];
 #pragma unroll
-  for (int v = 0; v < TOPK_MAX_VPT; ++v) {
-    int vi = v * ARGMAX_THREADS + tid;
+  for (int v = 0; v < VPT; ++v) {
+    const int vi = v * ARGMAX_THREADS + tid;
     vec[v] = vi < nvec_full ? ldg_stream_v4(base + (size_t)vi * 16) : make_uint4(0, 0, 0, 0);
   }
   unsigned long long best = 0;
   bool nan_seen = false;
+  if (DT == DDTREE_BF16) {
+    uint32_t b32 = 0;
 #pragma unroll
-  for (int v = 0; v < TOPK_MAX_VPT; ++v) {
-    const int vi = v * ARGMAX_THREADS + tid;
-    if (vi < nvec_full) {
+    for (int v = 0; v < VPT; ++v) {
+      const int vi = v * ARGMAX_THREADS + tid;
+      if (vi < nvec_full) {
 #pragma unroll
-      for (int j = 0; j < EPV; ++j) {
-        uint32_t bits = (DT == DDTREE_BF16) ? ((u32_at(vec[v], j >> 1) >> (16 * (j & 1))) & 0xFFFFu)
-                                            : u32_at(vec[v], j);
-        uint32_t key;
-        if (DT == DDTREE_BF16) {
-          nan_seen |= bf16_is_nan((uint16_t)bits);
-          key = key16_of_bf16((uint16_t)bits);
-        } else {
-          float f = __uint_as_float(bits);
-          nan_seen |= (f != f);
-          key = key32_of_f32(f);
+        for (int j = 0; j < EPV; ++j) {
+          const uint16_t bits = (uint16_t)((u32_at(vec[v], j >> 1) >> (16 * (j & 1))) & 0xFFFFu);
+          nan_seen |= bf16_is_nan(bits);
+          const uint32_t k = (key16_of_bf16(bits) << LID_BITS) | (LID_MASK - (uint32_t)(vi * EPV + j));
+          b32 = k > b32 ? k : b32;
         }
-        const uint32_t gid = (uint32_t)(c0 + (long long)vi * EPV + j);
-        unsigned long long k = ((unsigned long long)key << TOPK_ID_BITS) | (TOPK_ID_MASK - gid);
-        best = k > best ? k : best;
       }
     }
-  }
-  // ragged tail (V not a multiple of the vector width)
-  for (int e = nvec_full * EPV + tid; e < len; e += ARGMAX_THREADS) {
-    uint32_t key;
-    if (DT == DDTREE_BF16) {
-      uint16_t bits = ((const uint16_t*)base)[e];
+    for (int e = nvec_full * EPV + tid; e < len; e += ARGMAX_THREADS) {   // ragged tail
+      const uint16_t bits = ((const uint16_t*)base)[e];
       nan_seen |= bf16_is_nan(bits);
-      key = key16_of_bf16(bits);
-    } else {
-      float f = ((const float*)base)[e];
-      nan_seen |= (f != f);
-      key = key32_of_f32(f);
+      const uint32_t k = (key16_of_bf16(bits) << LID_BITS) | (LID_MASK - (uint32_t)e);
+      b32 = k > b32 ? k : b32;
     }
-    const uint32_t gid = (uint32_t)(c0 + e);
-    unsigned long long k = ((unsigned long long)key << TOPK_ID_BITS) | (TOPK_ID_MASK - gid);
-    best = k > best ? k : best;
+    b32 = __reduce_max_sync(0xffffffffu, b32);
+    const uint32_t gid = (uint32_t)(c0 + (LID_MASK - (b32 & LID_MASK)));
+    best = b32 ? (((unsigned long long)(b32 >> LID_BITS) << TOPK_ID_BITS) | (TOPK_ID_MASK - gid)) : 0ull;
+  } else {
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) {
+      const int vi = v * ARGMAX_THREADS + tid;
+      if (vi < nvec_full) {
+#pragma unroll
+        for (int j = 0; j < EPV; ++j) {
+          const float f = __uint_as_float(u32_at(vec[v], j));
+          nan_seen |= (f != f);
+          const uint32_t gid = (uint32_t)(c0 + (long long)vi * EPV + j);
+          const unsigned long long k = ((unsigned long long)key32_of_f32(f) << TOPK_ID_BITS) | (TOPK_ID_MASK - gid);
+          best = k > best ? k : best;
+        }
+      }
+    }
+    for (int e = nvec_full * EPV + tid; e < len; e += ARGMAX_THREADS) {
+      const float f = ((const float*)base)[e];
+      nan_seen |= (f != f);
+      const uint32_t gid = (uint32_t)(c0 + e);
+      const unsigned long long k = ((unsigned long long)key32_of_f32(f) << TOPK_ID_BITS) | (TOPK_ID_MASK - gid);
+      best = k > best ? k : best;
+    }
+    best = warp_max_u64(best);
   }
   if (__any_sync(0xffffffffu, nan_seen) && (tid & 31) == 0) flag_status(DDTREE_STATUS_NONFINITE);
-  best = warp_max_u64(best);
   if ((tid & 31) == 0) red[tid >> 5] = best;
   __syncthreads();
   if (tid == 0) {
@@ -125,11 +136,10 @@ argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_strid
     for (int i = 1; i < ARGMAX_THREADS / 32; ++i) b = red[i] > b ? red[i] : b;
     atomicMax(&ws.best[row], b);
     __threadfence();
-    unsigned t = atomicAdd(&ws.ticket[row], 1u);
-    s_last = (t == (unsigned)(cpr - 1));
-    if (s_last) {
+    const unsigned t = atomicAdd(&ws.ticket[row], 1u);
+    if (t == (unsigned)(cpr - 1)) {
       __threadfence();
-      unsigned long long fin = atomicExch(&ws.best[row], 0ull);   // read and reset
+      const unsigned long long fin = atomicExch(&ws.best[row], 0ull);   // read and reset
       ws.argmax[row] = (int32_t)(TOPK_ID_MASK - (uint32_t)(fin & TOPK_ID_MASK));
       ws.ticket[row] = 0;
     }

@@ -419,22 +419,38 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&sm.bar_sfree);
-      // mask: keys >= P are tree slots (visible iff an ancestor), keys >= T absent
+      // mask: keys >= P are tree slots (visible iff an ancestor), keys >= T absent.
+      // Four 32-key visibility words per tile, built from the node's ancestor row.
       if (k0 + TC_BN > P) {
-        const bool live = node < nn;
+        uint32_t mw[TC_BN / 32];
 #pragma unroll
-        for (int c = 0; c < TC_BN; ++c) {
-          const int key = k0 + c;
-          if (key >= P) {
-            const int tj = key - P;
-            bool vis = live && key < T && ((arow[tj >> 5] >> (tj & 31)) & 1u);
-            if (!vis) s[c] = -INFINITY;
+        for (int w = 0; w < TC_BN / 32; ++w) {
+          const int kb = k0 + 32 * w;
+          const int j0 = kb - P;                       // tree index of the word's first key
+          uint32_t word;
+          if (j0 <= -32) {
+            word = 0xffffffffu;                        // all prefix keys
+          } else if (j0 < 0) {
+            word = (node < nn ? (arow[0] << (-j0)) : 0u) | ((1u << (-j0)) - 1u);
+          } else {
+            const int wi = j0 >> 5, sh = j0 & 31;
+            const uint32_t lo = (node < nn && wi < g.W) ? arow[wi] : 0u;
+            const uint32_t hi = (node < nn && wi + 1 < g.W) ? arow[wi + 1] : 0u;
+            word = __funnelshift_r(lo, hi, sh);
           }
+          mw[w] = word;
         }
-      }
-      float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < TC_BN; ++c) mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < TC_BN; ++c)
+          if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+      }
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < TC_BN; c += 4) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) mx4[t] = fmaxf(mx4[t], s[c + t]);
+      }
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       const float m_tile = mx * sl2;
       bool rescale = false;
       float m_new = m_used;
@@ -464,29 +480,26 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         if (rescale) m_used = m_new;
       }
-      // P = exp2(s*sl2 - m) as bf16 into the swizzled K-major tile
+      // P = exp2(s*sl2 - m) as bf16 into the swizzled K-major tile (exp2(-inf) = 0 masks)
       const float mneg = (m_used == -INFINITY) ? 0.f : -m_used;
-      float lsum = 0.f;
-      unsigned char* prow = sm.p + (row >> 3) * 1024 + (row & 7) * 128;
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+      unsigned char* prow = sm.p + row * 128;
 #pragma unroll
       for (int ch = 0; ch < TC_BN / 8; ++ch) {       // 16-byte chunks of 8 keys
         float e[8];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const float x = s[ch * 8 + t];
-          e[t] = (x == -INFINITY) ? 0.f : exp2f(fmaf(x, sl2, mneg));
-        }
+        for (int t = 0; t < 8; ++t) e[t] = exp2f(fmaf(s[ch * 8 + t], sl2, mneg));
         uint4 pk;
         pk.x = pack_bf16x2(e[0], e[1]);
         pk.y = pack_bf16x2(e[2], e[3]);
         pk.z = pack_bf16x2(e[4], e[5]);
         pk.w = pack_bf16x2(e[6], e[7]);
 #pragma unroll
-        for (int t = 0; t < 8; ++t) lsum += e[t];
+        for (int t = 0; t < 8; ++t) ls4[t & 3] += e[t];
         const int atom = ch >> 3, c16 = ch & 7;
         *reinterpret_cast<uint4*>(prow + atom * TC_ATOM + ((c16 ^ (row & 7)) << 4)) = pk;
       }
-      l += lsum;
+      l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
       mbar_arrive(&sm.bar_pfull);
@@ -552,10 +565,18 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 }
 
 // Merge the key splits of every (unit, row): O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
+// One CTA per (unit, group of 8 rows); 16 threads share a row, each owning 8
+// consecutive dims, so every split's partial row is read with coalesced
+// 16-byte loads.
+constexpr int TC_COMBINE_ROWS = 8;
+constexpr int TC_MAX_SPLITS = 16;
+
 __global__ void __launch_bounds__(128)
 tree_attn_combine_kernel(const TcParams p) {
   const AttnGeom& g = p.g;
-  int u = blockIdx.x;
+  const int groups = TC_BM / TC_COMBINE_ROWS;
+  int u = blockIdx.x / groups;
+  const int rg = blockIdx.x - u * groups;
   const int unit = u;
   const int mt = u % p.mtiles; u /= p.mtiles;
   const int kvh = u % g.Hkv; u /= g.Hkv;
@@ -567,45 +588,46 @@ tree_attn_combine_kernel(const TcParams p) {
   const int P = p.prefix_len[r];
   const long long cap = g.paged ? (long long)g.max_blocks * DDTREE_PAGE : (long long)g.s_max;
   if (P < 0 || (long long)P + nn > cap) return;
-  // thread t: row = t, all 128 dims
-  const int row = threadIdx.x;
+  const int row = rg * TC_COMBINE_ROWS + (threadIdx.x >> 4);
+  const int d0 = (threadIdx.x & 15) * 8;
   const int node = node0 + row / p.G;
   if (node >= nn) return;
   const int hq = kvh * p.G + row % p.G;
+  float2 ml[TC_MAX_SPLITS];
   float M = -INFINITY;
-  for (int s = 0; s < p.splits; ++s) M = fmaxf(M, p.ws_ml[((size_t)unit * p.splits + s) * TC_BM + row].x);
+#pragma unroll
+  for (int s = 0; s < TC_MAX_SPLITS; ++s) {
+    if (s < p.splits) {
+      ml[s] = p.ws_ml[((size_t)unit * p.splits + s) * TC_BM + row];
+      M = fmaxf(M, ml[s].x);
+    }
+  }
   float wsum = 0.f;
-  float acc[TC_D];
+  float acc[8];
 #pragma unroll
-  for (int d = 0; d < TC_D; ++d) acc[d] = 0.f;
-  for (int s = 0; s < p.splits; ++s) {
-    const size_t slot = (size_t)unit * p.splits + s;
-    const float2 ml = p.ws_ml[slot * TC_BM + row];
-    if (ml.x == -INFINITY) continue;
-    const float w = exp2f(ml.x - M);
-    wsum += w * ml.y;
-    const float4* wo = reinterpret_cast<const float4*>(p.ws_o + (slot * TC_BM + row) * TC_D);
+  for (int d = 0; d < 8; ++d) acc[d] = 0.f;
 #pragma unroll
-    for (int d4 = 0; d4 < TC_D / 4; ++d4) {
-      const float4 v = wo[d4];
-      acc[4 * d4] += w * v.x;
-      acc[4 * d4 + 1] += w * v.y;
-      acc[4 * d4 + 2] += w * v.z;
-      acc[4 * d4 + 3] += w * v.w;
+  for (int s = 0; s < TC_MAX_SPLITS; ++s) {
+    if (s < p.splits && ml[s].x != -INFINITY) {
+      const float w = exp2f(ml[s].x - M);
+      wsum += w * ml[s].y;
+      const float4* wo =
+          reinterpret_cast<const float4*>(p.ws_o + (((size_t)unit * p.splits + s) * TC_BM + row) * TC_D + d0);
+      const float4 a = wo[0], b = wo[1];
+      acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
+      acc[4] += w * b.x; acc[5] += w * b.y; acc[6] += w * b.z; acc[7] += w * b.w;
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  __nv_bfloat16* orow = p.out + ((((size_t)layer * g.n_req + r) * g.n + node) * g.Hq + hq) * TC_D;
-#pragma unroll
-  for (int d = 0; d < TC_D; d += 8) {
-    uint4 pk;
-    pk.x = pack_bf16x2(acc[d] * inv, acc[d + 1] * inv);
-    pk.y = pack_bf16x2(acc[d + 2] * inv, acc[d + 3] * inv);
-    pk.z = pack_bf16x2(acc[d + 4] * inv, acc[d + 5] * inv);
-    pk.w = pack_bf16x2(acc[d + 6] * inv, acc[d + 7] * inv);
-    *reinterpret_cast<uint4*>(orow + d) = pk;
-  }
-  if (p.out_lse) p.out_lse[(((size_t)layer * g.n_req + r) * g.n + node) * g.Hq + hq] = (M + log2f(wsum)) * 0.6931471805599453f;
+  __nv_bfloat16* orow = p.out + ((((size_t)layer * g.n_req + r) * g.n + node) * g.Hq + hq) * TC_D + d0;
+  uint4 pk;
+  pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  pk.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  pk.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  *reinterpret_cast<uint4*>(orow) = pk;
+  if (p.out_lse && d0 == 0)
+    p.out_lse[(((size_t)layer * g.n_req + r) * g.n + node) * g.Hq + hq] = (M + log2f(wsum)) * 0.6931471805599453f;
 }
 
 // ---------------------------------------------------------------- host side
@@ -623,7 +645,7 @@ inline TcPlan tc_plan(const AttnGeom& g, int num_sms) {
   int splits = 1;
   if (pl.units < num_sms) {
     splits = num_sms / pl.units;
-    if (splits > 16) splits = 16;
+    if (splits > TC_MAX_SPLITS) splits = TC_MAX_SPLITS;
     if (splits < 1) splits = 1;
   }
   pl.splits = splits;
@@ -716,7 +738,7 @@ inline int tc_attn_launch(const void* q, const void* kc, const void* vc, const i
   tree_attn_tc_kernel<<<(unsigned)grid, TC_THREADS, TC_SMEM_BYTES, stream>>>(mq, mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return DDTREE_ERR_CUDA;
   if (pl.splits > 1) {
-    tree_attn_combine_kernel<<<pl.units, 128, 0, stream>>>(p);
+    tree_attn_combine_kernel<<<pl.units * (TC_BM / TC_COMBINE_ROWS), 128, 0, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return DDTREE_ERR_CUDA;
   }
   return DDTREE_OK;

@@ -14,13 +14,17 @@
 //
 // Design: one CTA per request.  The lp table (ranks < min(K, B)) is staged
 // in shared memory.  Warp 0 runs the queue: frontier slot s lives in
-// shared memory and belongs to lane s % 32, every lane caches the best of
-// its slots, and a pop is one `redux.sync.max` over the lanes' 32-bit order
-// keys plus a ballot.  Equal keys (equal fp32 scores) fall back to an exact
-// rank-tuple comparison that walks parent pointers.  A popped slot is
-// reused for the popped entry's next sibling, so only two lanes ever
-// rescan.  After the pops every thread writes one node row and builds its
-// ancestor bitmask by walking its parent chain (at most L+1 nodes).
+// shared memory and belongs to lane s % 32, and every lane caches its best
+// entry (order key, score, parent score, packed parent/depth/rank) in
+// registers, so a pop is one `redux.sync.max` over the lanes' 32-bit order
+// keys, a ballot and four shuffles, with no shared-memory read of the
+// popped entry.  Equal keys (exactly equal fp32 scores, common with bf16
+// logits) fall back to an exact rank-tuple comparison that walks parent
+// pointers to the common ancestor.  A popped slot is reused for the popped
+// entry's next sibling, so only the popped entry's lane rescans its slots
+// and the child's lane compares one entry.  After the pops every thread
+// writes one node row and builds its ancestor bitmask by walking its
+// parent chain (at most L+1 nodes).
 #pragma once
 
 #include "common.cuh"
@@ -45,6 +49,7 @@ struct BuildSmem {
   float* lp;          // [L][kc]
   uint32_t* fr_key;   // [B+1]
   float* fr_score;    // [B+1]
+  float* fr_pscore;   // [B+1] score of the entry's parent node
   uint32_t* fr_meta;  // [B+1]
   int* nd_parent;     // [B+1]
   int* nd_rank;       // [B+1]
@@ -52,21 +57,23 @@ struct BuildSmem {
   float* nd_score;    // [B+1]
 };
 
-// True iff the rank tuple of entry a is lexicographically smaller than b's
-// (a proper prefix is smaller than its extensions).  Tuples are rebuilt
-// from the parent chain; only used when two scores are exactly equal.
-__device__ __noinline__ bool tuple_less(uint32_t ma, uint32_t mb, const int* nd_parent,
-                                        const int* nd_rank) {
-  int ta[33], tb[33];
-  int da = meta_depth(ma), db = meta_depth(mb);
-  ta[da - 1] = meta_rank(ma);
-  for (int p = meta_parent(ma), k = da - 2; k >= 0; --k) { ta[k] = nd_rank[p]; p = nd_parent[p]; }
-  tb[db - 1] = meta_rank(mb);
-  for (int p = meta_parent(mb), k = db - 2; k >= 0; --k) { tb[k] = nd_rank[p]; p = nd_parent[p]; }
-  int n = da < db ? da : db;
-  for (int k = 0; k < n; ++k)
-    if (ta[k] != tb[k]) return ta[k] < tb[k];
-  return da < db;
+// True iff the rank tuple of frontier entry a is lexicographically smaller
+// than entry b's (a proper prefix is smaller than its extensions).  Only
+// used when two scores are exactly equal.  Walks the parent chains: lift
+// the deeper entry to the other's depth, then both to their common parent,
+// and compare the ranks just below it.
+__device__ __forceinline__ bool tuple_less(uint32_t ma, uint32_t mb, const int* nd_parent, const int* nd_rank) {
+  int pa = meta_parent(ma), ra = meta_rank(ma), da = meta_depth(ma);
+  int pb = meta_parent(mb), rb = meta_rank(mb), db = meta_depth(mb);
+  const bool a_shorter = da < db;
+  while (da > db) { ra = nd_rank[pa]; pa = nd_parent[pa]; --da; }
+  while (db > da) { rb = nd_rank[pb]; pb = nd_parent[pb]; --db; }
+  if (pa == pb && ra == rb) return a_shorter;   // one tuple is a prefix of the other
+  while (pa != pb) {
+    ra = nd_rank[pa]; pa = nd_parent[pa];
+    rb = nd_rank[pb]; pb = nd_parent[pb];
+  }
+  return ra < rb;
 }
 
 __global__ void __launch_bounds__(BUILD_THREADS)
@@ -87,6 +94,7 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
     sm.lp = (float*)p;          p += (size_t)L * kc * 4;
     sm.fr_key = (uint32_t*)p;   p += (size_t)n * 4;
     sm.fr_score = (float*)p;    p += (size_t)n * 4;
+    sm.fr_pscore = (float*)p;   p += (size_t)n * 4;
     sm.fr_meta = (uint32_t*)p;  p += (size_t)n * 4;
     sm.nd_parent = (int*)p;     p += (size_t)n * 4;
     sm.nd_rank = (int*)p;       p += (size_t)n * 4;
@@ -98,32 +106,35 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
   // stage the lp table (only ranks < kc can ever be popped)
   const float* lpr = lp + (size_t)r * L * K;
   for (int i = tid; i < L * kc; i += BUILD_THREADS) {
-    int d = i / kc, k = i - d * kc;
+    const int d = i / kc, k = i - d * kc;
     sm.lp[i] = lpr[(size_t)d * K + k];
   }
-  for (int i = tid; i < n; i += BUILD_THREADS) sm.fr_key[i] = 0;
   __syncthreads();
 
   if (tid < 32) {
     const int lane = tid;
-    // root
     if (lane == 0) {
       sm.nd_parent[0] = -1;
       sm.nd_rank[0] = -1;
       sm.nd_depth[0] = 0;
       sm.nd_score[0] = 0.f;
     }
-    int next_slot = 0;
-    uint32_t bkey = 0;
+    // this lane's best frontier entry, cached in registers (key 0: none)
+    uint32_t bkey = 0, bmeta = 0;
+    float bscore = 0.f, bpscore = 0.f;
     int bslot = -1;
-    if (B > 0) {
-      // the frontier starts with the best token of position 1
+    int next_slot = 0;
+    if (B > 0) {   // the frontier starts with the best token of position 1
       const float s0 = __fadd_rn(0.f, sm.lp[0]);
       if (lane == 0) {
         sm.fr_key[0] = score_key(s0);
         sm.fr_score[0] = s0;
+        sm.fr_pscore[0] = 0.f;
         sm.fr_meta[0] = pack_meta(0, 1, 0);
         bkey = score_key(s0);
+        bmeta = pack_meta(0, 1, 0);
+        bscore = s0;
+        bpscore = 0.f;
         bslot = 0;
       }
       next_slot = 1;
@@ -135,64 +146,77 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
       if (m == 0) break;   // frontier empty
       unsigned ties = __ballot_sync(0xffffffffu, bkey == m);
       int wl = __ffs(ties) - 1;
-      int slot = __shfl_sync(0xffffffffu, bslot, wl);
       ties &= ties - 1;
-      while (ties) {       // equal scores in several lanes: smallest rank tuple wins
-        const int l2 = __ffs(ties) - 1;
-        ties &= ties - 1;
-        const int s2 = __shfl_sync(0xffffffffu, bslot, l2);
-        if (tuple_less(sm.fr_meta[s2], sm.fr_meta[slot], sm.nd_parent, sm.nd_rank)) slot = s2;
+      if (ties) {          // equal scores in several lanes: the smallest rank tuple wins
+        uint32_t wm = __shfl_sync(0xffffffffu, bmeta, wl);
+        while (ties) {
+          const int l2 = __ffs(ties) - 1;
+          ties &= ties - 1;
+          const uint32_t m2 = __shfl_sync(0xffffffffu, bmeta, l2);
+          if (tuple_less(m2, wm, sm.nd_parent, sm.nd_rank)) { wl = l2; wm = m2; }
+        }
       }
-      const uint32_t meta = sm.fr_meta[slot];
-      const float sc = sm.fr_score[slot];
+      const uint32_t meta = __shfl_sync(0xffffffffu, bmeta, wl);
+      const float sc = __shfl_sync(0xffffffffu, bscore, wl);
+      const float ps = __shfl_sync(0xffffffffu, bpscore, wl);
+      const int slot = __shfl_sync(0xffffffffu, bslot, wl);
       const int par = meta_parent(meta), d = meta_depth(meta), rk = meta_rank(meta);
       const int node = ++pops;
+      const bool sib = rk + 1 < kc;              // next sibling: same parent, next rank
+      const bool child = d < L;                  // first child: one position deeper
+      const float lsib = sib ? sm.lp[(d - 1) * kc + rk + 1] : 0.f;
+      const float lchild = child ? sm.lp[d * kc] : 0.f;
       if (lane == 0) {
         sm.nd_parent[node] = par;
         sm.nd_rank[node] = rk;
         sm.nd_depth[node] = d;
         sm.nd_score[node] = sc;
       }
-      // next sibling replaces the popped entry in its slot
-      const bool sib = rk + 1 < kc;
-      const float ssib = sib ? __fadd_rn(sm.nd_score[par], sm.lp[(d - 1) * kc + rk + 1]) : 0.f;
-      // first child goes to a fresh slot
-      const bool child = d < L;
-      const float schild = child ? __fadd_rn(sc, sm.lp[d * kc]) : 0.f;
+      const float ssib = __fadd_rn(ps, lsib);
+      const float schild = __fadd_rn(sc, lchild);
+      const uint32_t ksib = sib ? score_key(ssib) : 0u;
+      const uint32_t kchild = score_key(schild);
+      const uint32_t msib = pack_meta(par, d, rk + 1), mchild = pack_meta(node, d + 1, 0);
       const int cslot = next_slot;
       if (child) ++next_slot;
       const int sl = slot & 31, cl = cslot & 31;
       if (lane == sl) {
-        sm.fr_key[slot] = sib ? score_key(ssib) : 0u;
+        sm.fr_key[slot] = ksib;
         sm.fr_score[slot] = ssib;
-        sm.fr_meta[slot] = pack_meta(par, d, rk + 1);
+        sm.fr_pscore[slot] = ps;
+        sm.fr_meta[slot] = msib;
       }
       if (child && lane == cl) {
-        sm.fr_key[cslot] = score_key(schild);
+        sm.fr_key[cslot] = kchild;
         sm.fr_score[cslot] = schild;
-        sm.fr_meta[cslot] = pack_meta(node, d + 1, 0);
+        sm.fr_pscore[cslot] = sc;
+        sm.fr_meta[cslot] = mchild;
       }
       __syncwarp();
-      if (lane == sl) {          // rescan this lane's slots
+      if (lane == sl) {          // this lane's best was popped: rescan its slots
         bkey = 0;
         bslot = -1;
-        for (int s = lane; s < next_slot; s += 32) {
-          const uint32_t k = sm.fr_key[s];
-          if (k > bkey || (k != 0 && k == bkey &&
-                           tuple_less(sm.fr_meta[s], sm.fr_meta[bslot], sm.nd_parent, sm.nd_rank))) {
+        for (int s2 = lane; s2 < next_slot; s2 += 32) {
+          const uint32_t k = sm.fr_key[s2];
+          if (k > bkey || (k != 0 && k == bkey && tuple_less(sm.fr_meta[s2], bmeta, sm.nd_parent, sm.nd_rank))) {
             bkey = k;
-            bslot = s;
+            bslot = s2;
+            bmeta = sm.fr_meta[s2];
           }
         }
+        if (bslot >= 0) {
+          bscore = sm.fr_score[bslot];
+          bpscore = sm.fr_pscore[bslot];
+        }
       } else if (child && lane == cl) {
-        const uint32_t k = sm.fr_key[cslot];
-        if (k > bkey || (k == bkey && tuple_less(sm.fr_meta[cslot], sm.fr_meta[bslot], sm.nd_parent,
-                                                 sm.nd_rank))) {
-          bkey = k;
+        if (kchild > bkey || (kchild == bkey && tuple_less(mchild, bmeta, sm.nd_parent, sm.nd_rank))) {
+          bkey = kchild;
           bslot = cslot;
+          bmeta = mchild;
+          bscore = schild;
+          bpscore = sc;
         }
       }
-      __syncwarp();
     }
     if (lane == 0) s_pops = pops;
   }
@@ -227,7 +251,7 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
 }
 
 inline size_t build_smem_bytes(int L, int kc, int B) {
-  return (size_t)L * kc * 4 + (size_t)(B + 1) * 4 * 7;
+  return (size_t)L * kc * 4 + (size_t)(B + 1) * 4 * 8;
 }
 
 }  // namespace ddt

@@ -81,20 +81,36 @@ int topk_launch(const void* logits, int dtype, int rows, int V, long long row_st
   int st = topk_check(logits, dtype, rows, V, row_stride, K, ids, lp);
   if (st) return st;
   TopkPlan p = topk_plan(rows, V, K, esize_of(dtype), num_sms());
-  if (p.cand > TOPK_MAX_CAND) return DDTREE_ERR_UNSUPPORTED;
+  if (p.cpr == 0 || p.cand > TOPK_MAX_CAND) return DDTREE_ERR_UNSUPPORTED;
   if (!ws || !aligned16(ws) || ws_bytes < topk_ws_bytes(rows, p)) return DDTREE_ERR_INVALID_ARG;
   TopkWs w = topk_ws_carve(ws, rows, p);
   const size_t smem = topk_smem_bytes(p, K);
   const long long grid = (long long)rows * p.cpr;
   if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
   if (dtype == DDTREE_BF16) {
-    if ((st = set_smem(topk_kernel<DDTREE_BF16>, smem))) return st;
-    topk_kernel<DDTREE_BF16><<<(unsigned)grid, TOPK_THREADS, smem, s>>>(logits, rows, V, row_stride, K, p, w,
-                                                                       ids, lp, lse);
+    switch (p.vpt) {
+#define DDT_TOPK_CASE(VP)                                                                                   \
+  case VP:                                                                                                  \
+    if ((st = set_smem(topk_kernel<DDTREE_BF16, VP>, smem))) return st;                                     \
+    topk_kernel<DDTREE_BF16, VP><<<(unsigned)grid, TOPK_THREADS, smem, s>>>(logits, rows, V, row_stride, K, \
+                                                                            p, w, ids, lp, lse);            \
+    break;
+      DDT_TOPK_CASE(1) DDT_TOPK_CASE(2) DDT_TOPK_CASE(3) DDT_TOPK_CASE(4) DDT_TOPK_CASE(5) DDT_TOPK_CASE(6)
+#undef DDT_TOPK_CASE
+      default: return DDTREE_ERR_UNSUPPORTED;
+    }
   } else {
-    if ((st = set_smem(topk_kernel<DDTREE_F32>, smem))) return st;
-    topk_kernel<DDTREE_F32><<<(unsigned)grid, TOPK_THREADS, smem, s>>>(logits, rows, V, row_stride, K, p, w,
-                                                                      ids, lp, lse);
+    switch (p.vpt) {
+#define DDT_TOPK_CASE(VP)                                                                                  \
+  case VP:                                                                                                 \
+    if ((st = set_smem(topk_kernel<DDTREE_F32, VP>, smem))) return st;                                     \
+    topk_kernel<DDTREE_F32, VP><<<(unsigned)grid, TOPK_THREADS, smem, s>>>(logits, rows, V, row_stride, K, \
+                                                                           p, w, ids, lp, lse);            \
+    break;
+      DDT_TOPK_CASE(1) DDT_TOPK_CASE(2) DDT_TOPK_CASE(3) DDT_TOPK_CASE(4) DDT_TOPK_CASE(5) DDT_TOPK_CASE(6)
+#undef DDT_TOPK_CASE
+      default: return DDTREE_ERR_UNSUPPORTED;
+    }
   }
   return launch_status();
 }
@@ -254,12 +270,24 @@ int accept_launch(const void* target_logits, int dtype, int V, long long row_str
   ArgmaxWs w = argmax_ws_carve(ws, rows);
   const long long grid = (long long)rows * p.cpr;
   if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
-  if (dtype == DDTREE_BF16)
-    argmax_kernel<DDTREE_BF16><<<(unsigned)grid, ARGMAX_THREADS, 0, s>>>(target_logits, n, V, row_stride,
-                                                                        n_nodes, p.cpr, p.chunk, w);
-  else
-    argmax_kernel<DDTREE_F32><<<(unsigned)grid, ARGMAX_THREADS, 0, s>>>(target_logits, n, V, row_stride,
-                                                                       n_nodes, p.cpr, p.chunk, w);
+  const int vpt = ceil_div(ceil_div(p.chunk, 16 / esize_of(dtype)), ARGMAX_THREADS);
+  switch (vpt) {
+#define DDT_ARGMAX_CASE(VP)                                                                               \
+  case VP:                                                                                                \
+    if (dtype == DDTREE_BF16)                                                                             \
+      argmax_kernel<DDTREE_BF16, VP><<<(unsigned)grid, ARGMAX_THREADS, 0, s>>>(target_logits, n, V,      \
+                                                                              row_stride, n_nodes, p.cpr, \
+                                                                              p.chunk, w);                \
+    else                                                                                                  \
+      argmax_kernel<DDTREE_F32, VP><<<(unsigned)grid, ARGMAX_THREADS, 0, s>>>(target_logits, n, V,       \
+                                                                             row_stride, n_nodes, p.cpr,  \
+                                                                             p.chunk, w);                 \
+    break;
+    DDT_ARGMAX_CASE(1) DDT_ARGMAX_CASE(2) DDT_ARGMAX_CASE(3) DDT_ARGMAX_CASE(4) DDT_ARGMAX_CASE(5)
+    DDT_ARGMAX_CASE(6)
+#undef DDT_ARGMAX_CASE
+    default: return DDTREE_ERR_UNSUPPORTED;
+  }
   int st = launch_status();
   if (st) return st;
   WalkArgs a;

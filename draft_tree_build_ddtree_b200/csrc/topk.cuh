@@ -5,78 +5,91 @@
 //
 // Design (HBM-bound: every logit is read once, nothing else is large):
 //  * A row of V logits is cut into `cpr` chunks; one 512-thread CTA per
-//    chunk issues all of its 128-bit loads up front into registers (at most
-//    6 vectors per thread), so one wave of CTAs keeps the whole input in
-//    flight.
-//  * Each CTA reduces its chunk to (max, sum exp(z - max)) and to its local
-//    top-K' (K' = min(K, chunk length)).  The sum is taken in fp64 (fp64
-//    exp and adds) so that log q = z - lse, rounded once to fp32, is the
-//    correctly rounded value in all but vanishingly rare cases: bf16 logits
-//    sit on a coarse grid, many prefixes tie exactly in real arithmetic, and
-//    only a correctly rounded log-prob table orders them reproducibly.  The
-//    local top-K' comes from a radix select on a unique
-//    composite key (order key of the logit, then the complemented local
-//    index so that lower ids win ties).  For bf16 the first pass is a
-//    256-bin histogram anchored at the chunk maximum: each bin is one bf16
-//    value, so one pass finds the threshold value whenever the K'-th best
-//    logit lies within 256 bf16 steps of the maximum; otherwise the generic
-//    8-bit-digit radix select runs.
-//  * The candidates go to the workspace; the last CTA of the row (atomic
-//    ticket, nobody waits) merges the row: combines the chunk sums into lse,
-//    selects the global top-K among the candidates with the same radix
-//    select, sorts them with a bitonic network and writes ids, lp, lse.
+//    chunk issues all of its 128-bit loads up front into registers (VPT
+//    vectors per thread, a template parameter), so one wave of CTAs keeps
+//    the whole input in flight.  Order keys are computed once into
+//    registers.
+//  * The chunk's sum of exp(z - max) is taken in fp64 with a table-driven
+//    exponential (Tang's method: 2^(k/64) from a table times a degree-5
+//    polynomial of the reduced argument), so that log q = z - lse, rounded
+//    once to fp32, is the correctly rounded value in all but vanishingly
+//    rare cases.  bf16 logits sit on a coarse grid, many prefixes tie
+//    exactly in real arithmetic, and only a correctly rounded log-prob
+//    table orders them reproducibly.
+//  * The chunk's threshold value (the K'-th largest logit, K' = min(K,
+//    chunk length)) comes, for bf16, from one 256-bin histogram anchored at
+//    the chunk maximum: each bin is one bf16 value, so one pass finds it
+//    whenever it lies within 256 bf16 steps of the maximum (2 octaves, 13-16%
+//    of a Gaussian row).  Otherwise (and for fp32) an 8-bit-digit radix
+//    select over the value keys runs.  Every logit >= the threshold is
+//    emitted when they fit the chunk's candidate capacity (K + min(K, 512));
+//    only then are ties at the threshold cut by lowest token id with a
+//    radix select over the complemented index.
+//  * The last CTA of the row (atomic ticket, nobody waits) merges the row:
+//    combines the chunk sums into lse, selects the top-K among the
+//    candidates (unique 64-bit keys: value key, complemented token id),
+//    sorts them with a bitonic network and writes ids, lp, lse.
 #pragma once
 
 #include "common.cuh"
+#include "exp64_table.h"
 
 namespace ddt {
 
 constexpr int TOPK_THREADS = 512;
 constexpr int TOPK_MAX_VPT = 6;            // 16-byte vectors per thread
 constexpr int TOPK_MAX_CAND = 16384;       // merge capacity (candidates per row)
+constexpr int TOPK_MAX_CPR = 128;          // chunks per row
 constexpr int TOPK_ID_BITS = 20;           // V <= 2^20
 constexpr uint32_t TOPK_ID_MASK = (1u << TOPK_ID_BITS) - 1u;
+constexpr int LID_BITS = 15;               // chunk <= 24576 < 32768
+constexpr uint32_t LID_MASK = (1u << LID_BITS) - 1u;
 
 struct TopkPlan {
-  int cpr;      // chunks per row
+  int cpr;      // chunks per row (0: unsupported)
   int chunk;    // elements per chunk (multiple of the vector width)
-  int kmax;     // candidates per chunk = min(K, chunk)
-  int cand;     // candidates per row
+  int vpt;      // 16-byte vectors per thread
+  int cap;      // candidate slots per chunk
+  int cand;     // candidate slots per row = cpr * cap
 };
+
+inline int topk_cap(int K) { return K + (K < 512 ? K : 512); }
 
 inline TopkPlan topk_plan(int rows, int V, int K, int esize, int num_sms) {
   const int epv = 16 / esize;
   const int max_chunk = TOPK_THREADS * TOPK_MAX_VPT * epv;
-  int cpr_min = ceil_div(V, max_chunk);
-  int cpr_fill = num_sms / (rows > 0 ? rows : 1);
-  if (cpr_fill < 1) cpr_fill = 1;
-  int cpr_small = ceil_div(V, 2048);
-  int cpr = cpr_fill < cpr_small ? cpr_fill : cpr_small;
-  if (cpr < cpr_min) cpr = cpr_min;
-  int chunk = ceil_div(ceil_div(V, cpr), epv) * epv;
-  cpr = ceil_div(V, chunk);
   TopkPlan p;
-  p.cpr = cpr;
-  p.chunk = chunk;
-  p.kmax = K < chunk ? K : chunk;
-  // all chunks but the last hold `chunk` elements; the last one may be short
-  int last = V - (cpr - 1) * chunk;
-  p.cand = (cpr - 1) * p.kmax + (K < last ? K : last);
+  p.cap = topk_cap(K);
+  const int cpr_min = ceil_div(V, max_chunk);
+  int cpr = num_sms / (rows > 0 ? rows : 1);
+  const int cpr_small = ceil_div(V, 2048);
+  if (cpr > cpr_small) cpr = cpr_small;
+  int cpr_cap = TOPK_MAX_CAND / p.cap;
+  if (cpr_cap > TOPK_MAX_CPR) cpr_cap = TOPK_MAX_CPR;
+  if (cpr > cpr_cap) cpr = cpr_cap;
+  if (cpr < cpr_min) cpr = cpr_min;
+  if (cpr < 1) cpr = 1;
+  p.chunk = ceil_div(ceil_div(V, cpr), epv) * epv;
+  p.cpr = ceil_div(V, p.chunk);
+  p.vpt = ceil_div(ceil_div(p.chunk, epv), TOPK_THREADS);
+  p.cand = p.cpr * p.cap;
+  if (p.cpr > cpr_cap || p.vpt > TOPK_MAX_VPT) p.cpr = 0;   // unsupported shape
   return p;
 }
 
-// Workspace of the top-K stage, per row: [ticket u32] ... then per chunk
-// (max, sumexp) float2, then the candidates (u64).
+// Workspace of the top-K stage: tickets, chunk statistics, candidate counts
+// and candidates (value key << 20 | complemented token id).
 struct TopkWs {
-  uint32_t* ticket;        // [rows]
-  double2* stats;          // [rows][cpr]: (chunk max, sum of exp(z - max)) in fp64
-  unsigned long long* cand;  // [rows][cand]
+  uint32_t* ticket;          // [rows]
+  double2* stats;            // [rows][cpr]: (chunk max, sum of exp(z - max))
+  int* count;                // [rows][cpr]
+  unsigned long long* cand;  // [rows][cpr][cap]
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 inline size_t topk_ws_bytes(int rows, const TopkPlan& p) {
-  return align256((size_t)rows * 4) + align256((size_t)rows * p.cpr * 16) +
+  return align256((size_t)rows * 4) + align256((size_t)rows * p.cpr * 16) + align256((size_t)rows * p.cpr * 4) +
          align256((size_t)rows * p.cand * 8);
 }
 
@@ -87,24 +100,51 @@ inline TopkWs topk_ws_carve(void* ws, int rows, const TopkPlan& p) {
   b += align256((size_t)rows * 4);
   w.stats = (double2*)b;
   b += align256((size_t)rows * p.cpr * 16);
+  w.count = (int*)b;
+  b += align256((size_t)rows * p.cpr * 4);
   w.cand = (unsigned long long*)b;
   return w;
 }
 
+// exp(x) in fp64 for x <= 0 (table-driven; relative error ~1e-16; 0 below -708).
+__device__ __forceinline__ double exp64_nonpos(double x, const double* tab) {
+  if (!(x > -708.0)) return 0.0;
+  const double kd = rint(x * EXP64_INV_LN2_64);
+  const int k = (int)kd;
+  double r = fma(-kd, EXP64_C1, x);
+  r = fma(-kd, EXP64_C2, r);
+  double p = fma(r, 1.0 / 120.0, 1.0 / 24.0);
+  p = fma(p, r, 1.0 / 6.0);
+  p = fma(p, r, 0.5);
+  p = fma(p, r, 1.0);
+  p *= r;                                   // exp(r) - 1
+  const double tj = tab[k & 63];
+  const double y = fma(tj, p, tj);          // 2^(j/64) * exp(r), in [0.99, 2.02)
+  return __hiloint2double(__double2hiint(y) + ((k >> 6) << 20), __double2loint(y));
+}
+
 // ---------------------------------------------------------------------------
-// Block-wide radix select over unique keys.
+// Block-wide radix selection of the need-th largest key.
 //
-// Keys hold `shift_done` undetermined low bits below an already fixed
-// `prefix`; `need` of the keys that share that prefix must be selected (the
-// keys above the prefix are selected already).  Returns the threshold t: the
-// selection is every key >= t.  `each(f)` calls f(key) for every key this
-// thread holds (0 = empty slot), so the caller controls unrolling.
+// Keys are `nbits` wide; `each(f)` calls f(key) for every key the thread
+// holds (0 = empty).  Returns t, `above` (keys above t's final prefix) and
+// `eq` (keys sharing the final prefix).  Either eq equals the remaining need
+// (early exit: every key >= t is selected, t has zero low bits) or t is the
+// exact value of the need-th key and the eq keys equal to it tie.
 // ---------------------------------------------------------------------------
+template <typename KeyT>
+struct RadixOut {
+  KeyT t;
+  int above;
+  int eq;
+};
+
 template <typename KeyT, typename Each>
-__device__ __forceinline__ KeyT radix_select(Each each, int shift_done, KeyT prefix, int need,
-                                             uint32_t* hist /*[256]*/, int* bcast /*[4]*/) {
+__device__ __forceinline__ RadixOut<KeyT> radix_kth(Each each, int nbits, int need, uint32_t* hist,
+                                                    int* bcast) {
   const int tid = threadIdx.x;
-  int shift = shift_done;
+  KeyT prefix = 0;
+  int shift = nbits, above = 0, eq = 0;
   while (shift > 0) {
     const int width = shift < 8 ? shift : 8;
     shift -= width;
@@ -112,86 +152,91 @@ __device__ __forceinline__ KeyT radix_select(Each each, int shift_done, KeyT pre
     for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     const int hi = shift + width;
-    const KeyT want = (hi >= (int)(8 * sizeof(KeyT))) ? (KeyT)0 : (prefix >> hi);
+    const bool top = hi >= (int)(8 * sizeof(KeyT));
+    const KeyT want = top ? (KeyT)0 : (prefix >> hi);
     each([&](KeyT k) {
-      const KeyT top = (hi >= (int)(8 * sizeof(KeyT))) ? (KeyT)0 : (k >> hi);
-      if (k != 0 && top == want) atomicAdd(&hist[(uint32_t)(k >> shift) & dmask], 1u);
+      if (k != 0 && (top || (k >> hi) == want)) atomicAdd(&hist[(uint32_t)(k >> shift) & dmask], 1u);
     });
     __syncthreads();
     if (tid < 32) {
-      // lane l owns digits [8l, 8l+8); find digit d with above(d) < need <= above(d) + hist[d]
       uint32_t c[8];
       uint32_t mine = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) { c[j] = hist[8 * tid + j]; mine += c[j]; }
-      uint32_t incl = mine;   // suffix sum over lanes: keys in digits >= 8*lane
+      uint32_t incl = mine;   // keys in digits >= 8*lane
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        uint32_t v = __shfl_down_sync(0xffffffffu, incl, o);
+        const uint32_t v = __shfl_down_sync(0xffffffffu, incl, o);
         if (tid + o < 32) incl += v;
       }
       const uint32_t above_lane = incl - mine;
-      const bool here = above_lane < (uint32_t)need && (uint32_t)need <= incl;
-      const unsigned m = __ballot_sync(0xffffffffu, here);
+      const unsigned m = __ballot_sync(0xffffffffu, above_lane < (uint32_t)need && (uint32_t)need <= incl);
       if (tid == __ffs(m) - 1) {
-        uint32_t above = above_lane;
-        int d = 7;
-        for (; d > 0; --d) {
-          if (above + c[d] >= (uint32_t)need) break;
-          above += c[d];
+        uint32_t ab = above_lane, cd = c[0];
+        int d = 0;
+#pragma unroll
+        for (int j = 7; j >= 0; --j) {
+          if (ab + c[j] >= (uint32_t)need) { d = j; cd = c[j]; break; }
+          ab += c[j];
         }
         bcast[0] = 8 * tid + d;
-        bcast[1] = need - (int)above;
-        bcast[2] = (int)c[d];
+        bcast[1] = (int)ab;
+        bcast[2] = (int)cd;
       }
     }
     __syncthreads();
-    const int digit = bcast[0];
-    need = bcast[1];
-    const int cnt = bcast[2];
+    const int digit = bcast[0], ab = bcast[1], cnt = bcast[2];
     __syncthreads();
     prefix |= ((KeyT)digit) << shift;
-    if (cnt == need) break;   // every key with this prefix is selected
+    need -= ab;
+    above += ab;
+    eq = cnt;
+    if (cnt == need) break;
   }
-  return prefix;
+  return RadixOut<KeyT>{prefix, above, eq};
 }
 
-// ---------------------------------------------------------------------------
-// The chunk kernel (+ merge in the last CTA of each row).
-// ---------------------------------------------------------------------------
-template <int DT>  // DDTREE_BF16 or DDTREE_F32
+template <int DT>
 struct TopkTraits;
 template <>
 struct TopkTraits<DDTREE_BF16> {
-  typedef uint32_t LKey;                 // local composite key16 << 15 | ~lid
   static constexpr int EPV = 8;
   static constexpr int KEY_BITS = 16;
 };
 template <>
 struct TopkTraits<DDTREE_F32> {
-  typedef unsigned long long LKey;       // key32 << 15 | ~lid
   static constexpr int EPV = 4;
   static constexpr int KEY_BITS = 32;
 };
 
-constexpr int LID_BITS = 15;             // chunk <= 24576 < 32768
-constexpr uint32_t LID_MASK = (1u << LID_BITS) - 1u;
-
 template <int DT>
+__device__ __forceinline__ uint32_t elem_bits(const uint4& v, int j) {
+  if (DT == DDTREE_BF16) return (u32_at(v, j >> 1) >> (16 * (j & 1))) & 0xFFFFu;
+  return u32_at(v, j);
+}
+template <int DT>
+__device__ __forceinline__ uint32_t value_key(uint32_t bits) {
+  return DT == DDTREE_BF16 ? key16_of_bf16((uint16_t)bits) : key32_of_f32(__uint_as_float(bits));
+}
+template <int DT>
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return DT == DDTREE_BF16 ? bf16_of_key16(key) : f32_of_key32(key);
+}
+
+template <int DT, int VPT>
 __global__ void __launch_bounds__(TOPK_THREADS)
-topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stride, int K,
-            TopkPlan plan, TopkWs ws, int32_t* __restrict__ out_ids, float* __restrict__ out_lp,
-            float* __restrict__ out_lse) {
+topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stride, int K, TopkPlan plan,
+            TopkWs ws, int32_t* __restrict__ out_ids, float* __restrict__ out_lp, float* __restrict__ out_lse) {
   typedef TopkTraits<DT> T;
-  typedef typename T::LKey LKey;
   constexpr int EPV = T::EPV;
-  constexpr int E = TOPK_MAX_VPT * EPV;   // elements per thread (max)
+  constexpr int E = VPT * EPV;   // elements per thread
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ uint32_t hist[256];
   __shared__ int bcast[4];
+  __shared__ uint32_t red_u[TOPK_THREADS / 32];
   __shared__ double red_d[TOPK_THREADS / 32];
-  __shared__ LKey red_k[TOPK_THREADS / 32];
+  __shared__ double s_tab[64];
   __shared__ int s_count;
   __shared__ int s_last;
 
@@ -201,30 +246,27 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   const long long c0 = (long long)c * plan.chunk;
   const int len = (int)min((long long)plan.chunk, (long long)V - c0);
   const int kloc = K < len ? K : len;
+  if (tid < 64) s_tab[tid] = EXP64_TABLE[tid];
 
-  // ---- streaming load: all vectors of this thread in flight at once ----
-  const unsigned char* base =
-      (const unsigned char*)logits + ((long long)row * row_stride + c0) * (16 / EPV);
+  // ---- streaming load: all of this thread's vectors in flight at once ----
+  const unsigned char* base = (const unsigned char*)logits + ((long long)row * row_stride + c0) * (16 / EPV);
   const int nvec_full = len / EPV;
-  uint4 vec[TOPK_MAX_VPT];
+  uint4 vec[VPT];
 #pragma unroll
-  for (int v = 0; v < TOPK_MAX_VPT; ++v) {
-    int vi = v * TOPK_THREADS + tid;
-    if (vi < nvec_full) vec[v] = ldg_stream_v4(base + (size_t)vi * 16);
-    else vec[v] = make_uint4(0, 0, 0, 0);
+  for (int v = 0; v < VPT; ++v) {
+    const int vi = v * TOPK_THREADS + tid;
+    vec[v] = vi < nvec_full ? ldg_stream_v4(base + (size_t)vi * 16) : make_uint4(0, 0, 0, 0);
   }
-  // partial tail vector (only when V is not a multiple of the vector width)
-  const int tail = len - nvec_full * EPV;
-  if (tail > 0 && (nvec_full % TOPK_THREADS) == tid && nvec_full / TOPK_THREADS < TOPK_MAX_VPT) {
+  const int tail = len - nvec_full * EPV;   // ragged end (V not a multiple of the vector width)
+  if (tail > 0 && (nvec_full % TOPK_THREADS) == tid) {
     uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;
 #pragma unroll
     for (int j = 0; j < EPV; ++j) {
       if (j < tail) {
-        uint32_t bits;
-        if (DT == DDTREE_BF16) bits = ((const uint16_t*)(base + (size_t)nvec_full * 16))[j];
-        else bits = ((const uint32_t*)(base + (size_t)nvec_full * 16))[j];
-        const int word = (DT == DDTREE_BF16) ? (j >> 1) : j;
-        const uint32_t val = (DT == DDTREE_BF16) ? (bits << (16 * (j & 1))) : bits;
+        const uint32_t bits = DT == DDTREE_BF16 ? (uint32_t)((const uint16_t*)(base + (size_t)nvec_full * 16))[j]
+                                                : ((const uint32_t*)(base + (size_t)nvec_full * 16))[j];
+        const int word = DT == DDTREE_BF16 ? (j >> 1) : j;
+        const uint32_t val = DT == DDTREE_BF16 ? (bits << (16 * (j & 1))) : bits;
         if (word == 0) w0 |= val;
         else if (word == 1) w1 |= val;
         else if (word == 2) w2 |= val;
@@ -233,63 +275,45 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
     }
     const int vt = nvec_full / TOPK_THREADS;
 #pragma unroll
-    for (int v = 0; v < TOPK_MAX_VPT; ++v)
+    for (int v = 0; v < VPT; ++v)
       if (v == vt) vec[v] = make_uint4(w0, w1, w2, w3);
   }
 
-  // ---- keys, NaN check, chunk maximum ----
-  auto raw_at = [&](int e) -> uint32_t {   // e-th element of this thread (bits)
-    const int v = e / EPV, j = e % EPV;
-    if (DT == DDTREE_BF16) return (u32_at(vec[v], j >> 1) >> (16 * (j & 1))) & 0xFFFFu;
-    return u32_at(vec[v], j);
-  };
-  auto lid_at = [&](int e) -> int { return ((e / EPV) * TOPK_THREADS + tid) * EPV + (e % EPV); };
-  auto lkey_at = [&](int e) -> LKey {
-    const int lid = lid_at(e);
-    if (lid >= len) return 0;
-    uint32_t bits = raw_at(e);
-    LKey k = (DT == DDTREE_BF16) ? (LKey)key16_of_bf16((uint16_t)bits) : (LKey)key32_of_f32(__uint_as_float(bits));
-    return (k << LID_BITS) | (LKey)(LID_MASK - (uint32_t)lid);
-  };
-
-  LKey kmax_t = 0;
+  // ---- order keys (0 = no element), NaN check, chunk maximum ----
+  uint32_t key[E];
+  uint32_t kmax = 0;
   bool nan_seen = false;
 #pragma unroll
   for (int e = 0; e < E; ++e) {
-    if (lid_at(e) < len) {
-      uint32_t bits = raw_at(e);
-      nan_seen |= (DT == DDTREE_BF16) ? bf16_is_nan((uint16_t)bits) : (__uint_as_float(bits) != __uint_as_float(bits));
-      LKey k = lkey_at(e);
-      kmax_t = k > kmax_t ? k : kmax_t;
-    }
+    const int v = e / EPV, j = e % EPV;
+    const int lid = (v * TOPK_THREADS + tid) * EPV + j;
+    const uint32_t bits = elem_bits<DT>(vec[v], j);
+    const bool ok = lid < len;
+    if (DT == DDTREE_BF16) nan_seen |= ok && bf16_is_nan((uint16_t)bits);
+    else nan_seen |= ok && (__uint_as_float(bits) != __uint_as_float(bits));
+    key[e] = ok ? value_key<DT>(bits) : 0u;
+    kmax = key[e] > kmax ? key[e] : kmax;
   }
   if (__any_sync(0xffffffffu, nan_seen) && (tid & 31) == 0) flag_status(DDTREE_STATUS_NONFINITE);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    LKey w = __shfl_xor_sync(0xffffffffu, kmax_t, o);
-    kmax_t = w > kmax_t ? w : kmax_t;
-  }
-  if ((tid & 31) == 0) red_k[tid >> 5] = kmax_t;
-  __syncthreads();
-  LKey kmax = red_k[0];
-  for (int i = 1; i < TOPK_THREADS / 32; ++i) kmax = red_k[i] > kmax ? red_k[i] : kmax;
-  const uint32_t vkey_max = (uint32_t)(kmax >> LID_BITS);
-  const float m = (DT == DDTREE_BF16) ? bf16_of_key16(vkey_max) : f32_of_key32(vkey_max);
-
-  // ---- sum of exp(z - m); for bf16 also the max-anchored window histogram ----
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if ((tid & 31) == 0) red_u[tid >> 5] = kmax;
   for (int i = tid; i < 256; i += TOPK_THREADS) hist[i] = 0;
   __syncthreads();
+  kmax = red_u[0];
+#pragma unroll
+  for (int i = 1; i < TOPK_THREADS / 32; ++i) kmax = red_u[i] > kmax ? red_u[i] : kmax;
+  const float m = key_value<DT>(kmax);
+  const double md = (double)m;
+
+  // ---- fp64 sum of exp(z - m); bf16: max-anchored window histogram ----
   double s = 0.0;
   const bool m_finite = m > -INFINITY;
-  const double md = (double)m;
 #pragma unroll
   for (int e = 0; e < E; ++e) {
-    if (lid_at(e) < len) {
-      uint32_t bits = raw_at(e);
-      float z = (DT == DDTREE_BF16) ? bf16_bits_to_f32((uint16_t)bits) : __uint_as_float(bits);
-      if (m_finite) s += exp((double)z - md);
+    if (key[e] != 0) {
+      if (m_finite) s += exp64_nonpos((double)key_value<DT>(key[e]) - md, s_tab);
       if (DT == DDTREE_BF16) {
-        uint32_t d = vkey_max - key16_of_bf16((uint16_t)bits);
+        const uint32_t d = kmax - key[e];
         if (d < 256u) atomicAdd(&hist[d], 1u);
       }
     }
@@ -299,84 +323,99 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   if ((tid & 31) == 0) red_d[tid >> 5] = s;
   __syncthreads();
 
-  // ---- local threshold ----
-  LKey thr;
-  {
+  // ---- threshold value of the chunk's K'-th largest logit ----
+  uint32_t tval = 0;
+  int above = 0, eq = 0;
+  bool found = false;
+  if (DT == DDTREE_BF16) {
+    if (tid < 32) {     // bin b holds the value kmax - b
+      uint32_t cbin[8];
+      uint32_t mine = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { cbin[j] = hist[8 * tid + j]; mine += cbin[j]; }
+      uint32_t incl = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += v;
+      }
+      const uint32_t before = incl - mine;
+      const unsigned msk = __ballot_sync(0xffffffffu, before < (uint32_t)kloc && (uint32_t)kloc <= incl);
+      if (tid == 0) bcast[3] = msk ? 1 : 0;
+      if (msk && tid == __ffs(msk) - 1) {
+        uint32_t acc = before, cb = cbin[0];
+        int j0 = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (acc + cbin[j] >= (uint32_t)kloc) { j0 = j; cb = cbin[j]; break; }
+          acc += cbin[j];
+        }
+        bcast[0] = 8 * tid + j0;
+        bcast[1] = (int)acc;
+        bcast[2] = (int)cb;
+      }
+    }
+    __syncthreads();
+    if (bcast[3]) {
+      found = true;
+      tval = kmax - (uint32_t)bcast[0];
+      above = bcast[1];
+      eq = bcast[2];
+    }
+    __syncthreads();
+  }
+  if (!found) {
     auto each = [&](auto f) {
 #pragma unroll
-      for (int e = 0; e < E; ++e) f(lkey_at(e));
+      for (int e = 0; e < E; ++e) f(key[e]);
     };
-    int shift_done = T::KEY_BITS + LID_BITS;
-    LKey prefix = 0;
-    int need = kloc;
-    bool have = false;
-    if (DT == DDTREE_BF16) {
-      // warp 0 scans the window: bin b holds the value vkey_max - b
-      if (tid < 32) {
-        uint32_t cbin[8];
-        uint32_t mine = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) { cbin[j] = hist[8 * tid + j]; mine += cbin[j]; }
-        uint32_t incl = mine;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (tid >= o) incl += v;
-        }
-        uint32_t before = incl - mine;     // count in bins < 8*tid (closer to the max)
-        bool here = before < (uint32_t)need && (uint32_t)need <= incl;
-        unsigned msk = __ballot_sync(0xffffffffu, here);
-        if (tid == 0) bcast[3] = msk ? 1 : 0;
-        if (msk && tid == __ffs(msk) - 1) {
-          uint32_t acc = before;
-          int j = 0;
-          for (; j < 7; ++j) {
-            if (acc + cbin[j] >= (uint32_t)need) break;
-            acc += cbin[j];
-          }
-          bcast[0] = 8 * tid + j;
-          bcast[1] = need - (int)acc;
-          bcast[2] = (int)cbin[j];
-        }
-      }
-      __syncthreads();
-      if (bcast[3]) {
-        const uint32_t tval = vkey_max - (uint32_t)bcast[0];
-        prefix = ((LKey)tval) << LID_BITS;
-        need = bcast[1];
-        shift_done = LID_BITS;
-        have = (bcast[2] == need);
-      }
-      __syncthreads();
-    }
-    thr = have ? prefix : radix_select<LKey>(each, shift_done, prefix, need, hist, bcast);
+    const RadixOut<uint32_t> ro = radix_kth<uint32_t>(each, T::KEY_BITS, kloc, hist, bcast);
+    tval = ro.t;
+    above = ro.above;
+    eq = ro.eq;
   }
 
-  // ---- emit the local candidates and the chunk statistics ----
+  // ---- emit candidates: every key >= tval, or cut the ties at tval by lowest id ----
+  const bool all_ties = above + eq <= plan.cap;
+  uint32_t lid_thr = 0;
+  if (!all_ties) {
+    auto each_lid = [&](auto f) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int lid = ((e / EPV) * TOPK_THREADS + tid) * EPV + (e % EPV);
+        f(key[e] == tval ? (LID_MASK - (uint32_t)lid) : 0u);
+      }
+    };
+    lid_thr = radix_kth<uint32_t>(each_lid, LID_BITS, kloc - above, hist, bcast).t;
+  }
   if (tid == 0) s_count = 0;
   __syncthreads();
   unsigned long long* cand_row = ws.cand + (size_t)row * plan.cand;
-  unsigned long long* cand = cand_row + (size_t)c * plan.kmax;
+  unsigned long long* cand = cand_row + (size_t)c * plan.cap;
 #pragma unroll
   for (int e = 0; e < E; ++e) {
-    LKey k = lkey_at(e);
-    if (k != 0 && k >= thr) {
-      int slot = atomicAdd(&s_count, 1);
-      const uint32_t vkey = (uint32_t)(k >> LID_BITS);
-      const uint32_t gid = (uint32_t)(c0 + (LID_MASK - (uint32_t)(k & LID_MASK)));
-      if (slot < kloc)
-        cand[slot] = ((unsigned long long)vkey << TOPK_ID_BITS) | (unsigned long long)(TOPK_ID_MASK - gid);
+    const uint32_t k = key[e];
+    const int lid = ((e / EPV) * TOPK_THREADS + tid) * EPV + (e % EPV);
+    const bool take =
+        k != 0 && (k > tval || (k == tval && (all_ties || (LID_MASK - (uint32_t)lid) >= lid_thr)));
+    if (take) {
+      const int slot = atomicAdd(&s_count, 1);
+      const uint32_t gid = (uint32_t)(c0 + lid);
+      if (slot < plan.cap)
+        cand[slot] = ((unsigned long long)k << TOPK_ID_BITS) | (unsigned long long)(TOPK_ID_MASK - gid);
     }
   }
+  __syncthreads();
   if (tid == 0) {
     double tot = 0.0;
     for (int i = 0; i < TOPK_THREADS / 32; ++i) tot += red_d[i];
     ws.stats[(size_t)row * plan.cpr + c] = make_double2(md, tot);
+    ws.count[(size_t)row * plan.cpr + c] = s_count < plan.cap ? s_count : plan.cap;
   }
   __threadfence();
   __syncthreads();
   if (tid == 0) {
-    unsigned t = atomicAdd(&ws.ticket[row], 1u);
+    const unsigned t = atomicAdd(&ws.ticket[row], 1u);
     s_last = (t == (unsigned)(plan.cpr - 1));
   }
   __syncthreads();
@@ -384,44 +423,57 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   __threadfence();
 
   // =================== merge (last CTA of this row) ===================
-  unsigned long long* sc = (unsigned long long*)smem_raw;           // [plan.cand]
+  unsigned long long* sc = (unsigned long long*)smem_raw;   // [plan.cand]
   int kpow = 1;
   while (kpow < K) kpow <<= 1;
-  unsigned long long* win = sc + plan.cand;                         // [kpow]
-  const int ncand = plan.cand;
-  for (int i = tid; i < ncand; i += TOPK_THREADS) sc[i] = __ldcg(cand_row + i);
-  for (int i = tid; i < kpow; i += TOPK_THREADS) win[i] = 0ull;
-  if (tid == 0) s_count = 0;
+  unsigned long long* win = sc + plan.cand;                 // [kpow]
+  __shared__ int s_off[TOPK_MAX_CPR];
+  __shared__ int s_cnt[TOPK_MAX_CPR];
+  __shared__ int s_ncand;
   __shared__ double s_lse;
   if (tid == 0) {
+    int off = 0;
     double M = -INFINITY;
-    for (int i = 0; i < plan.cpr; ++i) M = fmax(M, __ldcg(&ws.stats[(size_t)row * plan.cpr + i].x));
+    for (int i = 0; i < plan.cpr; ++i) {
+      s_off[i] = off;
+      s_cnt[i] = __ldcg(&ws.count[(size_t)row * plan.cpr + i]);
+      off += s_cnt[i];
+      M = fmax(M, __ldcg(&ws.stats[(size_t)row * plan.cpr + i].x));
+    }
+    s_ncand = off;
     double S = 0.0;
     if (M > -INFINITY) {
       for (int i = 0; i < plan.cpr; ++i) {
-        double2 st = __ldcg(&ws.stats[(size_t)row * plan.cpr + i]);
-        if (st.x > -INFINITY) S += st.y * exp(st.x - M);
+        const double2 st = __ldcg(&ws.stats[(size_t)row * plan.cpr + i]);
+        if (st.x > -INFINITY) S += st.y * exp64_nonpos(st.x - M, s_tab);
       }
     }
     s_lse = M + log(S);
     ws.ticket[row] = 0;   // leave the workspace ready for the next call
   }
+  for (int i = tid; i < kpow; i += TOPK_THREADS) win[i] = 0ull;
   __syncthreads();
-
+  for (int ci = 0; ci < plan.cpr; ++ci) {
+    const unsigned long long* src = cand_row + (size_t)ci * plan.cap;
+    for (int i = tid; i < s_cnt[ci]; i += TOPK_THREADS) sc[s_off[ci] + i] = __ldcg(src + i);
+  }
+  if (tid == 0) s_count = 0;
+  __syncthreads();
+  const int ncand = s_ncand;
   const int per = (ncand + TOPK_THREADS - 1) / TOPK_THREADS;
-  auto gget = [&](int i) -> unsigned long long {
-    int idx = i * TOPK_THREADS + tid;
-    return idx < ncand ? sc[idx] : 0ull;
-  };
-  const int gbits = T::KEY_BITS + TOPK_ID_BITS;
   auto geach = [&](auto f) {
-    for (int i = 0; i < per; ++i) f(gget(i));
+    for (int i = 0; i < per; ++i) {
+      const int idx = i * TOPK_THREADS + tid;
+      f(idx < ncand ? sc[idx] : 0ull);
+    }
   };
-  unsigned long long gthr = radix_select<unsigned long long>(geach, gbits, 0ull, K, hist, bcast);
+  const unsigned long long gt =
+      radix_kth<unsigned long long>(geach, T::KEY_BITS + TOPK_ID_BITS, K, hist, bcast).t;
   for (int i = 0; i < per; ++i) {
-    unsigned long long k = gget(i);
-    if (k != 0 && k >= gthr) {
-      int slot = atomicAdd(&s_count, 1);
+    const int idx = i * TOPK_THREADS + tid;
+    const unsigned long long k = idx < ncand ? sc[idx] : 0ull;
+    if (k != 0 && k >= gt) {
+      const int slot = atomicAdd(&s_count, 1);
       if (slot < kpow) win[slot] = k;
     }
   }
@@ -430,10 +482,10 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   for (int size = 2; size <= kpow; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       for (int i = tid; i < kpow / 2; i += TOPK_THREADS) {
-        int lo = 2 * stride * (i / stride) + (i % stride);
-        int hi = lo + stride;
-        bool desc = ((lo & size) == 0);
-        unsigned long long a = win[lo], b = win[hi];
+        const int lo = 2 * stride * (i / stride) + (i % stride);
+        const int hi = lo + stride;
+        const bool desc = ((lo & size) == 0);
+        const unsigned long long a = win[lo], b = win[hi];
         if ((a < b) == desc) { win[lo] = b; win[hi] = a; }
       }
       __syncthreads();
@@ -441,12 +493,10 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   }
   const double lse = s_lse;
   for (int i = tid; i < K; i += TOPK_THREADS) {
-    unsigned long long k = win[i];
-    uint32_t vkey = (uint32_t)(k >> TOPK_ID_BITS);
-    int id = (int)(TOPK_ID_MASK - (uint32_t)(k & TOPK_ID_MASK));
-    float z = (DT == DDTREE_BF16) ? bf16_of_key16(vkey) : f32_of_key32(vkey);
-    out_ids[(size_t)row * K + i] = id;
-    out_lp[(size_t)row * K + i] = (float)((double)z - lse);   // one rounding of the fp64 value
+    const unsigned long long k = win[i];
+    const uint32_t vkey = (uint32_t)(k >> TOPK_ID_BITS);
+    out_ids[(size_t)row * K + i] = (int)(TOPK_ID_MASK - (uint32_t)(k & TOPK_ID_MASK));
+    out_lp[(size_t)row * K + i] = (float)((double)key_value<DT>(vkey) - lse);   // one rounding of the fp64 value
   }
   if (out_lse != nullptr && tid == 0) out_lse[row] = (float)lse;
 }

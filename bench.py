@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="launch rounds eagerly instead of CUDA graphs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="profiling driver: one input set, warmup + steps eager rounds, no timing")
     return ap.parse_args()
 
 
@@ -539,10 +541,29 @@ def run_reference(a):
     print(json.dumps(line))
 
 
+def run_profile(a):
+    """A small, untimed run for ncu: one input set, then warmup + steps eager rounds.
+
+    Kernel launch order: per input-set setup one top-K and one build, then per
+    round top-K, build, tree attention (+ combine when split), argmax, walk.
+    """
+    import draft_tree_build_ddtree_b200 as dd
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    w = workload_from_args(a)
+    rb = make_sets(w, 1, device)[0]
+    for _ in range(a.warmup + a.steps):
+        dd.ddtree_round(rb, rb._args)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_run": w.name, "rounds": a.warmup + a.steps, "device_status": dd.device_status()}))
+
+
 def main():
     a = parse()
     if a.impl == "reference":
         run_reference(a)
+    elif a.profile:
+        run_profile(a)
     else:
         run_ours(a)
 

@@ -16,11 +16,13 @@
 // in shared memory.  Warp 0 runs the queue: frontier slot s lives in
 // shared memory and belongs to lane s % 32, and every lane caches its best
 // entry (order key, score, parent score, packed parent/depth/rank) in
-// registers, so a pop is one `redux.sync.max` over the lanes' 32-bit order
-// keys, a ballot and four shuffles, with no shared-memory read of the
-// popped entry.  Equal keys (exactly equal fp32 scores, common with bf16
-// logits) fall back to an exact rank-tuple comparison that walks parent
-// pointers to the common ancestor.  A popped slot is reused for the popped
+// registers.  The order key of an entry is 64 bits: the fp32 score's order
+// key, then a tie key that packs the tuple's first ranks (exactly equal fp32
+// scores are common with bf16 logits: 45-65% of popped prefixes share a
+// score).  A pop is two `redux.sync.max` rounds and a ballot plus four
+// shuffles, with no shared-memory read of the popped entry; only entries
+// that agree on score and on every packed rank fall back to an exact
+// rank-tuple comparison that walks parent pointers to the common ancestor.  A popped slot is reused for the popped
 // entry's next sibling, so only the popped entry's lane rescans its slots
 // and the child's lane compares one entry.  After the pops every thread
 // writes one node row and builds its ancestor bitmask by walking its
@@ -47,7 +49,7 @@ __device__ __forceinline__ uint32_t score_key(float s) { return key32_of_f32(s);
 
 struct BuildSmem {
   float* lp;          // [L][kc]
-  uint32_t* fr_key;   // [B+1]
+  uint2* fr_key;      // [B+1] (score key, tie key); (0,0) = empty slot
   float* fr_score;    // [B+1]
   float* fr_pscore;   // [B+1] score of the entry's parent node
   uint32_t* fr_meta;  // [B+1]
@@ -57,11 +59,22 @@ struct BuildSmem {
   float* nd_score;    // [B+1]
 };
 
-// True iff the rank tuple of frontier entry a is lexicographically smaller
-// than entry b's (a proper prefix is smaller than its extensions).  Only
-// used when two scores are exactly equal.  Walks the parent chains: lift
-// the deeper entry to the other's depth, then both to their common parent,
-// and compare the ranks just below it.
+// Tie key: the first `tdepth` ranks of the tuple packed as (rank + 1) in
+// `tbits`-bit fields, most significant first, absent depths 0, then
+// complemented.  Between entries with equal scores, a larger tie key means a
+// lexicographically smaller tuple (a proper prefix is smaller than its
+// extensions); equal tie keys mean the first tdepth ranks agree.
+struct TieCode {
+  int tbits, tdepth;
+  __device__ __forceinline__ uint32_t unit(int depth) const {   // +1 at the field of this depth (1-based)
+    return depth <= tdepth ? (1u << (tbits * (tdepth - depth))) : 0u;
+  }
+};
+
+// Exact lexicographic comparison of two frontier entries' rank tuples (a
+// proper prefix is smaller), for the rare case of equal scores and equal tie
+// keys.  Walks the parent chains: lift the deeper entry to the other's depth,
+// then both to their common parent, and compare the ranks just below it.
 __device__ __forceinline__ bool tuple_less(uint32_t ma, uint32_t mb, const int* nd_parent, const int* nd_rank) {
   int pa = meta_parent(ma), ra = meta_rank(ma), da = meta_depth(ma);
   int pb = meta_parent(mb), rb = meta_rank(mb), db = meta_depth(mb);
@@ -76,9 +89,18 @@ __device__ __forceinline__ bool tuple_less(uint32_t ma, uint32_t mb, const int* 
   return ra < rb;
 }
 
+// a before b in the pop order: larger score key, then larger tie key, then
+// (both equal) the smaller rank tuple.
+__device__ __forceinline__ bool entry_before(uint2 ka, uint32_t ma, uint2 kb, uint32_t mb, const int* nd_parent,
+                                             const int* nd_rank) {
+  if (ka.x != kb.x) return ka.x > kb.x;
+  if (ka.y != kb.y) return ka.y > kb.y;
+  return tuple_less(ma, mb, nd_parent, nd_rank);
+}
+
 __global__ void __launch_bounds__(BUILD_THREADS)
 build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
-             const int32_t* __restrict__ root_token, int L, int K, int B, int kc,
+             const int32_t* __restrict__ root_token, int L, int K, int B, int kc, TieCode tc,
              int32_t* __restrict__ node_token, int32_t* __restrict__ parent,
              int32_t* __restrict__ depth, int32_t* __restrict__ node_rank,
              float* __restrict__ score, uint32_t* __restrict__ anc, int32_t* __restrict__ n_nodes) {
@@ -91,8 +113,8 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
   BuildSmem sm;
   {
     unsigned char* p = smem_raw;
+    sm.fr_key = (uint2*)p;      p += (size_t)n * 8;
     sm.lp = (float*)p;          p += (size_t)L * kc * 4;
-    sm.fr_key = (uint32_t*)p;   p += (size_t)n * 4;
     sm.fr_score = (float*)p;    p += (size_t)n * 4;
     sm.fr_pscore = (float*)p;   p += (size_t)n * 4;
     sm.fr_meta = (uint32_t*)p;  p += (size_t)n * 4;
@@ -119,35 +141,38 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
       sm.nd_depth[0] = 0;
       sm.nd_score[0] = 0.f;
     }
-    // this lane's best frontier entry, cached in registers (key 0: none)
-    uint32_t bkey = 0, bmeta = 0;
+    // this lane's best frontier entry, cached in registers (bkey (0,0): none)
+    uint2 bkey = make_uint2(0u, 0u);
+    uint32_t bmeta = 0;
     float bscore = 0.f, bpscore = 0.f;
     int bslot = -1;
     int next_slot = 0;
     if (B > 0) {   // the frontier starts with the best token of position 1
       const float s0 = __fadd_rn(0.f, sm.lp[0]);
       if (lane == 0) {
-        sm.fr_key[0] = score_key(s0);
-        sm.fr_score[0] = s0;
-        sm.fr_pscore[0] = 0.f;
-        sm.fr_meta[0] = pack_meta(0, 1, 0);
-        bkey = score_key(s0);
+        bkey = make_uint2(score_key(s0), ~tc.unit(1));
         bmeta = pack_meta(0, 1, 0);
         bscore = s0;
         bpscore = 0.f;
         bslot = 0;
+        sm.fr_key[0] = bkey;
+        sm.fr_score[0] = s0;
+        sm.fr_pscore[0] = 0.f;
+        sm.fr_meta[0] = bmeta;
       }
       next_slot = 1;
     }
     __syncwarp();
     int pops = 0;
     while (pops < B) {
-      const uint32_t m = __reduce_max_sync(0xffffffffu, bkey);
-      if (m == 0) break;   // frontier empty
-      unsigned ties = __ballot_sync(0xffffffffu, bkey == m);
+      // the frontier's best entry: max score key, then max tie key, then (rare) tuple walk
+      const uint32_t mhi = __reduce_max_sync(0xffffffffu, bkey.x);
+      if (mhi == 0) break;   // frontier empty
+      const uint32_t mlo = __reduce_max_sync(0xffffffffu, bkey.x == mhi ? bkey.y : 0u);
+      unsigned ties = __ballot_sync(0xffffffffu, bkey.x == mhi && bkey.y == mlo);
       int wl = __ffs(ties) - 1;
       ties &= ties - 1;
-      if (ties) {          // equal scores in several lanes: the smallest rank tuple wins
+      if (ties) {
         uint32_t wm = __shfl_sync(0xffffffffu, bmeta, wl);
         while (ties) {
           const int l2 = __ffs(ties) - 1;
@@ -160,6 +185,7 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
       const float sc = __shfl_sync(0xffffffffu, bscore, wl);
       const float ps = __shfl_sync(0xffffffffu, bpscore, wl);
       const int slot = __shfl_sync(0xffffffffu, bslot, wl);
+      const uint32_t packed = ~mlo;                         // the popped entry's packed ranks
       const int par = meta_parent(meta), d = meta_depth(meta), rk = meta_rank(meta);
       const int node = ++pops;
       const bool sib = rk + 1 < kc;              // next sibling: same parent, next rank
@@ -174,8 +200,8 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
       }
       const float ssib = __fadd_rn(ps, lsib);
       const float schild = __fadd_rn(sc, lchild);
-      const uint32_t ksib = sib ? score_key(ssib) : 0u;
-      const uint32_t kchild = score_key(schild);
+      const uint2 ksib = sib ? make_uint2(score_key(ssib), ~(packed + tc.unit(d))) : make_uint2(0u, 0u);
+      const uint2 kchild = make_uint2(score_key(schild), ~(packed + tc.unit(d + 1)));
       const uint32_t msib = pack_meta(par, d, rk + 1), mchild = pack_meta(node, d + 1, 0);
       const int cslot = next_slot;
       if (child) ++next_slot;
@@ -194,11 +220,12 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
       }
       __syncwarp();
       if (lane == sl) {          // this lane's best was popped: rescan its slots
-        bkey = 0;
+        bkey = make_uint2(0u, 0u);
         bslot = -1;
         for (int s2 = lane; s2 < next_slot; s2 += 32) {
-          const uint32_t k = sm.fr_key[s2];
-          if (k > bkey || (k != 0 && k == bkey && tuple_less(sm.fr_meta[s2], bmeta, sm.nd_parent, sm.nd_rank))) {
+          const uint2 k = sm.fr_key[s2];
+          if (k.x == 0) continue;
+          if (bslot < 0 || entry_before(k, sm.fr_meta[s2], bkey, bmeta, sm.nd_parent, sm.nd_rank)) {
             bkey = k;
             bslot = s2;
             bmeta = sm.fr_meta[s2];
@@ -209,7 +236,7 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
           bpscore = sm.fr_pscore[bslot];
         }
       } else if (child && lane == cl) {
-        if (kchild > bkey || (kchild == bkey && tuple_less(mchild, bmeta, sm.nd_parent, sm.nd_rank))) {
+        if (bslot < 0 || entry_before(kchild, mchild, bkey, bmeta, sm.nd_parent, sm.nd_rank)) {
           bkey = kchild;
           bslot = cslot;
           bmeta = mchild;
@@ -250,8 +277,17 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
   if (tid == 0) n_nodes[r] = nn;
 }
 
+inline TieCode tie_code(int kc, int L) {
+  TieCode t;
+  t.tbits = 1;
+  while ((1 << t.tbits) <= kc) ++t.tbits;      // fields hold rank + 1 <= kc
+  t.tdepth = 32 / t.tbits;
+  if (t.tdepth > L) t.tdepth = L;
+  return t;
+}
+
 inline size_t build_smem_bytes(int L, int kc, int B) {
-  return (size_t)L * kc * 4 + (size_t)(B + 1) * 4 * 8;
+  return (size_t)L * kc * 4 + (size_t)(B + 1) * (8 + 4 * 7);
 }
 
 }  // namespace ddt

@@ -126,8 +126,8 @@ int build_launch(const int32_t* ids, const float* lp, const int32_t* root_token,
   const size_t smem = build_smem_bytes(L, kc, B);
   int st = set_smem(build_kernel, smem);
   if (st) return st;
-  build_kernel<<<n_req, BUILD_THREADS, smem, s>>>(ids, lp, root_token, L, K, B, kc, node_token, parent, depth,
-                                                   node_rank, score, anc, n_nodes);
+  build_kernel<<<n_req, BUILD_THREADS, smem, s>>>(ids, lp, root_token, L, K, B, kc, tie_code(kc, L), node_token,
+                                                   parent, depth, node_rank, score, anc, n_nodes);
   return launch_status();
 }
 

@@ -5,10 +5,12 @@
 //
 // Design (HBM-bound: every logit is read once, nothing else is large):
 //  * A row of V logits is cut into `cpr` chunks; one 512-thread CTA per
-//    chunk issues all of its 128-bit loads up front into registers (VPT
-//    vectors per thread, a template parameter), so one wave of CTAs keeps
-//    the whole input in flight.  Order keys are computed once into
-//    registers.
+//    chunk issues all of its 128-bit loads up front (VPT vectors per
+//    thread, a template parameter), so one wave of CTAs keeps the whole
+//    input in flight, and stages the chunk in shared memory.  The passes
+//    over it are rolled loops over 16-byte vectors, which keeps the kernel's
+//    code small enough to stay in the instruction cache (fully unrolled
+//    register passes stalled on instruction fetch).
 //  * The chunk's sum of exp(z - max) is taken in fp64 with a table-driven
 //    exponential (Tang's method: 2^(k/64) from a table times a degree-5
 //    polynomial of the reduced argument), so that log q = z - lse, rounded
@@ -229,7 +231,6 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
             TopkWs ws, int32_t* __restrict__ out_ids, float* __restrict__ out_lp, float* __restrict__ out_lse) {
   typedef TopkTraits<DT> T;
   constexpr int EPV = T::EPV;
-  constexpr int E = VPT * EPV;   // elements per thread
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ uint32_t hist[256];
@@ -247,57 +248,64 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   const int len = (int)min((long long)plan.chunk, (long long)V - c0);
   const int kloc = K < len ? K : len;
   if (tid < 64) s_tab[tid] = EXP64_TABLE[tid];
+  for (int i = tid; i < 256; i += TOPK_THREADS) hist[i] = 0;
 
-  // ---- streaming load: all of this thread's vectors in flight at once ----
+  // ---- streaming load: every vector of this thread in flight at once, then staged in shared memory ----
   const unsigned char* base = (const unsigned char*)logits + ((long long)row * row_stride + c0) * (16 / EPV);
   const int nvec_full = len / EPV;
-  uint4 vec[VPT];
+  const int tail = len - nvec_full * EPV;          // ragged end (V not a multiple of the vector width)
+  const int nvec = nvec_full + (tail > 0 ? 1 : 0);
+  uint4* chunk_s = reinterpret_cast<uint4*>(smem_raw);
+  {
+    uint4 vec[VPT];
 #pragma unroll
-  for (int v = 0; v < VPT; ++v) {
-    const int vi = v * TOPK_THREADS + tid;
-    vec[v] = vi < nvec_full ? ldg_stream_v4(base + (size_t)vi * 16) : make_uint4(0, 0, 0, 0);
-  }
-  const int tail = len - nvec_full * EPV;   // ragged end (V not a multiple of the vector width)
-  if (tail > 0 && (nvec_full % TOPK_THREADS) == tid) {
-    uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;
-#pragma unroll
-    for (int j = 0; j < EPV; ++j) {
-      if (j < tail) {
-        const uint32_t bits = DT == DDTREE_BF16 ? (uint32_t)((const uint16_t*)(base + (size_t)nvec_full * 16))[j]
-                                                : ((const uint32_t*)(base + (size_t)nvec_full * 16))[j];
-        const int word = DT == DDTREE_BF16 ? (j >> 1) : j;
-        const uint32_t val = DT == DDTREE_BF16 ? (bits << (16 * (j & 1))) : bits;
-        if (word == 0) w0 |= val;
-        else if (word == 1) w1 |= val;
-        else if (word == 2) w2 |= val;
-        else w3 |= val;
-      }
+    for (int v = 0; v < VPT; ++v) {
+      const int vi = v * TOPK_THREADS + tid;
+      vec[v] = vi < nvec_full ? ldg_stream_v4(base + (size_t)vi * 16) : make_uint4(0, 0, 0, 0);
     }
-    const int vt = nvec_full / TOPK_THREADS;
 #pragma unroll
-    for (int v = 0; v < VPT; ++v)
-      if (v == vt) vec[v] = make_uint4(w0, w1, w2, w3);
+    for (int v = 0; v < VPT; ++v) {
+      const int vi = v * TOPK_THREADS + tid;
+      if (vi < nvec_full) chunk_s[vi] = vec[v];
+    }
   }
+  if (tail > 0 && tid == 0) {
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    for (int j = 0; j < tail; ++j) {
+      if (DT == DDTREE_BF16) w[j >> 1] |= (uint32_t)((const uint16_t*)(base + (size_t)nvec_full * 16))[j] << (16 * (j & 1));
+      else w[j] = ((const uint32_t*)(base + (size_t)nvec_full * 16))[j];
+    }
+    chunk_s[nvec_full] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  __syncthreads();
 
-  // ---- order keys (0 = no element), NaN check, chunk maximum ----
-  uint32_t key[E];
+  // Element e of vector vi is logit c0 + vi*EPV + e; its order key is 0 past the chunk end.
+  auto keys_of = [&](int vi, uint32_t* k) {
+    const uint4 v = chunk_s[vi];
+#pragma unroll
+    for (int j = 0; j < EPV; ++j)
+      k[j] = (vi * EPV + j < len) ? value_key<DT>(elem_bits<DT>(v, j)) : 0u;
+  };
+
+  // ---- NaN check and chunk maximum ----
   uint32_t kmax = 0;
   bool nan_seen = false;
+  for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+    const uint4 v = chunk_s[vi];
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const int v = e / EPV, j = e % EPV;
-    const int lid = (v * TOPK_THREADS + tid) * EPV + j;
-    const uint32_t bits = elem_bits<DT>(vec[v], j);
-    const bool ok = lid < len;
-    if (DT == DDTREE_BF16) nan_seen |= ok && bf16_is_nan((uint16_t)bits);
-    else nan_seen |= ok && (__uint_as_float(bits) != __uint_as_float(bits));
-    key[e] = ok ? value_key<DT>(bits) : 0u;
-    kmax = key[e] > kmax ? key[e] : kmax;
+    for (int j = 0; j < EPV; ++j) {
+      if (vi * EPV + j < len) {
+        const uint32_t bits = elem_bits<DT>(v, j);
+        if (DT == DDTREE_BF16) nan_seen |= bf16_is_nan((uint16_t)bits);
+        else nan_seen |= __uint_as_float(bits) != __uint_as_float(bits);
+        const uint32_t k = value_key<DT>(bits);
+        kmax = k > kmax ? k : kmax;
+      }
+    }
   }
   if (__any_sync(0xffffffffu, nan_seen) && (tid & 31) == 0) flag_status(DDTREE_STATUS_NONFINITE);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
   if ((tid & 31) == 0) red_u[tid >> 5] = kmax;
-  for (int i = tid; i < 256; i += TOPK_THREADS) hist[i] = 0;
   __syncthreads();
   kmax = red_u[0];
 #pragma unroll
@@ -308,13 +316,17 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   // ---- fp64 sum of exp(z - m); bf16: max-anchored window histogram ----
   double s = 0.0;
   const bool m_finite = m > -INFINITY;
+  for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+    uint32_t k[EPV];
+    keys_of(vi, k);
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    if (key[e] != 0) {
-      if (m_finite) s += exp64_nonpos((double)key_value<DT>(key[e]) - md, s_tab);
-      if (DT == DDTREE_BF16) {
-        const uint32_t d = kmax - key[e];
-        if (d < 256u) atomicAdd(&hist[d], 1u);
+    for (int j = 0; j < EPV; ++j) {
+      if (k[j] != 0) {
+        if (m_finite) s += exp64_nonpos((double)key_value<DT>(k[j]) - md, s_tab);
+        if (DT == DDTREE_BF16) {
+          const uint32_t d = kmax - k[j];
+          if (d < 256u) atomicAdd(&hist[d], 1u);
+        }
       }
     }
   }
@@ -366,8 +378,12 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   }
   if (!found) {
     auto each = [&](auto f) {
+      for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+        uint32_t k[EPV];
+        keys_of(vi, k);
 #pragma unroll
-      for (int e = 0; e < E; ++e) f(key[e]);
+        for (int j = 0; j < EPV; ++j) f(k[j]);
+      }
     };
     const RadixOut<uint32_t> ro = radix_kth<uint32_t>(each, T::KEY_BITS, kloc, hist, bcast);
     tval = ro.t;
@@ -380,10 +396,11 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   uint32_t lid_thr = 0;
   if (!all_ties) {
     auto each_lid = [&](auto f) {
+      for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+        uint32_t k[EPV];
+        keys_of(vi, k);
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const int lid = ((e / EPV) * TOPK_THREADS + tid) * EPV + (e % EPV);
-        f(key[e] == tval ? (LID_MASK - (uint32_t)lid) : 0u);
+        for (int j = 0; j < EPV; ++j) f(k[j] == tval ? (LID_MASK - (uint32_t)(vi * EPV + j)) : 0u);
       }
     };
     lid_thr = radix_kth<uint32_t>(each_lid, LID_BITS, kloc - above, hist, bcast).t;
@@ -392,17 +409,20 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   __syncthreads();
   unsigned long long* cand_row = ws.cand + (size_t)row * plan.cand;
   unsigned long long* cand = cand_row + (size_t)c * plan.cap;
+  for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+    uint32_t k[EPV];
+    keys_of(vi, k);
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const uint32_t k = key[e];
-    const int lid = ((e / EPV) * TOPK_THREADS + tid) * EPV + (e % EPV);
-    const bool take =
-        k != 0 && (k > tval || (k == tval && (all_ties || (LID_MASK - (uint32_t)lid) >= lid_thr)));
-    if (take) {
-      const int slot = atomicAdd(&s_count, 1);
-      const uint32_t gid = (uint32_t)(c0 + lid);
-      if (slot < plan.cap)
-        cand[slot] = ((unsigned long long)k << TOPK_ID_BITS) | (unsigned long long)(TOPK_ID_MASK - gid);
+    for (int j = 0; j < EPV; ++j) {
+      const int lid = vi * EPV + j;
+      const bool take =
+          k[j] != 0 && (k[j] > tval || (k[j] == tval && (all_ties || (LID_MASK - (uint32_t)lid) >= lid_thr)));
+      if (take) {
+        const int slot = atomicAdd(&s_count, 1);
+        const uint32_t gid = (uint32_t)(c0 + lid);
+        if (slot < plan.cap)
+          cand[slot] = ((unsigned long long)k[j] << TOPK_ID_BITS) | (unsigned long long)(TOPK_ID_MASK - gid);
+      }
     }
   }
   __syncthreads();
@@ -422,7 +442,7 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   if (!s_last) return;
   __threadfence();
 
-  // =================== merge (last CTA of this row) ===================
+  // =================== merge (last CTA of this row; the staged chunk is dead) ===================
   unsigned long long* sc = (unsigned long long*)smem_raw;   // [plan.cand]
   int kpow = 1;
   while (kpow < K) kpow <<= 1;
@@ -451,8 +471,8 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
     s_lse = M + log(S);
     ws.ticket[row] = 0;   // leave the workspace ready for the next call
   }
-  for (int i = tid; i < kpow; i += TOPK_THREADS) win[i] = 0ull;
   __syncthreads();
+  for (int i = tid; i < kpow; i += TOPK_THREADS) win[i] = 0ull;
   for (int ci = 0; ci < plan.cpr; ++ci) {
     const unsigned long long* src = cand_row + (size_t)ci * plan.cap;
     for (int i = tid; i < s_cnt[ci]; i += TOPK_THREADS) sc[s_off[ci] + i] = __ldcg(src + i);
@@ -501,10 +521,13 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   if (out_lse != nullptr && tid == 0) out_lse[row] = (float)lse;
 }
 
+// Dynamic shared memory: the staged chunk, later reused by the merge.
 inline size_t topk_smem_bytes(const TopkPlan& p, int K) {
   int kpow = 1;
   while (kpow < K) kpow <<= 1;
-  return (size_t)(p.cand + kpow) * 8;
+  const size_t merge = (size_t)(p.cand + kpow) * 8;
+  const size_t chunk = (size_t)(p.chunk + 16) * 4;    // worst case fp32 elements, + one ragged vector
+  return merge > chunk ? merge : chunk;
 }
 
 }  // namespace ddt

@@ -81,6 +81,7 @@ _SIGS = {
     "ddtree_status_string": (ctypes.c_char_p, [_i]),
     "ddtree_device_status": (_i, [_vp, ctypes.POINTER(ctypes.c_uint)]),
     "ddtree_version": (_i, []),
+    "ddtree_topk_static_ws": (_i, [_vp, _i, _i, _i, _ll, _i, _vp, _vp, _vp, _vp]),
 }
 
 

@@ -422,6 +422,7 @@ const char* ddtree_status_string(int status) {
     case DDTREE_ERR_NONFINITE: return "non-finite logits";
     case DDTREE_ERR_TIMEOUT: return "bounded wait timed out";
     case DDTREE_ERR_CAPACITY: return "prefix plus tree exceeds the KV cache";
+    case DDTREE_ERR_SCRATCH_LIMIT: return "request needs more than the built-in 4 MiB scratch";
     default: return "unknown status";
   }
 }
@@ -437,5 +438,55 @@ int ddtree_device_status(cudaStream_t stream, unsigned int* bits) {
 }
 
 int ddtree_version(void) { return 100; }
+
+}  // extern "C"
+
+// ----------------------------------------------------------------------
+// Top-K with built-in scratch, for callers that cannot allocate device
+// memory while they run (see ddtree_topk_static_ws in ddtree.h).
+// ----------------------------------------------------------------------
+namespace {
+
+constexpr size_t STATIC_SCRATCH_BYTES = (size_t)4 << 20;   // 4 MiB per device
+constexpr int STATIC_SCRATCH_MAX_DEVICES = 64;
+
+// The scratch array itself.  In host code its name is only a stand-in:
+// kernels get the device address looked up below, never the symbol.
+__device__ __align__(256) unsigned char g_topk_static_scratch[STATIC_SCRATCH_BYTES];
+
+void* g_static_scratch_ptr[STATIC_SCRATCH_MAX_DEVICES];
+
+// Device address of the scratch array on the current device, looked up once
+// per device (nullptr on failure).
+void* static_scratch_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= STATIC_SCRATCH_MAX_DEVICES) return nullptr;
+  if (g_static_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_topk_static_scratch) != cudaSuccess) return nullptr;
+    g_static_scratch_ptr[dev] = ptr;
+  }
+  return g_static_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int ddtree_topk_static_ws(const void* logits, int dtype, int rows, int V, long long row_stride, int K, int32_t* ids,
+                          float* lp, float* lse, cudaStream_t stream) {
+  int st = topk_check(logits, dtype, rows, V, row_stride, K, ids, lp);
+  if (st) return st;
+  const TopkPlan p = topk_plan(rows, V, K, esize_of(dtype), num_sms());
+  if (p.cpr == 0) return DDTREE_ERR_UNSUPPORTED;
+  const size_t need = topk_ws_bytes(rows, p);
+  if (need > STATIC_SCRATCH_BYTES) return DDTREE_ERR_SCRATCH_LIMIT;
+  void* ws = static_scratch_ptr();
+  if (ws == nullptr) return DDTREE_ERR_CUDA;
+  // the per-row tickets must start at zero; a previous call normally leaves
+  // them at zero, but the array is shared, so clear them every time
+  if (cudaMemsetAsync(ws, 0, align256((size_t)rows * 4), stream) != cudaSuccess) return DDTREE_ERR_CUDA;
+  return topk_launch(logits, dtype, rows, V, row_stride, K, ids, lp, lse, ws, need, stream);
+}
 
 }  // extern "C"

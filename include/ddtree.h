@@ -54,7 +54,8 @@ typedef enum {
   DDTREE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
   DDTREE_ERR_NONFINITE = 4,    /* device status bit: NaN in logits */
   DDTREE_ERR_TIMEOUT = 5,      /* device status bit: a bounded wait gave up */
-  DDTREE_ERR_CAPACITY = 6      /* device status bit: prefix + tree exceeds the cache */
+  DDTREE_ERR_CAPACITY = 6,     /* device status bit: prefix + tree exceeds the cache */
+  DDTREE_ERR_SCRATCH_LIMIT = 7 /* request needs more than the built-in scratch of ddtree_topk_static_ws */
 } ddtree_status;
 
 /* Device status word bits (ddtree_device_status). */
@@ -245,6 +246,37 @@ size_t ddtree_round_workspace_bytes(const ddtree_round_args* a);
  * node_token, parent, depth, anc, n_nodes and new_prefix_len are required,
  * the other outputs may be NULL. */
 int ddtree_round(const ddtree_round_args* a, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Top-K without a caller workspace (no counterpart in the paper: an      */
+/* interface convenience of this library).                                */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * Same computation, arguments and results as ddtree_topk, but the scratch
+ * memory lives in a fixed array built into the library instead of a
+ * caller workspace, so the call allocates nothing and needs no workspace.
+ * It is meant for callers that cannot allocate device memory while they
+ * run rounds: serving engines that hand all free device memory to their KV
+ * cache pool at start-up, where a cudaMalloc at decode time can synchronize
+ * the device or fail because the pool already holds the memory.
+ *
+ * Limits and behaviour:
+ *  - The built-in scratch is 4 MiB per device (allocated when the library is
+ *    loaded, held until the process exits).  A request whose scratch need,
+ *    ddtree_topk_workspace_bytes(rows, V, K), exceeds it is rejected with
+ *    DDTREE_ERR_SCRATCH_LIMIT before anything is launched (at V = 151936
+ *    and bf16 logits: up to 573 rows at K = 64, 145 at K = 256, 48 at
+ *    K = 1024 on a 148-SM B200).
+ *  - The first call on a device looks up the array's device address on the
+ *    current device; make that first call before any stream capture.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; each call clears the counters it needs at its start.  Calls
+ *    that overlap on the GPU (other streams, other host threads) race on the
+ *    array and must be serialized by the caller.
+ */
+int ddtree_topk_static_ws(const void* logits, int dtype, int rows, int V, long long row_stride, int K,
+                          int32_t* ids, float* lp, float* lse, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------- */
 /* Status                                                                 */

@@ -51,16 +51,18 @@ inline ArgmaxWs argmax_ws_carve(void* ws, int rows) {
   return w;
 }
 
-// The argmax of one chunk: bf16 keys are 32-bit composites (16-bit order key,
-// then the complemented 15-bit chunk-local index) reduced with redux.sync;
-// fp32 keys need 64 bits.  The chunk winner becomes a 64-bit composite with
-// the global token id for the row-wide atomicMax.
+// The argmax of one chunk.  bf16: a 16-bit SIMD max over order keys (two
+// logits per instruction) finds the chunk's largest key, then a compare pass
+// finds the lowest index holding it.  fp32: 64-bit (key, complemented id)
+// composites.  The chunk winner becomes a 64-bit composite with the global
+// token id for the row-wide atomicMax.
 template <int DT, int VPT>
 __global__ void __launch_bounds__(ARGMAX_THREADS)
 argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_stride,
               const int32_t* __restrict__ n_nodes, int cpr, int chunk, ArgmaxWs ws) {
   constexpr int EPV = (DT == DDTREE_BF16) ? 8 : 4;
   __shared__ unsigned long long red[ARGMAX_THREADS / 32];
+  __shared__ uint32_t red32[ARGMAX_THREADS / 32];
   const int tid = threadIdx.x;
   const int row = blockIdx.x / cpr;              // row = req * n + node
   const int c = blockIdx.x - row * cpr;
@@ -81,29 +83,57 @@ argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_strid
   unsigned long long best = 0;
   bool nan_seen = false;
   if (DT == DDTREE_BF16) {
-    uint32_t b32 = 0;
+    // pass 1: the chunk's largest order key, two bf16 at a time (16-bit SIMD max)
+    uint32_t m2 = 0;
 #pragma unroll
     for (int v = 0; v < VPT; ++v) {
-      const int vi = v * ARGMAX_THREADS + tid;
-      if (vi < nvec_full) {
+      if (v * ARGMAX_THREADS + tid < nvec_full) {
 #pragma unroll
-        for (int j = 0; j < EPV; ++j) {
-          const uint16_t bits = (uint16_t)((u32_at(vec[v], j >> 1) >> (16 * (j & 1))) & 0xFFFFu);
-          nan_seen |= bf16_is_nan(bits);
-          const uint32_t k = (key16_of_bf16(bits) << LID_BITS) | (LID_MASK - (uint32_t)(vi * EPV + j));
-          b32 = k > b32 ? k : b32;
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t w = u32_at(vec[v], q);
+          nan_seen |= bf16x2_nan(w) != 0u;
+          m2 = __vmaxu2(m2, key16x2_of_bf16x2(w));
         }
       }
     }
+    uint32_t kt = max(m2 & 0xFFFFu, m2 >> 16);
     for (int e = nvec_full * EPV + tid; e < len; e += ARGMAX_THREADS) {   // ragged tail
       const uint16_t bits = ((const uint16_t*)base)[e];
       nan_seen |= bf16_is_nan(bits);
-      const uint32_t k = (key16_of_bf16(bits) << LID_BITS) | (LID_MASK - (uint32_t)e);
-      b32 = k > b32 ? k : b32;
+      kt = max(kt, key16_of_bf16(bits));
     }
-    b32 = __reduce_max_sync(0xffffffffu, b32);
-    const uint32_t gid = (uint32_t)(c0 + (LID_MASK - (b32 & LID_MASK)));
-    best = b32 ? (((unsigned long long)(b32 >> LID_BITS) << TOPK_ID_BITS) | (TOPK_ID_MASK - gid)) : 0ull;
+    kt = __reduce_max_sync(0xffffffffu, kt);
+    if ((tid & 31) == 0) red32[tid >> 5] = kt;
+    __syncthreads();
+    uint32_t kmax = red32[0];
+#pragma unroll
+    for (int i = 1; i < ARGMAX_THREADS / 32; ++i) kmax = max(kmax, red32[i]);
+    __syncthreads();
+    // pass 2: the lowest chunk-local index holding that key
+    const uint32_t kmax2 = kmax | (kmax << 16);
+    uint32_t lowest = 0xFFFFFFFFu;
+#pragma unroll
+    for (int v = VPT - 1; v >= 0; --v) {           // later vectors first, so the lowest index wins
+      const int vi = v * ARGMAX_THREADS + tid;
+      if (vi < nvec_full) {
+#pragma unroll
+        for (int q = 3; q >= 0; --q) {
+          const uint32_t hit = __vcmpeq2(key16x2_of_bf16x2(u32_at(vec[v], q)), kmax2);
+          if (hit & 0xFFFF0000u) lowest = (uint32_t)(vi * EPV + 2 * q + 1);
+          if (hit & 0x0000FFFFu) lowest = (uint32_t)(vi * EPV + 2 * q);
+        }
+      }
+    }
+    for (int e = nvec_full * EPV + tid; e < len; e += ARGMAX_THREADS)
+      if (key16_of_bf16(((const uint16_t*)base)[e]) == kmax) lowest = min(lowest, (uint32_t)e);
+    lowest = __reduce_min_sync(0xffffffffu, lowest);
+    if ((tid & 31) == 0) red32[tid >> 5] = lowest;
+    __syncthreads();
+    uint32_t lmin = red32[0];
+#pragma unroll
+    for (int i = 1; i < ARGMAX_THREADS / 32; ++i) lmin = min(lmin, red32[i]);
+    const uint32_t gid = (uint32_t)(c0 + lmin);
+    best = ((unsigned long long)kmax << TOPK_ID_BITS) | (TOPK_ID_MASK - gid);
   } else {
 #pragma unroll
     for (int v = 0; v < VPT; ++v) {

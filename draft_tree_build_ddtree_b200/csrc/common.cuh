@@ -42,6 +42,18 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t bits) {
   return __uint_as_float(((uint32_t)bits) << 16);
 }
 
+// Order keys of the two bf16 values packed in a 32-bit word, two at a time:
+// each 16-bit half becomes key16_of_bf16 of that half (-0.0 canonicalised).
+__device__ __forceinline__ uint32_t key16x2_of_bf16x2(uint32_t w) {
+  w &= ~__vcmpeq2(w, 0x80008000u);                      // -0.0 -> +0.0
+  const uint32_t neg = ((w >> 15) & 0x00010001u) * 0xFFFFu;
+  return w ^ (neg | 0x80008000u);
+}
+// Nonzero iff either half of the word is a bf16 NaN.
+__device__ __forceinline__ uint32_t bf16x2_nan(uint32_t w) {
+  return __vcmpgtu2(w & 0x7FFF7FFFu, 0x7F807F80u);
+}
+
 // 16-byte read-only global load that does not allocate in L1 (streamed once).
 __device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
   uint4 r;

@@ -11,11 +11,13 @@
 //    over it are rolled loops over 16-byte vectors, which keeps the kernel's
 //    code small enough to stay in the instruction cache (fully unrolled
 //    register passes stalled on instruction fetch).
-//  * The chunk's sum of exp(z - max) is taken in fp64 with a table-driven
-//    exponential (Tang's method: 2^(k/64) from a table times a degree-5
-//    polynomial of the reduced argument), so that log q = z - lse, rounded
-//    once to fp32, is the correctly rounded value in all but vanishingly
-//    rare cases.  bf16 logits sit on a coarse grid, many prefixes tie
+//  * The chunk's sum of exp(z - max) is taken in fp64 so that
+//    log q = z - lse, rounded once to fp32, is the correctly rounded value
+//    in all but vanishingly rare cases.  For bf16 logits exp(z) comes from a
+//    65536-entry fp64 table indexed by the logit's bit pattern (built once
+//    per device with a table-driven exponential, Tang's method: 2^(k/64)
+//    from a table times a degree-5 polynomial of the reduced argument), so
+//    the sum costs one load and one add per logit.  bf16 logits sit on a coarse grid, many prefixes tie
 //    exactly in real arithmetic, and only a correctly rounded log-prob
 //    table orders them reproducibly.
 //  * The chunk's threshold value (the K'-th largest logit, K' = min(K,
@@ -108,9 +110,11 @@ inline TopkWs topk_ws_carve(void* ws, int rows, const TopkPlan& p) {
   return w;
 }
 
-// exp(x) in fp64 for x <= 0 (table-driven; relative error ~1e-16; 0 below -708).
-__device__ __forceinline__ double exp64_nonpos(double x, const double* tab) {
+// exp(x) in fp64 (table-driven; relative error ~1e-16): 0 below -708,
+// +inf above 709.
+__device__ __forceinline__ double exp64(double x, const double* tab) {
   if (!(x > -708.0)) return 0.0;
+  if (x > 709.0) return INFINITY;
   const double kd = rint(x * EXP64_INV_LN2_64);
   const int k = (int)kd;
   double r = fma(-kd, EXP64_C1, x);
@@ -124,6 +128,22 @@ __device__ __forceinline__ double exp64_nonpos(double x, const double* tab) {
   const double y = fma(tj, p, tj);          // 2^(j/64) * exp(r), in [0.99, 2.02)
   return __hiloint2double(__double2hiint(y) + ((k >> 6) << 20), __double2loint(y));
 }
+
+// exp(z) in fp64 for every bf16 bit pattern z, built once per device by
+// exp_bf16_table_kernel.  With it the sum of exp(z - m) over a chunk is one
+// table load and one fp64 add per logit, scaled by exp(-m) once.
+__device__ double g_exp_bf16[65536];
+
+__global__ void exp_bf16_table_kernel() {
+  __shared__ double tab[64];
+  if (threadIdx.x < 64) tab[threadIdx.x] = EXP64_TABLE[threadIdx.x];
+  __syncthreads();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < 65536) g_exp_bf16[i] = exp64((double)bf16_bits_to_f32((uint16_t)i), tab);
+}
+
+// Table use is exact when the chunk maximum keeps every sum in range.
+constexpr double EXP_TABLE_MAX_M = 600.0;
 
 // ---------------------------------------------------------------------------
 // Block-wide radix selection of the need-th largest key.
@@ -280,28 +300,42 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   __syncthreads();
 
   // Element e of vector vi is logit c0 + vi*EPV + e; its order key is 0 past the chunk end.
+  // bf16 keys are computed two at a time with 16-bit SIMD integer ops.
   auto keys_of = [&](int vi, uint32_t* k) {
     const uint4 v = chunk_s[vi];
+    const int valid = len - vi * EPV;              // >= EPV except in the ragged last vector
+    if (DT == DDTREE_BF16) {
 #pragma unroll
-    for (int j = 0; j < EPV; ++j)
-      k[j] = (vi * EPV + j < len) ? value_key<DT>(elem_bits<DT>(v, j)) : 0u;
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t k2 = key16x2_of_bf16x2(u32_at(v, q));
+        k[2 * q] = (2 * q < valid) ? (k2 & 0xFFFFu) : 0u;
+        k[2 * q + 1] = (2 * q + 1 < valid) ? (k2 >> 16) : 0u;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < EPV; ++j) k[j] = (j < valid) ? key32_of_f32(__uint_as_float(u32_at(v, j))) : 0u;
+    }
   };
 
   // ---- NaN check and chunk maximum ----
   uint32_t kmax = 0;
   bool nan_seen = false;
   for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+    uint32_t k[EPV];
+    keys_of(vi, k);
     const uint4 v = chunk_s[vi];
+    if (DT == DDTREE_BF16) {
+      // the staging zero-fills the ragged vector's tail, and 0 is no NaN
+      nan_seen |= (bf16x2_nan(v.x) | bf16x2_nan(v.y) | bf16x2_nan(v.z) | bf16x2_nan(v.w)) != 0u;
+    } else {
 #pragma unroll
-    for (int j = 0; j < EPV; ++j) {
-      if (vi * EPV + j < len) {
-        const uint32_t bits = elem_bits<DT>(v, j);
-        if (DT == DDTREE_BF16) nan_seen |= bf16_is_nan((uint16_t)bits);
-        else nan_seen |= __uint_as_float(bits) != __uint_as_float(bits);
-        const uint32_t k = value_key<DT>(bits);
-        kmax = k > kmax ? k : kmax;
+      for (int j = 0; j < EPV; ++j) {
+        const float f = __uint_as_float(u32_at(v, j));
+        nan_seen |= f != f;
       }
     }
+#pragma unroll
+    for (int j = 0; j < EPV; ++j) kmax = k[j] > kmax ? k[j] : kmax;
   }
   if (__any_sync(0xffffffffu, nan_seen) && (tid & 31) == 0) flag_status(DDTREE_STATUS_NONFINITE);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
@@ -314,15 +348,20 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   const double md = (double)m;
 
   // ---- fp64 sum of exp(z - m); bf16: max-anchored window histogram ----
-  double s = 0.0;
+  double s0 = 0.0, s1 = 0.0;
   const bool m_finite = m > -INFINITY;
+  const bool use_table = DT == DDTREE_BF16 && md <= EXP_TABLE_MAX_M && md >= -EXP_TABLE_MAX_M;
   for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
     uint32_t k[EPV];
     keys_of(vi, k);
+    const uint4 v = chunk_s[vi];
 #pragma unroll
     for (int j = 0; j < EPV; ++j) {
       if (k[j] != 0) {
-        if (m_finite) s += exp64_nonpos((double)key_value<DT>(k[j]) - md, s_tab);
+        double e;
+        if (use_table) e = g_exp_bf16[elem_bits<DT>(v, j)];           // exp(z); scaled below
+        else e = m_finite ? exp64((double)key_value<DT>(k[j]) - md, s_tab) : 0.0;
+        if (j & 1) s1 += e; else s0 += e;
         if (DT == DDTREE_BF16) {
           const uint32_t d = kmax - k[j];
           if (d < 256u) atomicAdd(&hist[d], 1u);
@@ -330,6 +369,7 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
       }
     }
   }
+  double s = s0 + s1;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if ((tid & 31) == 0) red_d[tid >> 5] = s;
@@ -429,6 +469,7 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   if (tid == 0) {
     double tot = 0.0;
     for (int i = 0; i < TOPK_THREADS / 32; ++i) tot += red_d[i];
+    if (use_table) tot *= exp64(-md, s_tab);           // sum of exp(z) -> sum of exp(z - m)
     ws.stats[(size_t)row * plan.cpr + c] = make_double2(md, tot);
     ws.count[(size_t)row * plan.cpr + c] = s_count < plan.cap ? s_count : plan.cap;
   }
@@ -449,33 +490,49 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   unsigned long long* win = sc + plan.cand;                 // [kpow]
   __shared__ int s_off[TOPK_MAX_CPR];
   __shared__ int s_cnt[TOPK_MAX_CPR];
+  __shared__ double2 s_st[TOPK_MAX_CPR];
   __shared__ int s_ncand;
   __shared__ double s_lse;
+  for (int i = tid; i < plan.cpr; i += TOPK_THREADS) {
+    s_cnt[i] = __ldcg(&ws.count[(size_t)row * plan.cpr + i]);
+    s_st[i] = __ldcg(&ws.stats[(size_t)row * plan.cpr + i]);
+  }
+  for (int i = tid; i < kpow; i += TOPK_THREADS) win[i] = 0ull;
+  __syncthreads();
   if (tid == 0) {
     int off = 0;
     double M = -INFINITY;
     for (int i = 0; i < plan.cpr; ++i) {
       s_off[i] = off;
-      s_cnt[i] = __ldcg(&ws.count[(size_t)row * plan.cpr + i]);
       off += s_cnt[i];
-      M = fmax(M, __ldcg(&ws.stats[(size_t)row * plan.cpr + i].x));
+      M = fmax(M, s_st[i].x);
     }
     s_ncand = off;
     double S = 0.0;
-    if (M > -INFINITY) {
-      for (int i = 0; i < plan.cpr; ++i) {
-        const double2 st = __ldcg(&ws.stats[(size_t)row * plan.cpr + i]);
-        if (st.x > -INFINITY) S += st.y * exp64_nonpos(st.x - M, s_tab);
-      }
-    }
+    if (M > -INFINITY)
+      for (int i = 0; i < plan.cpr; ++i)
+        if (s_st[i].x > -INFINITY) S += s_st[i].y * exp64(s_st[i].x - M, s_tab);
     s_lse = M + log(S);
     ws.ticket[row] = 0;   // leave the workspace ready for the next call
   }
   __syncthreads();
-  for (int i = tid; i < kpow; i += TOPK_THREADS) win[i] = 0ull;
-  for (int ci = 0; ci < plan.cpr; ++ci) {
-    const unsigned long long* src = cand_row + (size_t)ci * plan.cap;
-    for (int i = tid; i < s_cnt[ci]; i += TOPK_THREADS) sc[s_off[ci] + i] = __ldcg(src + i);
+  {
+    constexpr int UNR = 4;   // issue several candidate loads before storing any
+    const int slots = plan.cpr * plan.cap;
+    for (int s0 = tid; s0 < slots; s0 += UNR * TOPK_THREADS) {
+      unsigned long long v[UNR];
+      int dst[UNR];
+#pragma unroll
+      for (int u = 0; u < UNR; ++u) {
+        const int sl = s0 + u * TOPK_THREADS;
+        const int ci = sl / plan.cap, j = sl - ci * plan.cap;
+        dst[u] = (sl < slots && j < s_cnt[ci]) ? s_off[ci] + j : -1;
+        v[u] = dst[u] >= 0 ? __ldcg(cand_row + sl) : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < UNR; ++u)
+        if (dst[u] >= 0) sc[dst[u]] = v[u];
+    }
   }
   if (tid == 0) s_count = 0;
   __syncthreads();

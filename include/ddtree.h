@@ -101,11 +101,14 @@ size_t ddtree_topk_workspace_bytes(int rows, int V, int K);
  *            of a row are read (rows = n_req * L block positions).
  * K          tokens kept per row, 1 <= K <= min(V, 1024).
  * ids        device int32 [rows][K]: token ids by (logit desc, id asc).
- * lp         device float [rows][K]: log q of those tokens, (z - max) - log S
- *            in fp32, where S = sum exp(z - max).
+ * lp         device float [rows][K]: log q of those tokens, z - lse.
  * lse        device float [rows] (may be NULL): max + log S.
  * NaN logits set DDTREE_STATUS_NONFINITE; -inf is allowed and ranks last;
  * -0.0 ranks equal to +0.0.
+ * lp is the fp64 value z - lse rounded once to fp32 (the sum of exp is taken
+ * in fp64).  The first bf16 call on a device builds a 512 KiB table of
+ * exp(z) for every bf16 value in static device memory and synchronizes
+ * `stream` once; make it before any stream capture.
  */
 int ddtree_topk(const void* logits, int dtype, int rows, int V, long long row_stride,
                 int K, int32_t* ids, float* lp, float* lse,

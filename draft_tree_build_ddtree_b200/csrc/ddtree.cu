@@ -50,13 +50,32 @@ int launch_status() {
   return e == cudaSuccess ? DDTREE_OK : DDTREE_ERR_CUDA;
 }
 
+// Opt a kernel in to `bytes` of dynamic shared memory when its static plus
+// dynamic shared memory exceeds the default 48 KB; the attribute is raised
+// once per kernel and size (cached per device-independent function pointer).
+struct SmemOptIn {
+  const void* fn;
+  size_t bytes;
+};
+SmemOptIn g_smem_optin[64];
+int g_smem_optin_n = 0;
+
 template <typename F>
 int set_smem(F* kernel, size_t bytes) {
-  if (bytes > (size_t)max_smem_optin()) return DDTREE_ERR_UNSUPPORTED;
-  if (bytes > 48 * 1024) {
+  const void* fn = (const void*)kernel;
+  int slot = -1;
+  for (int i = 0; i < g_smem_optin_n; ++i)
+    if (g_smem_optin[i].fn == fn) slot = i;
+  if (slot >= 0 && g_smem_optin[slot].bytes >= bytes) return DDTREE_OK;
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return DDTREE_ERR_CUDA;
+  if (bytes + attr.sharedSizeBytes > (size_t)max_smem_optin()) return DDTREE_ERR_UNSUPPORTED;
+  if (bytes + attr.sharedSizeBytes > 48 * 1024) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
       return DDTREE_ERR_CUDA;
   }
+  if (slot < 0 && g_smem_optin_n < 64) slot = g_smem_optin_n++;
+  if (slot >= 0) g_smem_optin[slot] = SmemOptIn{fn, bytes};
   return DDTREE_OK;
 }
 

@@ -51,9 +51,9 @@ inline ArgmaxWs argmax_ws_carve(void* ws, int rows) {
   return w;
 }
 
-// The argmax of one chunk.  bf16: a 16-bit SIMD max over order keys (two
-// logits per instruction) finds the chunk's largest key, then a compare pass
-// finds the lowest index holding it.  fp32: 64-bit (key, complemented id)
+// The argmax of one chunk.  bf16: an fp32 max pass (bf16 widens with a
+// shift) finds the chunk's largest value, then the threads holding it find
+// the lowest index with that value.  fp32: 64-bit (key, complemented id)
 // composites.  The chunk winner becomes a 64-bit composite with the global
 // token id for the row-wide atomicMax.
 template <int DT, int VPT>
@@ -63,6 +63,7 @@ argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_strid
   constexpr int EPV = (DT == DDTREE_BF16) ? 8 : 4;
   __shared__ unsigned long long red[ARGMAX_THREADS / 32];
   __shared__ uint32_t red32[ARGMAX_THREADS / 32];
+  __shared__ float redf[ARGMAX_THREADS / 32];
   const int tid = threadIdx.x;
   const int row = blockIdx.x / cpr;              // row = req * n + node
   const int c = blockIdx.x - row * cpr;
@@ -83,49 +84,54 @@ argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_strid
   unsigned long long best = 0;
   bool nan_seen = false;
   if (DT == DDTREE_BF16) {
-    // pass 1: the chunk's largest order key, two bf16 at a time (16-bit SIMD max)
-    uint32_t m2 = 0;
+    // pass 1: the chunk's largest value (bf16 widens to fp32 exactly with a
+    // shift; fmaxf skips NaN, which the magnitude maxima below detect)
+    float mx = -INFINITY;
+    uint32_t mag_lo = 0, mag_hi = 0;
 #pragma unroll
     for (int v = 0; v < VPT; ++v) {
       if (v * ARGMAX_THREADS + tid < nvec_full) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const uint32_t w = u32_at(vec[v], q);
-          nan_seen |= bf16x2_nan(w) != 0u;
-          m2 = __vmaxu2(m2, key16x2_of_bf16x2(w));
+          mx = fmaxf(mx, fmaxf(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
+          mag_lo = max(mag_lo, w & 0x7FFFu);
+          mag_hi = max(mag_hi, w & 0x7FFF0000u);
         }
       }
     }
-    uint32_t kt = max(m2 & 0xFFFFu, m2 >> 16);
     for (int e = nvec_full * EPV + tid; e < len; e += ARGMAX_THREADS) {   // ragged tail
-      const uint16_t bits = ((const uint16_t*)base)[e];
-      nan_seen |= bf16_is_nan(bits);
-      kt = max(kt, key16_of_bf16(bits));
+      const uint32_t bits = ((const uint16_t*)base)[e];
+      mx = fmaxf(mx, bf16_bits_to_f32((uint16_t)bits));
+      mag_lo = max(mag_lo, bits & 0x7FFFu);
     }
-    kt = __reduce_max_sync(0xffffffffu, kt);
-    if ((tid & 31) == 0) red32[tid >> 5] = kt;
+    nan_seen = mag_lo > 0x7F80u || mag_hi > 0x7F800000u;
+    const float tmx = mx;
+    mx = warp_max(mx);
+    if ((tid & 31) == 0) redf[tid >> 5] = mx;
     __syncthreads();
-    uint32_t kmax = red32[0];
+    mx = redf[0];
 #pragma unroll
-    for (int i = 1; i < ARGMAX_THREADS / 32; ++i) kmax = max(kmax, red32[i]);
-    __syncthreads();
-    // pass 2: the lowest chunk-local index holding that key
-    const uint32_t kmax2 = kmax | (kmax << 16);
+    for (int i = 1; i < ARGMAX_THREADS / 32; ++i) mx = fmaxf(mx, redf[i]);
+    // pass 2: the lowest chunk-local index holding the maximum (-0.0 == +0.0);
+    // only threads that hold it scan
     uint32_t lowest = 0xFFFFFFFFu;
+    if (tmx == mx) {
 #pragma unroll
-    for (int v = VPT - 1; v >= 0; --v) {           // later vectors first, so the lowest index wins
-      const int vi = v * ARGMAX_THREADS + tid;
-      if (vi < nvec_full) {
+      for (int v = VPT - 1; v >= 0; --v) {           // later vectors first, so the lowest index wins
+        const int vi = v * ARGMAX_THREADS + tid;
+        if (vi < nvec_full) {
 #pragma unroll
-        for (int q = 3; q >= 0; --q) {
-          const uint32_t hit = __vcmpeq2(key16x2_of_bf16x2(u32_at(vec[v], q)), kmax2);
-          if (hit & 0xFFFF0000u) lowest = (uint32_t)(vi * EPV + 2 * q + 1);
-          if (hit & 0x0000FFFFu) lowest = (uint32_t)(vi * EPV + 2 * q);
+          for (int q = 3; q >= 0; --q) {
+            const uint32_t w = u32_at(vec[v], q);
+            if (__uint_as_float(w & 0xFFFF0000u) == mx) lowest = (uint32_t)(vi * EPV + 2 * q + 1);
+            if (__uint_as_float(w << 16) == mx) lowest = (uint32_t)(vi * EPV + 2 * q);
+          }
         }
       }
+      for (int e = nvec_full * EPV + tid; e < len; e += ARGMAX_THREADS)
+        if (bf16_bits_to_f32(((const uint16_t*)base)[e]) == mx) lowest = min(lowest, (uint32_t)e);
     }
-    for (int e = nvec_full * EPV + tid; e < len; e += ARGMAX_THREADS)
-      if (key16_of_bf16(((const uint16_t*)base)[e]) == kmax) lowest = min(lowest, (uint32_t)e);
     lowest = __reduce_min_sync(0xffffffffu, lowest);
     if ((tid & 31) == 0) red32[tid >> 5] = lowest;
     __syncthreads();
@@ -133,7 +139,7 @@ argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_strid
 #pragma unroll
     for (int i = 1; i < ARGMAX_THREADS / 32; ++i) lmin = min(lmin, red32[i]);
     const uint32_t gid = (uint32_t)(c0 + lmin);
-    best = ((unsigned long long)kmax << TOPK_ID_BITS) | (TOPK_ID_MASK - gid);
+    best = ((unsigned long long)key32_of_f32(mx) << TOPK_ID_BITS) | (TOPK_ID_MASK - gid);
   } else {
 #pragma unroll
     for (int v = 0; v < VPT; ++v) {

@@ -320,22 +320,48 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   // ---- NaN check and chunk maximum ----
   uint32_t kmax = 0;
   bool nan_seen = false;
-  for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
-    uint32_t k[EPV];
-    keys_of(vi, k);
-    const uint4 v = chunk_s[vi];
-    if (DT == DDTREE_BF16) {
-      // the staging zero-fills the ragged vector's tail, and 0 is no NaN
-      nan_seen |= (bf16x2_nan(v.x) | bf16x2_nan(v.y) | bf16x2_nan(v.z) | bf16x2_nan(v.w)) != 0u;
-    } else {
+  if (DT == DDTREE_BF16) {
+    // bf16 widens to fp32 with a shift: the maximum is an fp32 max (fmaxf
+    // skips NaN; the magnitude maxima detect it); past-the-end elements of
+    // the ragged vector count as -inf
+    float mx = -INFINITY;
+    uint32_t mag_lo = 0, mag_hi = 0;
+    for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+      const uint4 v = chunk_s[vi];
+      const int valid = len - vi * EPV;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t w = u32_at(v, q);
+        const float lo = 2 * q < valid ? __uint_as_float(w << 16) : -INFINITY;
+        const float hi = 2 * q + 1 < valid ? __uint_as_float(w & 0xFFFF0000u) : -INFINITY;
+        mx = fmaxf(mx, fmaxf(lo, hi));
+        mag_lo = max(mag_lo, w & 0x7FFFu);
+        mag_hi = max(mag_hi, w & 0x7FFF0000u);
+      }
+    }
+    nan_seen = mag_lo > 0x7F80u || mag_hi > 0x7F800000u;
+    // the order key of the maximum (any element equal to it has this key)
+    kmax = mx > -INFINITY ? key32_of_f32(mx) >> 16 : 0u;
+    if (mx == -INFINITY) {                      // only -inf (or nothing) here: key of -inf if present
+      for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+        uint32_t k[EPV];
+        keys_of(vi, k);
+#pragma unroll
+        for (int j = 0; j < EPV; ++j) kmax = k[j] > kmax ? k[j] : kmax;
+      }
+    }
+  } else {
+    for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+      uint32_t k[EPV];
+      keys_of(vi, k);
+      const uint4 v = chunk_s[vi];
 #pragma unroll
       for (int j = 0; j < EPV; ++j) {
         const float f = __uint_as_float(u32_at(v, j));
         nan_seen |= f != f;
+        kmax = k[j] > kmax ? k[j] : kmax;
       }
     }
-#pragma unroll
-    for (int j = 0; j < EPV; ++j) kmax = k[j] > kmax ? k[j] : kmax;
   }
   if (__any_sync(0xffffffffu, nan_seen) && (tid & 31) == 0) flag_status(DDTREE_STATUS_NONFINITE);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
@@ -351,20 +377,37 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   double s0 = 0.0, s1 = 0.0;
   const bool m_finite = m > -INFINITY;
   const bool use_table = DT == DDTREE_BF16 && md <= EXP_TABLE_MAX_M && md >= -EXP_TABLE_MAX_M;
-  for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
-    uint32_t k[EPV];
-    keys_of(vi, k);
-    const uint4 v = chunk_s[vi];
+  if (DT == DDTREE_BF16) {
+    // values below the window's lowest bin skip the histogram with one compare
+    const float wlow = kmax >= 255u ? bf16_of_key16(kmax - 255u) : -INFINITY;
+    for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+      const uint4 v = chunk_s[vi];
+      const int valid = len - vi * EPV;
 #pragma unroll
-    for (int j = 0; j < EPV; ++j) {
-      if (k[j] != 0) {
-        double e;
-        if (use_table) e = g_exp_bf16[elem_bits<DT>(v, j)];           // exp(z); scaled below
-        else e = m_finite ? exp64((double)key_value<DT>(k[j]) - md, s_tab) : 0.0;
-        if (j & 1) s1 += e; else s0 += e;
-        if (DT == DDTREE_BF16) {
-          const uint32_t d = kmax - k[j];
-          if (d < 256u) atomicAdd(&hist[d], 1u);
+      for (int j = 0; j < EPV; ++j) {
+        if (j < valid) {
+          const uint32_t bits = elem_bits<DT>(v, j);
+          const float z = bf16_bits_to_f32((uint16_t)bits);
+          double e;
+          if (use_table) e = g_exp_bf16[bits];                            // exp(z); scaled below
+          else e = m_finite ? exp64((double)z - md, s_tab) : 0.0;
+          if (j & 1) s1 += e; else s0 += e;
+          if (z >= wlow) {
+            const uint32_t d = kmax - key16_of_bf16((uint16_t)bits);
+            if (d < 256u) atomicAdd(&hist[d], 1u);
+          }
+        }
+      }
+    }
+  } else {
+    for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+      uint32_t k[EPV];
+      keys_of(vi, k);
+#pragma unroll
+      for (int j = 0; j < EPV; ++j) {
+        if (k[j] != 0) {
+          const double e = m_finite ? exp64((double)key_value<DT>(k[j]) - md, s_tab) : 0.0;
+          if (j & 1) s1 += e; else s0 += e;
         }
       }
     }
@@ -449,19 +492,39 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   __syncthreads();
   unsigned long long* cand_row = ws.cand + (size_t)row * plan.cand;
   unsigned long long* cand = cand_row + (size_t)c * plan.cap;
-  for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
-    uint32_t k[EPV];
-    keys_of(vi, k);
+  if (DT == DDTREE_BF16 && all_ties) {
+    // every logit >= the threshold value: one fp32 compare per logit (-0.0 == +0.0)
+    const float tf = bf16_of_key16(tval);
+    for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+      const uint4 v = chunk_s[vi];
+      const int valid = len - vi * EPV;
 #pragma unroll
-    for (int j = 0; j < EPV; ++j) {
-      const int lid = vi * EPV + j;
-      const bool take =
-          k[j] != 0 && (k[j] > tval || (k[j] == tval && (all_ties || (LID_MASK - (uint32_t)lid) >= lid_thr)));
-      if (take) {
-        const int slot = atomicAdd(&s_count, 1);
-        const uint32_t gid = (uint32_t)(c0 + lid);
-        if (slot < plan.cap)
-          cand[slot] = ((unsigned long long)k[j] << TOPK_ID_BITS) | (unsigned long long)(TOPK_ID_MASK - gid);
+      for (int j = 0; j < EPV; ++j) {
+        const uint32_t bits = elem_bits<DT>(v, j);
+        if (j < valid && bf16_bits_to_f32((uint16_t)bits) >= tf) {
+          const int slot = atomicAdd(&s_count, 1);
+          const uint32_t gid = (uint32_t)(c0 + vi * EPV + j);
+          if (slot < plan.cap)
+            cand[slot] = ((unsigned long long)key16_of_bf16((uint16_t)bits) << TOPK_ID_BITS) |
+                         (unsigned long long)(TOPK_ID_MASK - gid);
+        }
+      }
+    }
+  } else {
+    for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+      uint32_t k[EPV];
+      keys_of(vi, k);
+#pragma unroll
+      for (int j = 0; j < EPV; ++j) {
+        const int lid = vi * EPV + j;
+        const bool take =
+            k[j] != 0 && (k[j] > tval || (k[j] == tval && (all_ties || (LID_MASK - (uint32_t)lid) >= lid_thr)));
+        if (take) {
+          const int slot = atomicAdd(&s_count, 1);
+          const uint32_t gid = (uint32_t)(c0 + lid);
+          if (slot < plan.cap)
+            cand[slot] = ((unsigned long long)k[j] << TOPK_ID_BITS) | (unsigned long long)(TOPK_ID_MASK - gid);
+        }
       }
     }
   }

@@ -12,19 +12,15 @@
 // prefixes in exactly that order.
 //
 // Design: one CTA per request; one warp runs the queue, the whole CTA
-// writes the outputs.  Instead of one pop per step the warp pops in rounds:
-//  * the frontier (the heap's contents) is kept sorted in shared memory;
-//  * a round takes its m = min(32, frontier, remaining budget) best entries;
-//    call the m-th one tau.  Every prefix that will ever be popped before
-//    tau is one of those entries or is generated from them by sibling/child
-//    pushes (a generated entry never beats its generator), so the round
-//    expands that closure level by level, keeping generated entries that
-//    beat tau and setting the others aside;
-//  * the closure is sorted (bitonic, one warp) and popped as consecutive
-//    nodes; the set-aside entries are sorted and merged into the frontier.
-// The pop sequence is exactly the heap's; a round replaces up to dozens of
-// dependent heap steps.  If a closure outgrows its buffer the round is
-// redone with a smaller m (m = 1 always fits: nothing beats its generator).
+// writes the outputs.  The queue is a two-level tournament: frontier slot s
+// (an entry of the heap) lives in shared memory in block s / 32, and the
+// best entry of each block (its order key and slot) is cached in the
+// registers of lane (block % 32).  A pop is a warp reduction over the cached
+// block bests; the popped slot takes the popped entry's next sibling and the
+// first child goes to a fresh slot, after which the one or two blocks that
+// changed are re-reduced with one 32-wide shared-memory read each.  A pop
+// costs a fixed handful of warp reductions whatever the budget (up to 64
+// blocks, 2048 slots), instead of a per-lane rescan that grew with B.
 //
 // Order keys are 64 bits: the fp32 score's order key, then a tie key that
 // packs the tuple's first ranks (exactly equal fp32 scores are common with
@@ -38,9 +34,6 @@
 namespace ddt {
 
 constexpr int BUILD_THREADS = 256;
-constexpr int BUILD_MAXM = 32;          // frontier entries taken per round
-constexpr int BUILD_CCAP = 128;         // closure capacity per round
-constexpr int BUILD_NCAP = 2 * BUILD_CCAP;
 
 // Entry metadata: parent node (11 bits), depth (6 bits), rank (15 bits).
 __device__ __forceinline__ uint32_t pack_meta(int parent, int depth, int rank) {
@@ -91,64 +84,19 @@ __device__ __forceinline__ bool tuple_less(uint32_t ma, uint32_t mb, const int* 
   return ra < rb;
 }
 
-// The entry arrays of one list (frontier, closure or set-aside entries).
-struct EntryList {
-  uint32_t* kx;    // score key
-  uint32_t* ky;    // tie key
-  float* sc;       // score
-  float* ps;       // score of the parent node
-  uint32_t* mt;    // packed parent/depth/rank
+// A frontier entry's 64-bit order key and its slot.
+struct Best {
+  uint32_t hi, lo;   // score key, tie key; hi == 0: none
+  int slot;
 };
-
-struct BuildCtx {
-  const int* nd_parent;
-  const int* nd_rank;
-  // a before b in the pop order
-  __device__ __forceinline__ bool before(uint32_t ax, uint32_t ay, uint32_t am, uint32_t bx, uint32_t by,
-                                         uint32_t bm) const {
-    if (ax != bx) return ax > bx;
-    if (ay != by) return ay > by;
-    return tuple_less(am, bm, nd_parent, nd_rank);
-  }
-};
-
-// Warp bitonic sort of indices idx[0..len) into pop order (best first);
-// padding up to a power of two with -1, which sorts last.
-__device__ __forceinline__ int warp_sort(int* idx, int len, const EntryList& e, const BuildCtx& cx, int lane) {
-  int p2 = 1;
-  while (p2 < len) p2 <<= 1;
-  for (int i = len + lane; i < p2; i += 32) idx[i] = -1;
-  __syncwarp();
-  for (int size = 2; size <= p2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = lane; i < p2 / 2; i += 32) {
-        const int lo = 2 * stride * (i / stride) + (i % stride);
-        const int hi = lo + stride;
-        const int a = idx[lo], b = idx[hi];
-        // desc: best first within blocks whose (lo & size) == 0
-        bool b_first;
-        if (a < 0) b_first = b >= 0;
-        else if (b < 0) b_first = false;
-        else b_first = cx.before(e.kx[b], e.ky[b], e.mt[b], e.kx[a], e.ky[a], e.mt[a]);
-        const bool asc = (lo & size) != 0;
-        if (b_first != asc) { idx[lo] = b; idx[hi] = a; }
-      }
-      __syncwarp();
-    }
-  }
-  return p2;
-}
 
 struct BuildSmem {
-  float* lp;                 // [L][kc]
-  EntryList F0, F1;          // frontier, double buffered, sorted best first [n + 1]
-  EntryList C;               // closure of the current round [CCAP]
-  EntryList N;               // entries set aside this round [NCAP]
-  int* cidx;                 // [CCAP] sort permutation of C
-  int* cinv;                 // [CCAP] sorted position of each closure entry
-  int* nidx;                 // [NCAP] sort permutation of N
-  int* nins;                 // [NCAP] insertion point of each sorted N entry in the frontier
-  int* nd_parent;            // [n + CCAP] (provisional ids during a round)
+  float* lp;         // [L][kc]
+  uint2* key;        // [B+1] slot order keys (score key, tie key); (0,0) = empty
+  float* sc;         // [B+1] slot score
+  float* ps;         // [B+1] score of the slot entry's parent node
+  uint32_t* mt;      // [B+1] packed parent/depth/rank
+  int* nd_parent;    // [B+1]
   int* nd_rank;
   int* nd_depth;
   float* nd_score;
@@ -156,27 +104,42 @@ struct BuildSmem {
 
 inline size_t build_smem_bytes(int L, int kc, int B) {
   const size_t n = (size_t)B + 1;
-  const size_t entry = 5 * 4;
-  return (size_t)L * kc * 4 + 2 * (n + 1) * entry + (BUILD_CCAP + BUILD_NCAP) * entry +
-         (2 * BUILD_CCAP + 2 * BUILD_NCAP) * 4 + (n + BUILD_CCAP) * 4 * 4;
+  return (size_t)L * kc * 4 + n * (8 + 4 + 4 + 4) + n * 4 * 4;
 }
 
-__device__ __forceinline__ EntryList carve_list(unsigned char*& p, int cap) {
-  EntryList e;
-  e.kx = (uint32_t*)p; p += (size_t)cap * 4;
-  e.ky = (uint32_t*)p; p += (size_t)cap * 4;
-  e.sc = (float*)p;    p += (size_t)cap * 4;
-  e.ps = (float*)p;    p += (size_t)cap * 4;
-  e.mt = (uint32_t*)p; p += (size_t)cap * 4;
-  return e;
+// a before b in the pop order
+__device__ __forceinline__ bool best_before(const Best& a, const Best& b, const BuildSmem& sm) {
+  if (a.hi != b.hi) return a.hi > b.hi;
+  if (a.lo != b.lo) return a.lo > b.lo;
+  return tuple_less(sm.mt[a.slot], sm.mt[b.slot], sm.nd_parent, sm.nd_rank);
 }
 
-__device__ __forceinline__ void put(const EntryList& e, int i, uint32_t kx, uint32_t ky, float sc, float ps,
-                                    uint32_t mt) {
-  e.kx[i] = kx; e.ky[i] = ky; e.sc[i] = sc; e.ps[i] = ps; e.mt[i] = mt;
-}
-__device__ __forceinline__ void copy_entry(const EntryList& d, int i, const EntryList& s, int j) {
-  d.kx[i] = s.kx[j]; d.ky[i] = s.ky[j]; d.sc[i] = s.sc[j]; d.ps[i] = s.ps[j]; d.mt[i] = s.mt[j];
+// The warp-wide best among one candidate per lane (hi == 0: none).  Equal
+// keys are rare and resolved by the exact tuple comparison.
+__device__ __forceinline__ Best warp_best(const Best& c, const BuildSmem& sm) {
+  Best r;
+  r.hi = __reduce_max_sync(0xffffffffu, c.hi);
+  if (r.hi == 0) { r.lo = 0; r.slot = -1; return r; }
+  unsigned eq = __ballot_sync(0xffffffffu, c.hi == r.hi);
+  r.lo = c.lo;
+  if (eq & (eq - 1)) {
+    r.lo = __reduce_max_sync(0xffffffffu, c.hi == r.hi ? c.lo : 0u);
+    eq = __ballot_sync(0xffffffffu, c.hi == r.hi && c.lo == r.lo);
+  }
+  int wl = __ffs(eq) - 1;
+  r.slot = __shfl_sync(0xffffffffu, c.slot, wl);
+  r.lo = __shfl_sync(0xffffffffu, c.lo, wl);
+  eq &= eq - 1;
+  while (eq) {                       // identical keys: smallest rank tuple
+    const int l2 = __ffs(eq) - 1;
+    eq &= eq - 1;
+    Best o;
+    o.hi = r.hi;
+    o.lo = r.lo;
+    o.slot = __shfl_sync(0xffffffffu, c.slot, l2);
+    if (best_before(o, r, sm)) r = o;
+  }
+  return r;
 }
 
 __global__ void __launch_bounds__(BUILD_THREADS, 1)
@@ -194,18 +157,14 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
   BuildSmem sm;
   {
     unsigned char* p = smem_raw;
-    sm.lp = (float*)p; p += (size_t)L * kc * 4;
-    sm.F0 = carve_list(p, n + 1);
-    sm.F1 = carve_list(p, n + 1);
-    sm.C = carve_list(p, BUILD_CCAP);
-    sm.N = carve_list(p, BUILD_NCAP);
-    sm.cidx = (int*)p; p += BUILD_CCAP * 4;
-    sm.cinv = (int*)p; p += BUILD_CCAP * 4;
-    sm.nidx = (int*)p; p += BUILD_NCAP * 4;
-    sm.nins = (int*)p; p += BUILD_NCAP * 4;
-    sm.nd_parent = (int*)p; p += (size_t)(n + BUILD_CCAP) * 4;
-    sm.nd_rank = (int*)p;   p += (size_t)(n + BUILD_CCAP) * 4;
-    sm.nd_depth = (int*)p;  p += (size_t)(n + BUILD_CCAP) * 4;
+    sm.key = (uint2*)p;     p += (size_t)n * 8;
+    sm.lp = (float*)p;      p += (size_t)L * kc * 4;
+    sm.sc = (float*)p;      p += (size_t)n * 4;
+    sm.ps = (float*)p;      p += (size_t)n * 4;
+    sm.mt = (uint32_t*)p;   p += (size_t)n * 4;
+    sm.nd_parent = (int*)p; p += (size_t)n * 4;
+    sm.nd_rank = (int*)p;   p += (size_t)n * 4;
+    sm.nd_depth = (int*)p;  p += (size_t)n * 4;
     sm.nd_score = (float*)p;
   }
   __shared__ int s_pops;
@@ -220,166 +179,81 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
 
   if (tid < 32) {
     const int lane = tid;
-    const BuildCtx cx{sm.nd_parent, sm.nd_rank};
     if (lane == 0) {
       sm.nd_parent[0] = -1;
       sm.nd_rank[0] = -1;
       sm.nd_depth[0] = 0;
       sm.nd_score[0] = 0.f;
     }
-    int cur = 0, nf = 0, pops = 0;
+    // cached best of blocks `lane` and `lane + 32`
+    Best b0{0u, 0u, -1}, b1{0u, 0u, -1};
+    int next_slot = 0;
     if (B > 0) {   // the frontier starts with the best token of position 1
+      const float s0 = __fadd_rn(0.f, sm.lp[0]);
+      const uint32_t k0 = score_key(s0), t0 = ~tc.unit(1);
       if (lane == 0) {
-        const float s0 = __fadd_rn(0.f, sm.lp[0]);
-        put(sm.F0, 0, score_key(s0), ~tc.unit(1), s0, 0.f, pack_meta(0, 1, 0));
+        sm.key[0] = make_uint2(k0, t0);
+        sm.sc[0] = s0;
+        sm.ps[0] = 0.f;
+        sm.mt[0] = pack_meta(0, 1, 0);
+        b0 = Best{k0, t0, 0};
       }
-      nf = 1;
+      next_slot = 1;
     }
     __syncwarp();
-    int mcap = BUILD_MAXM;
-    while (pops < B && nf > 0) {
-      const EntryList F = cur ? sm.F1 : sm.F0;
-      int m = min(min(mcap, nf), B - pops);
-      const uint32_t tx = F.kx[m - 1], ty = F.ky[m - 1], tm = F.mt[m - 1];   // tau
-      const int base = pops + 1;            // provisional id of closure entry c is base + c
-      // ---- closure: the m best entries, then everything they generate that beats tau ----
-      for (int c = lane; c < m; c += 32) {
-        copy_entry(sm.C, c, F, c);
-        const uint32_t mt = F.mt[c];
-        sm.nd_parent[base + c] = meta_parent(mt);
-        sm.nd_rank[base + c] = meta_rank(mt);
-        sm.nd_depth[base + c] = meta_depth(mt);
+    // re-reduce block `blk` from shared memory into its owner's cached best
+    auto refresh = [&](int blk) {
+      const int s = 32 * blk + lane;
+      Best c{0u, 0u, -1};
+      if (s < next_slot) {
+        const uint2 k = sm.key[s];
+        c = Best{k.x, k.y, s};
       }
-      __syncwarp();
-      int nc = m, nn = 0, lo = 0;
-      bool overflow = false;
-      while (lo < nc && !overflow) {
-        const int hi = nc;
-        for (int c0 = lo; c0 < hi; c0 += 32) {
-          const int c = c0 + lane;
-          uint32_t gx[2] = {0u, 0u}, gy[2], gm[2];
-          float gs[2], gp[2];
-          bool gv[2] = {false, false};
-          if (c < hi) {
-            const uint32_t mt = sm.C.mt[c];
-            const int d = meta_depth(mt), rk = meta_rank(mt), par = meta_parent(mt);
-            const uint32_t packed = ~sm.C.ky[c];
-            const float s = sm.C.sc[c], ps = sm.C.ps[c];
-            if (rk + 1 < kc) {         // next sibling
-              gs[0] = __fadd_rn(ps, sm.lp[(d - 1) * kc + rk + 1]);
-              gx[0] = score_key(gs[0]); gy[0] = ~(packed + tc.unit(d)); gp[0] = ps;
-              gm[0] = pack_meta(par, d, rk + 1); gv[0] = true;
-            }
-            if (d < L) {               // first child
-              gs[1] = __fadd_rn(s, sm.lp[d * kc]);
-              gx[1] = score_key(gs[1]); gy[1] = ~(packed + tc.unit(d + 1)); gp[1] = s;
-              gm[1] = pack_meta(base + c, d + 1, 0); gv[1] = true;
-            }
-          }
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            const bool to_c = gv[g] && cx.before(gx[g], gy[g], gm[g], tx, ty, tm);
-            const bool to_n = gv[g] && !to_c;
-            const unsigned bc = __ballot_sync(0xffffffffu, to_c);
-            const unsigned bn = __ballot_sync(0xffffffffu, to_n);
-            const unsigned below = (1u << lane) - 1u;
-            if (nc + __popc(bc) > BUILD_CCAP || nn + __popc(bn) > BUILD_NCAP) {
-              overflow = true;
-            } else {
-              if (to_c) {
-                const int ci = nc + __popc(bc & below);
-                put(sm.C, ci, gx[g], gy[g], gs[g], gp[g], gm[g]);
-                sm.nd_parent[base + ci] = meta_parent(gm[g]);
-                sm.nd_rank[base + ci] = meta_rank(gm[g]);
-                sm.nd_depth[base + ci] = meta_depth(gm[g]);
-              }
-              if (to_n) put(sm.N, nn + __popc(bn & below), gx[g], gy[g], gs[g], gp[g], gm[g]);
-              nc += __popc(bc);
-              nn += __popc(bn);
-            }
-          }
-          __syncwarp();
-          if (overflow) break;
-        }
-        lo = hi;
+      const Best w = warp_best(c, sm);
+      if (lane == (blk & 31)) {
+        if (blk < 32) b0 = w;
+        else b1 = w;
       }
-      if (overflow) {             // redo the round with fewer entries
-        mcap = max(1, m / 2);
-        __syncwarp();
-        continue;
-      }
-      mcap = BUILD_MAXM;
-      // ---- pop the closure in order ----
-      for (int c = lane; c < nc; c += 32) sm.cidx[c] = c;
+    };
+    int pops = 0;
+    while (pops < B) {
+      const Best lb = (b1.hi != 0 && (b0.hi == 0 || best_before(b1, b0, sm))) ? b1 : b0;
+      const Best top = warp_best(lb, sm);
+      if (top.hi == 0) break;   // frontier empty
+      const int slot = top.slot;
+      const uint32_t meta = sm.mt[slot];
+      const float sc = sm.sc[slot], ps = sm.ps[slot];
+      const uint32_t packed = ~top.lo;                     // the popped entry's packed ranks
+      const int par = meta_parent(meta), d = meta_depth(meta), rk = meta_rank(meta);
+      const int node = ++pops;
+      const bool sib = rk + 1 < kc;              // next sibling: same parent, next rank
+      const bool child = d < L;                  // first child: one position deeper
+      const float lsib = sib ? sm.lp[(d - 1) * kc + rk + 1] : 0.f;
+      const float lchild = child ? sm.lp[d * kc] : 0.f;
+      const float ssib = __fadd_rn(ps, lsib);
+      const float schild = __fadd_rn(sc, lchild);
+      const int cslot = next_slot;
       __syncwarp();
-      warp_sort(sm.cidx, nc, sm.C, cx, lane);
-      for (int s = lane; s < nc; s += 32) sm.cinv[sm.cidx[s]] = s;
-      __syncwarp();
-      const int npop = min(nc, B - pops);
-      int pv[4], rv[4], dv[4];
-      float sv[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {     // read every provisional record before writing final ones
-        const int s = lane + 32 * t;
-        if (s < npop) {
-          const int c = sm.cidx[s];
-          const uint32_t mt = sm.C.mt[c];
-          int p = meta_parent(mt);
-          if (p >= base) p = base + sm.cinv[p - base];
-          pv[t] = p; rv[t] = meta_rank(mt); dv[t] = meta_depth(mt); sv[t] = sm.C.sc[c];
+      if (lane == 0) {
+        sm.nd_parent[node] = par;
+        sm.nd_rank[node] = rk;
+        sm.nd_depth[node] = d;
+        sm.nd_score[node] = sc;
+        sm.key[slot] = sib ? make_uint2(score_key(ssib), ~(packed + tc.unit(d))) : make_uint2(0u, 0u);
+        sm.sc[slot] = ssib;
+        sm.ps[slot] = ps;
+        sm.mt[slot] = pack_meta(par, d, rk + 1);
+        if (child) {
+          sm.key[cslot] = make_uint2(score_key(schild), ~(packed + tc.unit(d + 1)));
+          sm.sc[cslot] = schild;
+          sm.ps[cslot] = sc;
+          sm.mt[cslot] = pack_meta(node, d + 1, 0);
         }
       }
+      if (child) ++next_slot;
       __syncwarp();
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const int s = lane + 32 * t;
-        if (s < npop) {
-          sm.nd_parent[base + s] = pv[t];
-          sm.nd_rank[base + s] = rv[t];
-          sm.nd_depth[base + s] = dv[t];
-          sm.nd_score[base + s] = sv[t];
-        }
-      }
-      pops += npop;
-      __syncwarp();
-      if (pops >= B) break;
-      // ---- set-aside entries: final parent ids, sort, merge into the rest of the frontier ----
-      for (int j = lane; j < nn; j += 32) {
-        const uint32_t mt = sm.N.mt[j];
-        const int p = meta_parent(mt);
-        if (p >= base) sm.N.mt[j] = pack_meta(base + sm.cinv[p - base], meta_depth(mt), meta_rank(mt));
-        sm.nidx[j] = j;
-      }
-      __syncwarp();
-      warp_sort(sm.nidx, nn, sm.N, cx, lane);
-      const int nrest = nf - m;
-      // insertion point of each sorted set-aside entry among the remaining frontier F[m..nf)
-      for (int j = lane; j < nn; j += 32) {
-        const int e = sm.nidx[j];
-        int a = 0, b = nrest;
-        while (a < b) {
-          const int mid = (a + b) >> 1;
-          const int fi = m + mid;
-          if (cx.before(F.kx[fi], F.ky[fi], F.mt[fi], sm.N.kx[e], sm.N.ky[e], sm.N.mt[e])) a = mid + 1;
-          else b = mid;
-        }
-        sm.nins[j] = a;
-      }
-      __syncwarp();
-      const EntryList G = cur ? sm.F0 : sm.F1;
-      for (int j = lane; j < nn; j += 32) copy_entry(G, sm.nins[j] + j, sm.N, sm.nidx[j]);
-      for (int i = lane; i < nrest; i += 32) {
-        int a = 0, b = nn;              // set-aside entries placed before frontier entry i
-        while (a < b) {
-          const int mid = (a + b) >> 1;
-          if (sm.nins[mid] <= i) a = mid + 1;
-          else b = mid;
-        }
-        copy_entry(G, i + a, F, m + i);
-      }
-      nf = nrest + nn;
-      cur ^= 1;
-      __syncwarp();
+      refresh(slot >> 5);
+      if (child && (cslot >> 5) != (slot >> 5)) refresh(cslot >> 5);
     }
     if (lane == 0) s_pops = pops;
   }

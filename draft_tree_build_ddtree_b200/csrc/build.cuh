@@ -142,6 +142,157 @@ __device__ __forceinline__ Best warp_best(const Best& c, const BuildSmem& sm) {
   return r;
 }
 
+// Register-resident queue for budgets with at most E slots per lane:
+// slot s's order key lives in register s / 32 of lane s % 32 (its score,
+// parent score and metadata in shared memory).  A pop is a lane-local best
+// over E registers and one warp-wide selection; the popped entry's lane
+// takes its next sibling and the child's lane its first child, in
+// registers, with no re-reduction.  Returns the number of pops.
+template <int E>
+__device__ __forceinline__ int heap_registers(const BuildSmem& sm, int L, int B, int kc, TieCode tc, int lane) {
+  uint32_t kh[E], kl[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) { kh[e] = 0u; kl[e] = 0u; }
+  int next_slot = 0;
+  if (B > 0) {
+    const float s0 = __fadd_rn(0.f, sm.lp[0]);
+    if (lane == 0) {
+      kh[0] = score_key(s0);
+      kl[0] = ~tc.unit(1);
+      sm.sc[0] = s0;
+      sm.ps[0] = 0.f;
+      sm.mt[0] = pack_meta(0, 1, 0);
+    }
+    next_slot = 1;
+  }
+  __syncwarp();
+  int pops = 0;
+  while (pops < B) {
+    Best lb{0u, 0u, -1};
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const Best c{kh[e], kl[e], lane + 32 * e};
+      if (c.hi != 0 && (lb.hi == 0 || best_before(c, lb, sm))) lb = c;
+    }
+    const Best top = warp_best(lb, sm);
+    if (top.hi == 0) break;   // frontier empty
+    const int slot = top.slot;
+    const uint32_t meta = sm.mt[slot];
+    const float sc = sm.sc[slot], ps = sm.ps[slot];
+    const uint32_t packed = ~top.lo;
+    const int par = meta_parent(meta), d = meta_depth(meta), rk = meta_rank(meta);
+    const int node = ++pops;
+    const bool sib = rk + 1 < kc;              // next sibling: same parent, next rank
+    const bool child = d < L;                  // first child: one position deeper
+    const float lsib = sib ? sm.lp[(d - 1) * kc + rk + 1] : 0.f;
+    const float lchild = child ? sm.lp[d * kc] : 0.f;
+    const float ssib = __fadd_rn(ps, lsib);
+    const float schild = __fadd_rn(sc, lchild);
+    const int cslot = next_slot;
+    __syncwarp();
+    if (lane == 0) {
+      sm.nd_parent[node] = par;
+      sm.nd_rank[node] = rk;
+      sm.nd_depth[node] = d;
+      sm.nd_score[node] = sc;
+      sm.sc[slot] = ssib;
+      sm.ps[slot] = ps;
+      sm.mt[slot] = pack_meta(par, d, rk + 1);
+      if (child) {
+        sm.sc[cslot] = schild;
+        sm.ps[cslot] = sc;
+        sm.mt[cslot] = pack_meta(node, d + 1, 0);
+      }
+    }
+    const uint32_t ksh = sib ? score_key(ssib) : 0u, ksl = sib ? ~(packed + tc.unit(d)) : 0u;
+    const uint32_t kch = score_key(schild), kcl = ~(packed + tc.unit(d + 1));
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      if (slot == lane + 32 * e) { kh[e] = ksh; kl[e] = ksl; }
+      if (child && cslot == lane + 32 * e) { kh[e] = kch; kl[e] = kcl; }
+    }
+    if (child) ++next_slot;
+    __syncwarp();
+  }
+  return pops;
+}
+
+// Tournament queue for large budgets (see the file comment).  Returns the
+// number of pops.
+__device__ __forceinline__ int heap_tournament(const BuildSmem& sm, int L, int B, int kc, TieCode tc, int lane) {
+  // cached best of blocks `lane` and `lane + 32`
+  Best b0{0u, 0u, -1}, b1{0u, 0u, -1};
+  int next_slot = 0;
+  if (B > 0) {   // the frontier starts with the best token of position 1
+    const float s0 = __fadd_rn(0.f, sm.lp[0]);
+    const uint32_t k0 = score_key(s0), t0 = ~tc.unit(1);
+    if (lane == 0) {
+      sm.key[0] = make_uint2(k0, t0);
+      sm.sc[0] = s0;
+      sm.ps[0] = 0.f;
+      sm.mt[0] = pack_meta(0, 1, 0);
+      b0 = Best{k0, t0, 0};
+    }
+    next_slot = 1;
+  }
+  __syncwarp();
+  // re-reduce block `blk` from shared memory into its owner's cached best
+  auto refresh = [&](int blk) {
+    const int s = 32 * blk + lane;
+    Best c{0u, 0u, -1};
+    if (s < next_slot) {
+      const uint2 k = sm.key[s];
+      c = Best{k.x, k.y, s};
+    }
+    const Best w = warp_best(c, sm);
+    if (lane == (blk & 31)) {
+      if (blk < 32) b0 = w;
+      else b1 = w;
+    }
+  };
+  int pops = 0;
+  while (pops < B) {
+    const Best lb = (b1.hi != 0 && (b0.hi == 0 || best_before(b1, b0, sm))) ? b1 : b0;
+    const Best top = warp_best(lb, sm);
+    if (top.hi == 0) break;   // frontier empty
+    const int slot = top.slot;
+    const uint32_t meta = sm.mt[slot];
+    const float sc = sm.sc[slot], ps = sm.ps[slot];
+    const uint32_t packed = ~top.lo;                     // the popped entry's packed ranks
+    const int par = meta_parent(meta), d = meta_depth(meta), rk = meta_rank(meta);
+    const int node = ++pops;
+    const bool sib = rk + 1 < kc;              // next sibling: same parent, next rank
+    const bool child = d < L;                  // first child: one position deeper
+    const float lsib = sib ? sm.lp[(d - 1) * kc + rk + 1] : 0.f;
+    const float lchild = child ? sm.lp[d * kc] : 0.f;
+    const float ssib = __fadd_rn(ps, lsib);
+    const float schild = __fadd_rn(sc, lchild);
+    const int cslot = next_slot;
+    __syncwarp();
+    if (lane == 0) {
+      sm.nd_parent[node] = par;
+      sm.nd_rank[node] = rk;
+      sm.nd_depth[node] = d;
+      sm.nd_score[node] = sc;
+      sm.key[slot] = sib ? make_uint2(score_key(ssib), ~(packed + tc.unit(d))) : make_uint2(0u, 0u);
+      sm.sc[slot] = ssib;
+      sm.ps[slot] = ps;
+      sm.mt[slot] = pack_meta(par, d, rk + 1);
+      if (child) {
+        sm.key[cslot] = make_uint2(score_key(schild), ~(packed + tc.unit(d + 1)));
+        sm.sc[cslot] = schild;
+        sm.ps[cslot] = sc;
+        sm.mt[cslot] = pack_meta(node, d + 1, 0);
+      }
+    }
+    if (child) ++next_slot;
+    __syncwarp();
+    refresh(slot >> 5);
+    if (child && (cslot >> 5) != (slot >> 5)) refresh(cslot >> 5);
+  }
+  return pops;
+}
+
 __global__ void __launch_bounds__(BUILD_THREADS, 1)
 build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
              const int32_t* __restrict__ root_token, int L, int K, int B, int kc, TieCode tc,
@@ -185,76 +336,10 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
       sm.nd_depth[0] = 0;
       sm.nd_score[0] = 0.f;
     }
-    // cached best of blocks `lane` and `lane + 32`
-    Best b0{0u, 0u, -1}, b1{0u, 0u, -1};
-    int next_slot = 0;
-    if (B > 0) {   // the frontier starts with the best token of position 1
-      const float s0 = __fadd_rn(0.f, sm.lp[0]);
-      const uint32_t k0 = score_key(s0), t0 = ~tc.unit(1);
-      if (lane == 0) {
-        sm.key[0] = make_uint2(k0, t0);
-        sm.sc[0] = s0;
-        sm.ps[0] = 0.f;
-        sm.mt[0] = pack_meta(0, 1, 0);
-        b0 = Best{k0, t0, 0};
-      }
-      next_slot = 1;
-    }
-    __syncwarp();
-    // re-reduce block `blk` from shared memory into its owner's cached best
-    auto refresh = [&](int blk) {
-      const int s = 32 * blk + lane;
-      Best c{0u, 0u, -1};
-      if (s < next_slot) {
-        const uint2 k = sm.key[s];
-        c = Best{k.x, k.y, s};
-      }
-      const Best w = warp_best(c, sm);
-      if (lane == (blk & 31)) {
-        if (blk < 32) b0 = w;
-        else b1 = w;
-      }
-    };
-    int pops = 0;
-    while (pops < B) {
-      const Best lb = (b1.hi != 0 && (b0.hi == 0 || best_before(b1, b0, sm))) ? b1 : b0;
-      const Best top = warp_best(lb, sm);
-      if (top.hi == 0) break;   // frontier empty
-      const int slot = top.slot;
-      const uint32_t meta = sm.mt[slot];
-      const float sc = sm.sc[slot], ps = sm.ps[slot];
-      const uint32_t packed = ~top.lo;                     // the popped entry's packed ranks
-      const int par = meta_parent(meta), d = meta_depth(meta), rk = meta_rank(meta);
-      const int node = ++pops;
-      const bool sib = rk + 1 < kc;              // next sibling: same parent, next rank
-      const bool child = d < L;                  // first child: one position deeper
-      const float lsib = sib ? sm.lp[(d - 1) * kc + rk + 1] : 0.f;
-      const float lchild = child ? sm.lp[d * kc] : 0.f;
-      const float ssib = __fadd_rn(ps, lsib);
-      const float schild = __fadd_rn(sc, lchild);
-      const int cslot = next_slot;
-      __syncwarp();
-      if (lane == 0) {
-        sm.nd_parent[node] = par;
-        sm.nd_rank[node] = rk;
-        sm.nd_depth[node] = d;
-        sm.nd_score[node] = sc;
-        sm.key[slot] = sib ? make_uint2(score_key(ssib), ~(packed + tc.unit(d))) : make_uint2(0u, 0u);
-        sm.sc[slot] = ssib;
-        sm.ps[slot] = ps;
-        sm.mt[slot] = pack_meta(par, d, rk + 1);
-        if (child) {
-          sm.key[cslot] = make_uint2(score_key(schild), ~(packed + tc.unit(d + 1)));
-          sm.sc[cslot] = schild;
-          sm.ps[cslot] = sc;
-          sm.mt[cslot] = pack_meta(node, d + 1, 0);
-        }
-      }
-      if (child) ++next_slot;
-      __syncwarp();
-      refresh(slot >> 5);
-      if (child && (cslot >> 5) != (slot >> 5)) refresh(cslot >> 5);
-    }
+    int pops;
+    if (n <= 32 * 3) pops = heap_registers<3>(sm, L, B, kc, tc, lane);
+    else if (n <= 32 * 9) pops = heap_registers<9>(sm, L, B, kc, tc, lane);
+    else pops = heap_tournament(sm, L, B, kc, tc, lane);
     if (lane == 0) s_pops = pops;
   }
   __syncthreads();

@@ -44,6 +44,7 @@ constexpr int TOPK_THREADS = 512;
 constexpr int TOPK_MAX_VPT = 6;            // 16-byte vectors per thread
 constexpr int TOPK_MAX_CAND = 16384;       // merge capacity (candidates per row)
 constexpr int TOPK_MAX_CPR = 128;          // chunks per row
+constexpr int TOPK_RANK_MAX = 2048;        // merge by rank counting up to this many candidates
 constexpr int TOPK_ID_BITS = 20;           // V <= 2^20
 constexpr uint32_t TOPK_ID_MASK = (1u << TOPK_ID_BITS) - 1u;
 constexpr int LID_BITS = 15;               // chunk <= 24576 < 32768
@@ -87,13 +88,14 @@ struct TopkWs {
   uint32_t* ticket;          // [rows]
   double2* stats;            // [rows][cpr]: (chunk max, sum of exp(z - max))
   int* count;                // [rows][cpr]
+  uint32_t* thr;             // [rows][cpr] the chunk's threshold value key
   unsigned long long* cand;  // [rows][cpr][cap]
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 inline size_t topk_ws_bytes(int rows, const TopkPlan& p) {
-  return align256((size_t)rows * 4) + align256((size_t)rows * p.cpr * 16) + align256((size_t)rows * p.cpr * 4) +
+  return align256((size_t)rows * 4) + align256((size_t)rows * p.cpr * 16) + 2 * align256((size_t)rows * p.cpr * 4) +
          align256((size_t)rows * p.cand * 8);
 }
 
@@ -105,6 +107,8 @@ inline TopkWs topk_ws_carve(void* ws, int rows, const TopkPlan& p) {
   w.stats = (double2*)b;
   b += align256((size_t)rows * p.cpr * 16);
   w.count = (int*)b;
+  b += align256((size_t)rows * p.cpr * 4);
+  w.thr = (uint32_t*)b;
   b += align256((size_t)rows * p.cpr * 4);
   w.cand = (unsigned long long*)b;
   return w;
@@ -535,6 +539,7 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
     if (use_table) tot *= exp64(-md, s_tab);           // sum of exp(z) -> sum of exp(z - m)
     ws.stats[(size_t)row * plan.cpr + c] = make_double2(md, tot);
     ws.count[(size_t)row * plan.cpr + c] = s_count < plan.cap ? s_count : plan.cap;
+    ws.thr[(size_t)row * plan.cpr + c] = tval;
   }
   __threadfence();
   __syncthreads();
@@ -556,21 +561,27 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   __shared__ double2 s_st[TOPK_MAX_CPR];
   __shared__ int s_ncand;
   __shared__ double s_lse;
+  __shared__ uint32_t s_floor;
+  // Every chunk emitted at least min(K, its length) logits at or above its
+  // threshold value, so the row's K-th best value is at least the largest
+  // chunk threshold: candidates below it cannot be selected.
+  if (tid == 0) s_floor = 0;
+  __syncthreads();
+  uint32_t tmax = 0;
   for (int i = tid; i < plan.cpr; i += TOPK_THREADS) {
     s_cnt[i] = __ldcg(&ws.count[(size_t)row * plan.cpr + i]);
     s_st[i] = __ldcg(&ws.stats[(size_t)row * plan.cpr + i]);
+    const int li = (int)min((long long)plan.chunk, (long long)V - (long long)i * plan.chunk);
+    if (li >= K) tmax = max(tmax, __ldcg(&ws.thr[(size_t)row * plan.cpr + i]));
   }
+  tmax = __reduce_max_sync(0xffffffffu, tmax);
+  if (tid == 0) s_count = 0;
   for (int i = tid; i < kpow; i += TOPK_THREADS) win[i] = 0ull;
+  if ((tid & 31) == 0 && tmax) atomicMax(&s_floor, tmax);
   __syncthreads();
   if (tid == 0) {
-    int off = 0;
     double M = -INFINITY;
-    for (int i = 0; i < plan.cpr; ++i) {
-      s_off[i] = off;
-      off += s_cnt[i];
-      M = fmax(M, s_st[i].x);
-    }
-    s_ncand = off;
+    for (int i = 0; i < plan.cpr; ++i) M = fmax(M, s_st[i].x);
     double S = 0.0;
     if (M > -INFINITY)
       for (int i = 0; i < plan.cpr; ++i)
@@ -578,28 +589,51 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
     s_lse = M + log(S);
     ws.ticket[row] = 0;   // leave the workspace ready for the next call
   }
-  __syncthreads();
+  const unsigned long long floor_key = (unsigned long long)s_floor << TOPK_ID_BITS;
+  // gather the candidates at or above the floor
   {
     constexpr int UNR = 4;   // issue several candidate loads before storing any
     const int slots = plan.cpr * plan.cap;
     for (int s0 = tid; s0 < slots; s0 += UNR * TOPK_THREADS) {
       unsigned long long v[UNR];
-      int dst[UNR];
+      bool ok[UNR];
 #pragma unroll
       for (int u = 0; u < UNR; ++u) {
         const int sl = s0 + u * TOPK_THREADS;
         const int ci = sl / plan.cap, j = sl - ci * plan.cap;
-        dst[u] = (sl < slots && j < s_cnt[ci]) ? s_off[ci] + j : -1;
-        v[u] = dst[u] >= 0 ? __ldcg(cand_row + sl) : 0ull;
+        ok[u] = sl < slots && j < s_cnt[ci];
+        v[u] = ok[u] ? __ldcg(cand_row + sl) : 0ull;
       }
 #pragma unroll
-      for (int u = 0; u < UNR; ++u)
-        if (dst[u] >= 0) sc[dst[u]] = v[u];
+      for (int u = 0; u < UNR; ++u) {
+        if (ok[u] && v[u] >= floor_key) {
+          const int slot = atomicAdd(&s_count, 1);
+          if (slot < plan.cand) sc[slot] = v[u];
+        }
+      }
     }
   }
+  __syncthreads();
+  const int ncand = min(s_count, plan.cand);
+  const double lse = s_lse;
+  if (ncand <= TOPK_RANK_MAX) {
+    // rank by counting (keys are unique): selects and orders in one pass
+    for (int i = tid; i < ncand; i += TOPK_THREADS) {
+      const unsigned long long k = sc[i];
+      int rank = 0;
+      for (int j = 0; j < ncand; ++j) rank += sc[j] > k;
+      if (rank < K) {
+        const uint32_t vkey = (uint32_t)(k >> TOPK_ID_BITS);
+        out_ids[(size_t)row * K + rank] = (int)(TOPK_ID_MASK - (uint32_t)(k & TOPK_ID_MASK));
+        out_lp[(size_t)row * K + rank] = (float)((double)key_value<DT>(vkey) - lse);   // one rounding of the fp64 value
+      }
+    }
+    if (out_lse != nullptr && tid == 0) out_lse[row] = (float)lse;
+    return;
+  }
+  // many ties at the floor: radix select of the top K, then a bitonic sort
   if (tid == 0) s_count = 0;
   __syncthreads();
-  const int ncand = s_ncand;
   const int per = (ncand + TOPK_THREADS - 1) / TOPK_THREADS;
   auto geach = [&](auto f) {
     for (int i = 0; i < per; ++i) {
@@ -618,8 +652,7 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
     }
   }
   __syncthreads();
-  // bitonic sort, descending
-  for (int size = 2; size <= kpow; size <<= 1) {
+  for (int size = 2; size <= kpow; size <<= 1) {     // bitonic sort, descending
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       for (int i = tid; i < kpow / 2; i += TOPK_THREADS) {
         const int lo = 2 * stride * (i / stride) + (i % stride);
@@ -631,7 +664,6 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
       __syncthreads();
     }
   }
-  const double lse = s_lse;
   for (int i = tid; i < K; i += TOPK_THREADS) {
     const unsigned long long k = win[i];
     const uint32_t vkey = (uint32_t)(k >> TOPK_ID_BITS);
@@ -641,7 +673,6 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   if (out_lse != nullptr && tid == 0) out_lse[row] = (float)lse;
 }
 
-// Dynamic shared memory: the staged chunk, later reused by the merge.
 inline size_t topk_smem_bytes(const TopkPlan& p, int K) {
   int kpow = 1;
   while (kpow < K) kpow <<= 1;

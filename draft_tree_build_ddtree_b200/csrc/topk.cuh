@@ -13,13 +13,11 @@
 //    register passes stalled on instruction fetch).
 //  * The chunk's sum of exp(z - max) is taken in fp64 so that
 //    log q = z - lse, rounded once to fp32, is the correctly rounded value
-//    in all but vanishingly rare cases.  For bf16 logits exp(z) comes from a
-//    65536-entry fp64 table indexed by the logit's bit pattern (built once
-//    per device with a table-driven exponential, Tang's method: 2^(k/64)
-//    from a table times a degree-5 polynomial of the reduced argument), so
-//    the sum costs one load and one add per logit.  bf16 logits sit on a coarse grid, many prefixes tie
-//    exactly in real arithmetic, and only a correctly rounded log-prob
-//    table orders them reproducibly.
+//    in all but vanishingly rare cases.  exp is a table-driven fp64
+//    exponential (Tang's method: 2^(k/64) from a 64-entry table times a
+//    degree-5 polynomial of the reduced argument).  bf16 logits sit on a
+//    coarse grid, many prefixes tie exactly in real arithmetic, and only a
+//    correctly rounded log-prob table orders them reproducibly.
 //  * The chunk's threshold value (the K'-th largest logit, K' = min(K,
 //    chunk length)) comes, for bf16, from one 256-bin histogram anchored at
 //    the chunk maximum: each bin is one bf16 value, so one pass finds it
@@ -44,7 +42,7 @@ constexpr int TOPK_THREADS = 512;
 constexpr int TOPK_MAX_VPT = 6;            // 16-byte vectors per thread
 constexpr int TOPK_MAX_CAND = 16384;       // merge capacity (candidates per row)
 constexpr int TOPK_MAX_CPR = 128;          // chunks per row
-constexpr int TOPK_RANK_MAX = 2048;        // merge by rank counting up to this many candidates
+constexpr int TOPK_MERGE_SMALL = 512;      // merge ranks by counting up to this many keys >= the K-th value
 constexpr int TOPK_ID_BITS = 20;           // V <= 2^20
 constexpr uint32_t TOPK_ID_MASK = (1u << TOPK_ID_BITS) - 1u;
 constexpr int LID_BITS = 15;               // chunk <= 24576 < 32768
@@ -133,21 +131,6 @@ __device__ __forceinline__ double exp64(double x, const double* tab) {
   return __hiloint2double(__double2hiint(y) + ((k >> 6) << 20), __double2loint(y));
 }
 
-// exp(z) in fp64 for every bf16 bit pattern z, built once per device by
-// exp_bf16_table_kernel.  With it the sum of exp(z - m) over a chunk is one
-// table load and one fp64 add per logit, scaled by exp(-m) once.
-__device__ double g_exp_bf16[65536];
-
-__global__ void exp_bf16_table_kernel() {
-  __shared__ double tab[64];
-  if (threadIdx.x < 64) tab[threadIdx.x] = EXP64_TABLE[threadIdx.x];
-  __syncthreads();
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < 65536) g_exp_bf16[i] = exp64((double)bf16_bits_to_f32((uint16_t)i), tab);
-}
-
-// Table use is exact when the chunk maximum keeps every sum in range.
-constexpr double EXP_TABLE_MAX_M = 600.0;
 
 // ---------------------------------------------------------------------------
 // Block-wide radix selection of the need-th largest key.
@@ -260,6 +243,7 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   __shared__ uint32_t hist[256];
   __shared__ int bcast[4];
   __shared__ uint32_t red_u[TOPK_THREADS / 32];
+  __shared__ uint32_t red_w[TOPK_THREADS / 32];
   __shared__ double red_d[TOPK_THREADS / 32];
   __shared__ double s_tab[64];
   __shared__ int s_count;
@@ -346,6 +330,31 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
     nan_seen = mag_lo > 0x7F80u || mag_hi > 0x7F800000u;
     // the order key of the maximum (any element equal to it has this key)
     kmax = mx > -INFINITY ? key32_of_f32(mx) >> 16 : 0u;
+    // Lower bound of the chunk's K'-th largest logit: the thread maxima are
+    // distinct elements, so if every warp contributes its r-th largest thread
+    // maximum (r = ceil(K'/warps)), at least K' logits are >= the smallest of
+    // those.  Only logits above the bound enter the window histogram.
+    {
+      constexpr int NW = TOPK_THREADS / 32;
+      const int r = (kloc + NW - 1) / NW;
+      uint32_t wk = 0;
+      if (r <= 32) {
+        uint32_t x = kmax;                      // this thread's maximum (0: none)
+        const int lane = tid & 31;
+#pragma unroll
+        for (int k = 2; k <= 32; k <<= 1) {     // bitonic sort across the warp, descending
+#pragma unroll
+          for (int j = k >> 1; j > 0; j >>= 1) {
+            const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
+            const bool lower = (lane & j) == 0;
+            const bool desc = (lane & k) == 0 || k == 32;
+            x = (lower == desc) ? max(x, y) : min(x, y);
+          }
+        }
+        wk = __shfl_sync(0xffffffffu, x, r - 1);
+      }
+      if ((tid & 31) == 0) red_w[tid >> 5] = wk;
+    }
     if (mx == -INFINITY) {                      // only -inf (or nothing) here: key of -inf if present
       for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
         uint32_t k[EPV];
@@ -380,10 +389,14 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   // ---- fp64 sum of exp(z - m); bf16: max-anchored window histogram ----
   double s0 = 0.0, s1 = 0.0;
   const bool m_finite = m > -INFINITY;
-  const bool use_table = DT == DDTREE_BF16 && md <= EXP_TABLE_MAX_M && md >= -EXP_TABLE_MAX_M;
   if (DT == DDTREE_BF16) {
-    // values below the window's lowest bin skip the histogram with one compare
-    const float wlow = kmax >= 255u ? bf16_of_key16(kmax - 255u) : -INFINITY;
+    // values below the window's lowest bin, or below the K'-th value's lower
+    // bound, skip the histogram with one compare
+    uint32_t wbound = red_w[0];
+#pragma unroll
+    for (int i = 1; i < TOPK_THREADS / 32; ++i) wbound = red_w[i] < wbound ? red_w[i] : wbound;
+    const uint32_t wkey = max(wbound, kmax >= 255u ? kmax - 255u : 0u);
+    const float wlow = wkey > 0u ? bf16_of_key16(wkey) : -INFINITY;
     for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
       const uint4 v = chunk_s[vi];
       const int valid = len - vi * EPV;
@@ -392,9 +405,7 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
         if (j < valid) {
           const uint32_t bits = elem_bits<DT>(v, j);
           const float z = bf16_bits_to_f32((uint16_t)bits);
-          double e;
-          if (use_table) e = g_exp_bf16[bits];                            // exp(z); scaled below
-          else e = m_finite ? exp64((double)z - md, s_tab) : 0.0;
+          const double e = m_finite ? exp64((double)z - md, s_tab) : 0.0;
           if (j & 1) s1 += e; else s0 += e;
           if (z >= wlow) {
             const uint32_t d = kmax - key16_of_bf16((uint16_t)bits);
@@ -536,7 +547,6 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   if (tid == 0) {
     double tot = 0.0;
     for (int i = 0; i < TOPK_THREADS / 32; ++i) tot += red_d[i];
-    if (use_table) tot *= exp64(-md, s_tab);           // sum of exp(z) -> sum of exp(z - m)
     ws.stats[(size_t)row * plan.cpr + c] = make_double2(md, tot);
     ws.count[(size_t)row * plan.cpr + c] = s_count < plan.cap ? s_count : plan.cap;
     ws.thr[(size_t)row * plan.cpr + c] = tval;
@@ -555,17 +565,17 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   unsigned long long* sc = (unsigned long long*)smem_raw;   // [plan.cand]
   int kpow = 1;
   while (kpow < K) kpow <<= 1;
-  unsigned long long* win = sc + plan.cand;                 // [kpow]
-  __shared__ int s_off[TOPK_MAX_CPR];
+  unsigned long long* win = sc + plan.cand;                 // [max(kpow, TOPK_MERGE_SMALL)]
   __shared__ int s_cnt[TOPK_MAX_CPR];
   __shared__ double2 s_st[TOPK_MAX_CPR];
-  __shared__ int s_ncand;
   __shared__ double s_lse;
   __shared__ uint32_t s_floor;
+  __shared__ int s_m;
+  const int lane = tid & 31;
   // Every chunk emitted at least min(K, its length) logits at or above its
   // threshold value, so the row's K-th best value is at least the largest
   // chunk threshold: candidates below it cannot be selected.
-  if (tid == 0) s_floor = 0;
+  if (tid == 0) { s_floor = 0; s_count = 0; s_m = 0; }
   __syncthreads();
   uint32_t tmax = 0;
   for (int i = tid; i < plan.cpr; i += TOPK_THREADS) {
@@ -575,66 +585,97 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
     if (li >= K) tmax = max(tmax, __ldcg(&ws.thr[(size_t)row * plan.cpr + i]));
   }
   tmax = __reduce_max_sync(0xffffffffu, tmax);
-  if (tid == 0) s_count = 0;
-  for (int i = tid; i < kpow; i += TOPK_THREADS) win[i] = 0ull;
-  if ((tid & 31) == 0 && tmax) atomicMax(&s_floor, tmax);
+  if (lane == 0 && tmax) atomicMax(&s_floor, tmax);
   __syncthreads();
-  if (tid == 0) {
+  if (tid < 32) {   // lse from the chunk statistics, combined across the lanes of warp 0
     double M = -INFINITY;
-    for (int i = 0; i < plan.cpr; ++i) M = fmax(M, s_st[i].x);
+    for (int i = lane; i < plan.cpr; i += 32) M = fmax(M, s_st[i].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmax(M, __shfl_xor_sync(0xffffffffu, M, o));
     double S = 0.0;
     if (M > -INFINITY)
-      for (int i = 0; i < plan.cpr; ++i)
+      for (int i = lane; i < plan.cpr; i += 32)
         if (s_st[i].x > -INFINITY) S += s_st[i].y * exp64(s_st[i].x - M, s_tab);
-    s_lse = M + log(S);
-    ws.ticket[row] = 0;   // leave the workspace ready for the next call
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);   // same value on every lane
+    if (lane == 0) {
+      s_lse = M + log(S);
+      ws.ticket[row] = 0;   // leave the workspace ready for the next call
+    }
   }
+  // gather the candidates at or above the floor (one shared atomic per warp and round)
   const unsigned long long floor_key = (unsigned long long)s_floor << TOPK_ID_BITS;
-  // gather the candidates at or above the floor
   {
     constexpr int UNR = 4;   // issue several candidate loads before storing any
     const int slots = plan.cpr * plan.cap;
-    for (int s0 = tid; s0 < slots; s0 += UNR * TOPK_THREADS) {
+    for (int s0 = tid & ~31; s0 < slots; s0 += UNR * TOPK_THREADS) {   // warp-uniform trip count
       unsigned long long v[UNR];
       bool ok[UNR];
 #pragma unroll
       for (int u = 0; u < UNR; ++u) {
-        const int sl = s0 + u * TOPK_THREADS;
+        const int sl = s0 + lane + u * TOPK_THREADS;
         const int ci = sl / plan.cap, j = sl - ci * plan.cap;
         ok[u] = sl < slots && j < s_cnt[ci];
         v[u] = ok[u] ? __ldcg(cand_row + sl) : 0ull;
       }
 #pragma unroll
       for (int u = 0; u < UNR; ++u) {
-        if (ok[u] && v[u] >= floor_key) {
-          const int slot = atomicAdd(&s_count, 1);
-          if (slot < plan.cand) sc[slot] = v[u];
+        const bool take = ok[u] && v[u] >= floor_key;
+        const unsigned bal = __ballot_sync(0xffffffffu, take);
+        if (bal) {
+          int base = 0;
+          if (lane == 0) base = atomicAdd(&s_count, __popc(bal));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (take) sc[base + __popc(bal & ((1u << lane) - 1u))] = v[u];
         }
       }
     }
   }
   __syncthreads();
-  const int ncand = min(s_count, plan.cand);
+  const int ncand = s_count;   // <= plan.cand: every chunk wrote at most cap slots
   const double lse = s_lse;
-  if (ncand <= TOPK_RANK_MAX) {
-    // rank by counting (keys are unique): selects and orders in one pass
-    for (int i = tid; i < ncand; i += TOPK_THREADS) {
-      const unsigned long long k = sc[i];
-      int rank = 0;
-      for (int j = 0; j < ncand; ++j) rank += sc[j] > k;
-      if (rank < K) {
-        const uint32_t vkey = (uint32_t)(k >> TOPK_ID_BITS);
-        out_ids[(size_t)row * K + rank] = (int)(TOPK_ID_MASK - (uint32_t)(k & TOPK_ID_MASK));
-        out_lp[(size_t)row * K + rank] = (float)((double)key_value<DT>(vkey) - lse);   // one rounding of the fp64 value
+  const int per = (ncand + TOPK_THREADS - 1) / TOPK_THREADS;
+  // the K-th largest value among the candidates: every key above it and the
+  // ties at it form the set that holds the row's top K
+  auto veach = [&](auto f) {
+    for (int i = 0; i < per; ++i) {
+      const int idx = i * TOPK_THREADS + tid;
+      f(idx < ncand ? (uint32_t)(sc[idx] >> TOPK_ID_BITS) : 0u);
+    }
+  };
+  const RadixOut<uint32_t> vt = radix_kth<uint32_t>(veach, T::KEY_BITS, K, hist, bcast);
+  const int nsel = vt.above + vt.eq;
+  if (nsel <= TOPK_MERGE_SMALL) {
+    for (int i = 0; i < per; ++i) {
+      const int idx = i * TOPK_THREADS + tid;
+      if (idx < ncand) {
+        const unsigned long long k = sc[idx];
+        if ((uint32_t)(k >> TOPK_ID_BITS) >= vt.t) win[atomicAdd(&s_m, 1)] = k;
       }
+    }
+    __syncthreads();
+    // rank by counting (keys are unique): g threads share one key's count
+    int g = 32;
+    while (g > 1 && nsel * g > TOPK_THREADS) g >>= 1;
+    const int q = tid / g, part = tid - q * g;
+    unsigned long long k = 0ull;
+    int rank = 0;
+    if (q < nsel) {
+      k = win[q];
+      for (int j = part; j < nsel; j += g) rank += win[j] > k;
+    }
+    for (int o = g >> 1; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+    if (q < nsel && part == 0 && rank < K) {
+      const uint32_t vkey = (uint32_t)(k >> TOPK_ID_BITS);
+      out_ids[(size_t)row * K + rank] = (int)(TOPK_ID_MASK - (uint32_t)(k & TOPK_ID_MASK));
+      out_lp[(size_t)row * K + rank] = (float)((double)key_value<DT>(vkey) - lse);   // one rounding of the fp64 value
     }
     if (out_lse != nullptr && tid == 0) out_lse[row] = (float)lse;
     return;
   }
-  // many ties at the floor: radix select of the top K, then a bitonic sort
+  // many ties at the K-th value: radix select of the top K keys, then a bitonic sort
   if (tid == 0) s_count = 0;
   __syncthreads();
-  const int per = (ncand + TOPK_THREADS - 1) / TOPK_THREADS;
   auto geach = [&](auto f) {
     for (int i = 0; i < per; ++i) {
       const int idx = i * TOPK_THREADS + tid;
@@ -676,7 +717,7 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
 inline size_t topk_smem_bytes(const TopkPlan& p, int K) {
   int kpow = 1;
   while (kpow < K) kpow <<= 1;
-  const size_t merge = (size_t)(p.cand + kpow) * 8;
+  const size_t merge = (size_t)(p.cand + (kpow > TOPK_MERGE_SMALL ? kpow : TOPK_MERGE_SMALL)) * 8;
   const size_t chunk = (size_t)(p.chunk + 16) * 4;    // worst case fp32 elements, + one ragged vector
   return merge > chunk ? merge : chunk;
 }

@@ -106,9 +106,7 @@ size_t ddtree_topk_workspace_bytes(int rows, int V, int K);
  * NaN logits set DDTREE_STATUS_NONFINITE; -inf is allowed and ranks last;
  * -0.0 ranks equal to +0.0.
  * lp is the fp64 value z - lse rounded once to fp32 (the sum of exp is taken
- * in fp64).  The first bf16 call on a device builds a 512 KiB table of
- * exp(z) for every bf16 value in static device memory and synchronizes
- * `stream` once; make it before any stream capture.
+ * in fp64).
  */
 int ddtree_topk(const void* logits, int dtype, int rows, int V, long long row_stride,
                 int K, int32_t* ids, float* lp, float* lse,

@@ -102,9 +102,14 @@ struct BuildSmem {
   float* nd_score;
 };
 
-inline size_t build_smem_bytes(int L, int kc, int B) {
+__host__ __device__ inline size_t build_smem_bytes(int L, int kc, int B) {
   const size_t n = (size_t)B + 1;
   return (size_t)L * kc * 4 + n * (8 + 4 + 4 + 4) + n * 4 * 4;
+}
+inline size_t enum_smem_bytes();
+// with the enumeration arrays after the heap's
+inline size_t build_smem_bytes_enum(int L, int kc, int B) {
+  return ((build_smem_bytes(L, kc, B) + 15) & ~(size_t)15) + enum_smem_bytes();
 }
 
 // a before b in the pop order
@@ -293,9 +298,243 @@ __device__ __forceinline__ int heap_tournament(const BuildSmem& sm, int L, int B
   return pops;
 }
 
+
+// ---------------------------------------------------------------------------
+// Threshold enumeration (all threads of the CTA).
+//
+// The heap pops prefixes in one total order: score descending, then rank
+// tuple ascending.  A child never precedes its parent (lp <= 0 and fp32
+// addition is monotone) and a next sibling never precedes its elder sibling
+// (lp sorted within a position), so the first B pops are exactly the B
+// largest prefixes of that order, in order.  This path finds them without
+// popping one at a time:
+//  1. A score threshold t that at least B prefixes reach: the B-th largest
+//     score among the prefixes (0,...,0,r) -- greedy chain, one deviation at
+//     the last position -- which are real prefixes with their exact scores.
+//  2. Every prefix scoring >= t, one depth level per step: a node's children
+//     that qualify are the ranks 0..c-1 (scores fall with the rank), c found
+//     by binary search; a block scan places them.  Prefix-closed by (1).
+//  3. Order the enumerated set by (score, tuple): 64-bit keys (score key,
+//     packed leading ranks) with an exact tuple walk on equal keys; the first
+//     B entries are the pops.
+// If the set exceeds ENUM_CAP entries the caller runs the heap instead.
+// ---------------------------------------------------------------------------
+constexpr int ENUM_CAP = 4096;
+constexpr uint32_t ENUM_ROOT = 0x1FFFu;        // parent field of depth-1 entries
+
+__device__ __forceinline__ uint32_t e_pack(uint32_t parent, int depth, int rank) {
+  return parent | ((uint32_t)depth << 13) | ((uint32_t)rank << 19);
+}
+__device__ __forceinline__ uint32_t e_parent(uint32_t m) { return m & 0x1FFFu; }
+__device__ __forceinline__ int e_depth(uint32_t m) { return (int)((m >> 13) & 0x3Fu); }
+__device__ __forceinline__ int e_rank(uint32_t m) { return (int)(m >> 19); }
+
+struct EnumSmem {
+  float* score;                 // [ENUM_CAP]
+  uint32_t* meta;               // [ENUM_CAP] parent entry, depth, rank
+  unsigned long long* key;      // [ENUM_CAP] score key << 32 | tie key
+  int* off;                     // [ENUM_CAP + 1] per-level child counts -> offsets
+  uint16_t* ord;                // [ENUM_CAP] sorted entry indices
+  uint16_t* pos;                // [ENUM_CAP] node index of an entry (0: not selected)
+};
+
+inline size_t enum_smem_bytes() { return (size_t)ENUM_CAP * (4 + 4 + 8 + 2 + 2) + (ENUM_CAP + 1) * 4; }
+
+// Lexicographic tuple comparison of two enumerated entries (a proper prefix
+// is smaller): lift the deeper entry, then walk both up to a common parent.
+__device__ __forceinline__ bool e_tuple_less(int a, int b, const uint32_t* meta) {
+  uint32_t ma = meta[a], mb = meta[b];
+  int da = e_depth(ma), db = e_depth(mb);
+  int ra = e_rank(ma), rb = e_rank(mb);
+  uint32_t pa = e_parent(ma), pb = e_parent(mb);
+  const bool a_shorter = da < db;
+  while (da > db) { ma = meta[pa]; ra = e_rank(ma); pa = e_parent(ma); --da; }
+  while (db > da) { mb = meta[pb]; rb = e_rank(mb); pb = e_parent(mb); --db; }
+  if (pa == pb && ra == rb) return a_shorter;
+  while (pa != pb) {
+    ma = meta[pa]; ra = e_rank(ma); pa = e_parent(ma);
+    mb = meta[pb]; rb = e_rank(mb); pb = e_parent(mb);
+  }
+  return ra < rb;
+}
+
+// entry a pops before entry b
+__device__ __forceinline__ bool e_before(int a, int b, const EnumSmem& es) {
+  const unsigned long long ka = es.key[a], kb = es.key[b];
+  if (ka != kb) return ka > kb;
+  return e_tuple_less(a, b, es.meta);
+}
+
+// In-place exclusive scan of v[0..m) by the whole block; returns the total.
+__device__ __forceinline__ int block_exclusive_scan(int* v, int m, int* warp_tot) {
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int per = (m + BUILD_THREADS - 1) / BUILD_THREADS;
+  const int b0 = tid * per, b1 = min(m, b0 + per);
+  int sum = 0;
+  for (int i = b0; i < b1; ++i) sum += v[i];
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[wid] = incl;
+  __syncthreads();
+  int wbase = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < BUILD_THREADS / 32; ++w) {
+    const int t = warp_tot[w];
+    if (w < wid) wbase += t;
+    total += t;
+  }
+  int run = wbase + incl - sum;
+  for (int i = b0; i < b1; ++i) {
+    const int c = v[i];
+    v[i] = run;
+    run += c;
+  }
+  __syncthreads();
+  return total;
+}
+
+// Returns the number of pops, or -1 when the enumeration exceeds ENUM_CAP.
+// Block-uniform.  Fills sm.nd_* for nodes 1..pops.
+__device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B, int kc, TieCode tc,
+                          uint32_t* hist, int* bcast, int* warp_tot, float* chain, int* s_lev) {
+  const int tid = threadIdx.x;
+  // ---- 1. threshold: B-th best score among the one-deviation chain prefixes ----
+  if (tid == 0) {
+    float c = 0.f;
+    for (int d = 0; d < L; ++d) {
+      chain[d] = c;                               // score of (0,...,0) of length d
+      c = __fadd_rn(c, sm.lp[d * kc]);
+    }
+  }
+  __syncthreads();
+  uint32_t t = 1u;                                // every finite or -inf score
+  if ((long long)L * kc >= B) {
+    auto each = [&](auto f) {
+      for (int i = tid; i < L * kc; i += BUILD_THREADS) {
+        const int d = i / kc;
+        f(score_key(__fadd_rn(chain[d], sm.lp[i])));
+      }
+    };
+    t = radix_kth<uint32_t>(each, 32, B, hist, bcast).t;
+  }
+  // ---- 2. every prefix with score key >= t, level by level ----
+  // depth 1: children of the root
+  if (tid == 0) {
+    int lo = 0, hi = kc;                          // first rank failing the threshold
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (score_key(sm.lp[mid]) >= t) lo = mid + 1; else hi = mid;
+    }
+    s_lev[0] = 0;
+    s_lev[1] = lo;
+    s_lev[2] = lo > ENUM_CAP ? 1 : 0;
+  }
+  __syncthreads();
+  if (s_lev[2]) return -1;
+  int ls = 0, le = s_lev[1];
+  for (int r = tid; r < le; r += BUILD_THREADS) {
+    const float sc = __fadd_rn(0.f, sm.lp[r]);
+    es.score[r] = sc;
+    es.meta[r] = e_pack(ENUM_ROOT, 1, r);
+    const uint32_t code = (uint32_t)(r + 1) * tc.unit(1);
+    es.key[r] = ((unsigned long long)score_key(sc) << 32) | (uint32_t)~code;
+  }
+  __syncthreads();
+  for (int d = 1; d < L && le > ls; ++d) {        // parents at depth d, children at depth d+1
+    const int m = le - ls;
+    const float* lpd = sm.lp + d * kc;
+    for (int i = tid; i < m; i += BUILD_THREADS) {
+      const float ps = es.score[ls + i];
+      int lo = 0, hi = kc;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (score_key(__fadd_rn(ps, lpd[mid])) >= t) lo = mid + 1; else hi = mid;
+      }
+      es.off[i] = lo;
+    }
+    __syncthreads();
+    const int T = block_exclusive_scan(es.off, m, warp_tot);
+    if (le + T > ENUM_CAP) return -1;             // block-uniform
+    if (tid == 0) es.off[m] = T;
+    __syncthreads();
+    const uint32_t unit = tc.unit(d + 1);
+    for (int j = tid; j < T; j += BUILD_THREADS) {
+      int lo = 0, hi = m;                         // last parent with off <= j
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (es.off[mid] <= j) lo = mid; else hi = mid;
+      }
+      const int par = ls + lo;
+      const int r = j - es.off[lo];
+      const float sc = __fadd_rn(es.score[par], lpd[r]);
+      const int e = le + j;
+      es.score[e] = sc;
+      es.meta[e] = e_pack((uint32_t)par, d + 1, r);
+      const uint32_t code = ~(uint32_t)es.key[par] + (uint32_t)(r + 1) * unit;
+      es.key[e] = ((unsigned long long)score_key(sc) << 32) | (uint32_t)~code;
+    }
+    __syncthreads();
+    ls = le;
+    le += T;
+  }
+  // ---- 3. order: position of every entry among the enumerated set ----
+  const int total = le;
+  const int npop = total < B ? total : B;
+  if (total <= BUILD_THREADS) {
+    // rank by counting; g threads share one entry
+    int g = 32;
+    while (g > 1 && total * g > BUILD_THREADS) g >>= 1;
+    const int q = tid / g, part = tid - q * g;
+    int rank = 0;
+    if (q < total)
+      for (int j = part; j < total; j += g) rank += (j != q && e_before(j, q, es)) ? 1 : 0;
+    for (int o = g >> 1; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+    if (q < total && part == 0) es.pos[q] = (uint16_t)(rank < npop ? rank + 1 : 0);
+  } else {
+    int P = 1;
+    while (P < total) P <<= 1;
+    for (int i = tid; i < P; i += BUILD_THREADS) es.ord[i] = (uint16_t)(i < total ? i : 0xFFFFu);
+    __syncthreads();
+    for (int size = 2; size <= P; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int i = tid; i < P / 2; i += BUILD_THREADS) {
+          const int lo = 2 * stride * (i / stride) + (i % stride);
+          const int hi = lo + stride;
+          const bool up = (lo & size) == 0;       // this run sorts in pop order
+          const uint16_t a = es.ord[lo], b = es.ord[hi];
+          // b before a (pads last)
+          const bool b_first = b != 0xFFFFu && (a == 0xFFFFu || e_before(b, a, es));
+          if (b_first == up) { es.ord[lo] = b; es.ord[hi] = a; }
+        }
+        __syncthreads();
+      }
+    }
+    for (int i = tid; i < total; i += BUILD_THREADS) es.pos[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < npop; i += BUILD_THREADS) es.pos[es.ord[i]] = (uint16_t)(i + 1);
+  }
+  __syncthreads();
+  // ---- nodes 1..npop in pop order ----
+  for (int e = tid; e < total; e += BUILD_THREADS) {
+    const int node = es.pos[e];
+    if (node == 0) continue;
+    const uint32_t mt = es.meta[e];
+    const uint32_t pe = e_parent(mt);
+    sm.nd_parent[node] = pe == ENUM_ROOT ? 0 : (int)es.pos[pe];
+    sm.nd_rank[node] = e_rank(mt);
+    sm.nd_depth[node] = e_depth(mt);
+    sm.nd_score[node] = es.score[e];
+  }
+  return npop;
+}
+
 __global__ void __launch_bounds__(BUILD_THREADS, 1)
 build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
-             const int32_t* __restrict__ root_token, int L, int K, int B, int kc, TieCode tc,
+             const int32_t* __restrict__ root_token, int L, int K, int B, int kc, TieCode tc, int use_enum,
              int32_t* __restrict__ node_token, int32_t* __restrict__ parent,
              int32_t* __restrict__ depth, int32_t* __restrict__ node_rank,
              float* __restrict__ score, uint32_t* __restrict__ anc, int32_t* __restrict__ n_nodes) {
@@ -318,7 +557,22 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
     sm.nd_depth = (int*)p;  p += (size_t)n * 4;
     sm.nd_score = (float*)p;
   }
+  EnumSmem es;
+  {
+    unsigned char* p = smem_raw + ((build_smem_bytes(L, kc, B) + 15) & ~(size_t)15);
+    es.key = (unsigned long long*)p; p += (size_t)ENUM_CAP * 8;
+    es.score = (float*)p;            p += (size_t)ENUM_CAP * 4;
+    es.meta = (uint32_t*)p;          p += (size_t)ENUM_CAP * 4;
+    es.off = (int*)p;                p += (size_t)(ENUM_CAP + 1) * 4;
+    es.ord = (uint16_t*)p;           p += (size_t)ENUM_CAP * 2;
+    es.pos = (uint16_t*)p;
+  }
   __shared__ int s_pops;
+  __shared__ uint32_t s_hist[256];
+  __shared__ int s_bcast[4];
+  __shared__ int s_warp_tot[BUILD_THREADS / 32];
+  __shared__ float s_chain[64];
+  __shared__ int s_lev[3];
 
   // stage the lp table (only ranks < kc can ever be popped)
   const float* lpr = lp + (size_t)r * L * K;
@@ -328,14 +582,18 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
   }
   __syncthreads();
 
-  if (tid < 32) {
+  if (tid == 0) {
+    sm.nd_parent[0] = -1;
+    sm.nd_rank[0] = -1;
+    sm.nd_depth[0] = 0;
+    sm.nd_score[0] = 0.f;
+  }
+  int epops = -1;
+  if (use_enum && B > 0) epops = enum_build(sm, es, L, B, kc, tc, s_hist, s_bcast, s_warp_tot, s_chain, s_lev);
+  if (epops >= 0) {
+    if (tid == 0) s_pops = epops;
+  } else if (tid < 32) {
     const int lane = tid;
-    if (lane == 0) {
-      sm.nd_parent[0] = -1;
-      sm.nd_rank[0] = -1;
-      sm.nd_depth[0] = 0;
-      sm.nd_score[0] = 0.f;
-    }
     int pops;
     if (n <= 32 * 3) pops = heap_registers<3>(sm, L, B, kc, tc, lane);
     else if (n <= 32 * 9) pops = heap_registers<9>(sm, L, B, kc, tc, lane);

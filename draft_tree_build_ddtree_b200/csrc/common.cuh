@@ -90,4 +90,78 @@ __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v)
 
 inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
+// ---------------------------------------------------------------------------
+// Block-wide radix selection of the need-th largest key.
+//
+// Keys are `nbits` wide; `each(f)` calls f(key) for every key the thread
+// holds (0 = empty).  Returns t, `above` (keys above t's final prefix) and
+// `eq` (keys sharing the final prefix).  Either eq equals the remaining need
+// (early exit: every key >= t is selected, t has zero low bits) or t is the
+// exact value of the need-th key and the eq keys equal to it tie.
+// ---------------------------------------------------------------------------
+template <typename KeyT>
+struct RadixOut {
+  KeyT t;
+  int above;
+  int eq;
+};
+
+template <typename KeyT, typename Each>
+__device__ __forceinline__ RadixOut<KeyT> radix_kth(Each each, int nbits, int need, uint32_t* hist,
+                                                    int* bcast) {
+  const int tid = threadIdx.x;
+  KeyT prefix = 0;
+  int shift = nbits, above = 0, eq = 0;
+  while (shift > 0) {
+    const int width = shift < 8 ? shift : 8;
+    shift -= width;
+    const uint32_t dmask = (1u << width) - 1u;
+    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const int hi = shift + width;
+    const bool top = hi >= (int)(8 * sizeof(KeyT));
+    const KeyT want = top ? (KeyT)0 : (prefix >> hi);
+    each([&](KeyT k) {
+      if (k != 0 && (top || (k >> hi) == want)) atomicAdd(&hist[(uint32_t)(k >> shift) & dmask], 1u);
+    });
+    __syncthreads();
+    if (tid < 32) {
+      uint32_t c[8];
+      uint32_t mine = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { c[j] = hist[8 * tid + j]; mine += c[j]; }
+      uint32_t incl = mine;   // keys in digits >= 8*lane
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xffffffffu, incl, o);
+        if (tid + o < 32) incl += v;
+      }
+      const uint32_t above_lane = incl - mine;
+      const unsigned m = __ballot_sync(0xffffffffu, above_lane < (uint32_t)need && (uint32_t)need <= incl);
+      if (tid == __ffs(m) - 1) {
+        uint32_t ab = above_lane, cd = c[0];
+        int d = 0;
+#pragma unroll
+        for (int j = 7; j >= 0; --j) {
+          if (ab + c[j] >= (uint32_t)need) { d = j; cd = c[j]; break; }
+          ab += c[j];
+        }
+        bcast[0] = 8 * tid + d;
+        bcast[1] = (int)ab;
+        bcast[2] = (int)cd;
+      }
+    }
+    __syncthreads();
+    const int digit = bcast[0], ab = bcast[1], cnt = bcast[2];
+    __syncthreads();
+    prefix |= ((KeyT)digit) << shift;
+    need -= ab;
+    above += ab;
+    eq = cnt;
+    if (cnt == need) break;
+  }
+  return RadixOut<KeyT>{prefix, above, eq};
+}
+
+
 }  // namespace ddt

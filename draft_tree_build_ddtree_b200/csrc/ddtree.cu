@@ -142,11 +142,16 @@ int build_launch(const int32_t* ids, const float* lp, const int32_t* root_token,
   if (n_req < 1 || n_req > MAX_REQ || L < 1 || L > MAX_L || K < 1 || K > MAX_K || B < 0 || B > MAX_B)
     return DDTREE_ERR_INVALID_ARG;
   const int kc = B < K ? B : K;
-  const size_t smem = build_smem_bytes(L, kc, B);
+  // the threshold enumeration when its arrays fit beside the heap's
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, build_kernel) != cudaSuccess) return DDTREE_ERR_CUDA;
+  const size_t smem_enum = build_smem_bytes_enum(L, kc, B);
+  const int use_enum = smem_enum + attr.sharedSizeBytes <= (size_t)max_smem_optin() ? 1 : 0;
+  const size_t smem = use_enum ? smem_enum : build_smem_bytes(L, kc, B);
   int st = set_smem(build_kernel, smem);
   if (st) return st;
-  build_kernel<<<n_req, BUILD_THREADS, smem, s>>>(ids, lp, root_token, L, K, B, kc, tie_code(kc, L), node_token,
-                                                   parent, depth, node_rank, score, anc, n_nodes);
+  build_kernel<<<n_req, BUILD_THREADS, smem, s>>>(ids, lp, root_token, L, K, B, kc, tie_code(kc, L), use_enum,
+                                                   node_token, parent, depth, node_rank, score, anc, n_nodes);
   return launch_status();
 }
 

@@ -106,39 +106,46 @@ struct RadixOut {
   int eq;
 };
 
-template <typename KeyT, typename Each>
-__device__ __forceinline__ RadixOut<KeyT> radix_kth(Each each, int nbits, int need, uint32_t* hist,
-                                                    int* bcast) {
-  const int tid = threadIdx.x;
+// Group form: the `gsize` threads with group-local ids `gtid` (its first 32
+// form one warp) call it together and `sync()` is their barrier.
+template <typename KeyT, typename Each, typename Sync>
+__device__ __forceinline__ RadixOut<KeyT> radix_kth_g(Each each, int nbits, int need, uint32_t* hist, int* bcast,
+                                                      int gtid, int gsize, Sync sync) {
   KeyT prefix = 0;
   int shift = nbits, above = 0, eq = 0;
   while (shift > 0) {
     const int width = shift < 8 ? shift : 8;
     shift -= width;
     const uint32_t dmask = (1u << width) - 1u;
-    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
+    for (int i = gtid; i < 256; i += gsize) hist[i] = 0;
+    sync();
     const int hi = shift + width;
     const bool top = hi >= (int)(8 * sizeof(KeyT));
     const KeyT want = top ? (KeyT)0 : (prefix >> hi);
     each([&](KeyT k) {
       if (k != 0 && (top || (k >> hi) == want)) atomicAdd(&hist[(uint32_t)(k >> shift) & dmask], 1u);
     });
-    __syncthreads();
-    if (tid < 32) {
+    sync();
+    if (gtid < 32) {
       uint32_t c[8];
       uint32_t mine = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) { c[j] = hist[8 * tid + j]; mine += c[j]; }
+      for (int j = 0; j < 8; ++j) { c[j] = hist[8 * gtid + j]; mine += c[j]; }
       uint32_t incl = mine;   // keys in digits >= 8*lane
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const uint32_t v = __shfl_down_sync(0xffffffffu, incl, o);
-        if (tid + o < 32) incl += v;
+        if (gtid + o < 32) incl += v;
       }
       const uint32_t above_lane = incl - mine;
       const unsigned m = __ballot_sync(0xffffffffu, above_lane < (uint32_t)need && (uint32_t)need <= incl);
-      if (tid == __ffs(m) - 1) {
+      if (m == 0 && gtid == 0) {          // fewer keys than need: all of them
+        bcast[0] = 0;
+        bcast[1] = (int)incl;
+        bcast[2] = 0;
+        bcast[3] = 0;
+      }
+      if (gtid == __ffs(m) - 1) {
         uint32_t ab = above_lane, cd = c[0];
         int d = 0;
 #pragma unroll
@@ -146,14 +153,16 @@ __device__ __forceinline__ RadixOut<KeyT> radix_kth(Each each, int nbits, int ne
           if (ab + c[j] >= (uint32_t)need) { d = j; cd = c[j]; break; }
           ab += c[j];
         }
-        bcast[0] = 8 * tid + d;
+        bcast[0] = 8 * gtid + d;
         bcast[1] = (int)ab;
         bcast[2] = (int)cd;
+        bcast[3] = 1;
       }
     }
-    __syncthreads();
-    const int digit = bcast[0], ab = bcast[1], cnt = bcast[2];
-    __syncthreads();
+    sync();
+    const int digit = bcast[0], ab = bcast[1], cnt = bcast[2], ok = bcast[3];
+    sync();
+    if (!ok) return RadixOut<KeyT>{(KeyT)0, above + ab, 0};
     prefix |= ((KeyT)digit) << shift;
     need -= ab;
     above += ab;
@@ -161,6 +170,17 @@ __device__ __forceinline__ RadixOut<KeyT> radix_kth(Each each, int nbits, int ne
     if (cnt == need) break;
   }
   return RadixOut<KeyT>{prefix, above, eq};
+}
+
+template <typename KeyT, typename Each>
+__device__ __forceinline__ RadixOut<KeyT> radix_kth(Each each, int nbits, int need, uint32_t* hist, int* bcast) {
+  return radix_kth_g<KeyT>(each, nbits, need, hist, bcast, (int)threadIdx.x, (int)blockDim.x,
+                           [] { __syncthreads(); });
+}
+
+// Barrier over `nthreads` threads (whole warps) on hardware barrier `id` (1..15).
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 

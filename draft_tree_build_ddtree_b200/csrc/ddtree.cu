@@ -247,22 +247,20 @@ struct AcceptPlan {
   int cpr, chunk;
 };
 
-AcceptPlan accept_plan(int rows, int V, int esize) {
-  const int epv = 16 / esize;
-  const int max_chunk = ARGMAX_THREADS * TOPK_MAX_VPT * epv;
-  int cpr_min = ceil_div(V, max_chunk);
-  int cpr_fill = num_sms() * 2 / (rows > 0 ? rows : 1);
-  int cpr_small = ceil_div(V, 4096);
-  int cpr = cpr_fill < cpr_small ? cpr_fill : cpr_small;
-  if (cpr < cpr_min) cpr = cpr_min;
+// Chunks per row: about one wave of resident CTAs over all rows.
+AcceptPlan accept_plan(int rows, int V) {
+  const int resident = num_sms() * ARGMAX_CTAS_PER_SM;
+  int cpr = resident / (rows > 0 ? rows : 1);
+  const int cpr_small = ceil_div(V, 4096);
+  if (cpr > cpr_small) cpr = cpr_small;
   if (cpr < 1) cpr = 1;
   AcceptPlan p;
-  p.chunk = ceil_div(ceil_div(V, cpr), epv) * epv;
+  p.chunk = ceil_div(ceil_div(V, cpr), 8) * 8;
   p.cpr = ceil_div(V, p.chunk);
   return p;
 }
 
-size_t accept_ws(int n_req, int B) { return argmax_ws_bytes(n_req * (B + 1)); }
+size_t accept_ws(int n_req, int B) { return argmax_ws_bytes(n_req * (B + 1), n_req); }
 
 int accept_launch(const void* target_logits, int dtype, int V, long long row_stride, const int32_t* node_token,
                   const int32_t* parent, const int32_t* n_nodes, int n_req, int L, int B,
@@ -280,7 +278,7 @@ int accept_launch(const void* target_logits, int dtype, int V, long long row_str
     return DDTREE_ERR_INVALID_ARG;
   const int n = B + 1;
   const int rows = n_req * n;
-  if (!ws || !aligned16(ws) || ws_bytes < argmax_ws_bytes(rows)) return DDTREE_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws) || ws_bytes < argmax_ws_bytes(rows, n_req)) return DDTREE_ERR_INVALID_ARG;
   int row_bytes = 0;
   if (k_cache) {
     int st = kv_check(kv);
@@ -290,30 +288,10 @@ int accept_launch(const void* target_logits, int dtype, int V, long long row_str
     row_bytes = kv->Hkv * kv->D * esize_of(dtype);
     if (row_bytes % 16 != 0) return DDTREE_ERR_UNSUPPORTED;
   }
-  AcceptPlan p = accept_plan(rows, V, esize_of(dtype));
+  AcceptPlan p = accept_plan(rows, V);
   ArgmaxWs w = argmax_ws_carve(ws, rows);
   const long long grid = (long long)rows * p.cpr;
   if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
-  const int vpt = ceil_div(ceil_div(p.chunk, 16 / esize_of(dtype)), ARGMAX_THREADS);
-  switch (vpt) {
-#define DDT_ARGMAX_CASE(VP)                                                                               \
-  case VP:                                                                                                \
-    if (dtype == DDTREE_BF16)                                                                             \
-      argmax_kernel<DDTREE_BF16, VP><<<(unsigned)grid, ARGMAX_THREADS, 0, s>>>(target_logits, n, V,      \
-                                                                              row_stride, n_nodes, p.cpr, \
-                                                                              p.chunk, w);                \
-    else                                                                                                  \
-      argmax_kernel<DDTREE_F32, VP><<<(unsigned)grid, ARGMAX_THREADS, 0, s>>>(target_logits, n, V,       \
-                                                                             row_stride, n_nodes, p.cpr,  \
-                                                                             p.chunk, w);                 \
-    break;
-    DDT_ARGMAX_CASE(1) DDT_ARGMAX_CASE(2) DDT_ARGMAX_CASE(3) DDT_ARGMAX_CASE(4) DDT_ARGMAX_CASE(5)
-    DDT_ARGMAX_CASE(6)
-#undef DDT_ARGMAX_CASE
-    default: return DDTREE_ERR_UNSUPPORTED;
-  }
-  int st = launch_status();
-  if (st) return st;
   WalkArgs a;
   a.node_token = node_token;
   a.parent = parent;
@@ -339,6 +317,16 @@ int accept_launch(const void* target_logits, int dtype, int V, long long row_str
   a.num_blocks = k_cache ? kv->num_blocks : 0;
   a.max_blocks = k_cache ? kv->max_blocks : 0;
   a.row_bytes = row_bytes;
+  // few layers: the CTA that publishes a request's last argmax walks and compacts it
+  const int fuse = (!k_cache || kv->layers <= WALK_FUSE_MAX_LAYERS) ? 1 : 0;
+  if (dtype == DDTREE_BF16)
+    argmax_kernel<DDTREE_BF16><<<(unsigned)grid, ARGMAX_THREADS, 0, s>>>(target_logits, n, V, row_stride, n_nodes,
+                                                                        p.cpr, p.chunk, w, a, fuse);
+  else
+    argmax_kernel<DDTREE_F32><<<(unsigned)grid, ARGMAX_THREADS, 0, s>>>(target_logits, n, V, row_stride, n_nodes,
+                                                                       p.cpr, p.chunk, w, a, fuse);
+  int st = launch_status();
+  if (st || fuse) return st;
   const size_t smem = (size_t)n * 8;
   dim3 grid2(n_req, a.layers * 2);
   walk_compact_kernel<<<grid2, WALK_THREADS, smem, s>>>(a);

@@ -42,6 +42,8 @@ constexpr int TOPK_THREADS = 512;
 constexpr int TOPK_MAX_VPT = 6;            // 16-byte vectors per thread
 constexpr int TOPK_MAX_CAND = 16384;       // merge capacity (candidates per row)
 constexpr int TOPK_MAX_CPR = 128;          // chunks per row
+constexpr int TOPK_EXP_WARPS = 8;          // warps of a CTA that sum exp while the others select
+constexpr int TOPK_LIST_CAP = 4096;        // bf16 candidate list entries per chunk
 constexpr int TOPK_MERGE_SMALL = 512;      // merge ranks by counting up to this many keys >= the K-th value
 constexpr int TOPK_ID_BITS = 20;           // V <= 2^20
 constexpr uint32_t TOPK_ID_MASK = (1u << TOPK_ID_BITS) - 1u;
@@ -54,6 +56,7 @@ struct TopkPlan {
   int vpt;      // 16-byte vectors per thread
   int cap;      // candidate slots per chunk
   int cand;     // candidate slots per row = cpr * cap
+  int esize;    // bytes per logit
 };
 
 inline int topk_cap(int K) { return K + (K < 512 ? K : 512); }
@@ -76,8 +79,15 @@ inline TopkPlan topk_plan(int rows, int V, int K, int esize, int num_sms) {
   p.cpr = ceil_div(V, p.chunk);
   p.vpt = ceil_div(ceil_div(p.chunk, epv), TOPK_THREADS);
   p.cand = p.cpr * p.cap;
+  p.esize = esize;
   if (p.cpr > cpr_cap || p.vpt > TOPK_MAX_VPT) p.cpr = 0;   // unsupported shape
   return p;
+}
+
+// Shared memory of a staged chunk (whole 16-byte vectors), 16-byte aligned.
+__host__ __device__ inline size_t topk_stage_bytes(const TopkPlan& p) {
+  const size_t v = ((size_t)p.chunk * p.esize + 15) / 16 + 1;
+  return v * 16;
 }
 
 // Workspace of the top-K stage: tickets, chunk statistics, candidate counts
@@ -112,13 +122,17 @@ inline TopkWs topk_ws_carve(void* ws, int rows, const TopkPlan& p) {
   return w;
 }
 
-// exp(x) in fp64 (table-driven; relative error ~1e-16): 0 below -708,
-// +inf above 709.
+// exp(x) in fp64 for x <= 0 (table-driven; relative error ~1e-16).  x is
+// clamped at -700, where exp is ~1e-304 and the result stays normal.  The
+// reduction k = round(x * 64/ln2) rounds with the 1.5*2^52 shifter (k lands in
+// the low word), r = x - k*ln2/64 in two exact-product steps, then
+// 2^(k/64) * exp(r) = 2^(k>>6) * T[k&63] * (1 + p(r)).
 __device__ __forceinline__ double exp64(double x, const double* tab) {
-  if (!(x > -708.0)) return 0.0;
-  if (x > 709.0) return INFINITY;
-  const double kd = rint(x * EXP64_INV_LN2_64);
-  const int k = (int)kd;
+  x = fmax(x, -700.0);
+  const double shifter = 0x1.8p52;
+  const double t = fma(x, EXP64_INV_LN2_64, shifter);
+  const int k = __double2loint(t);
+  const double kd = t - shifter;
   double r = fma(-kd, EXP64_C1, x);
   r = fma(-kd, EXP64_C2, r);
   double p = fma(r, 1.0 / 120.0, 1.0 / 24.0);
@@ -160,23 +174,28 @@ __device__ __forceinline__ float key_value(uint32_t key) {
 }
 
 template <int DT, int VPT>
-__global__ void __launch_bounds__(TOPK_THREADS)
+__global__ void __launch_bounds__(TOPK_THREADS, 1)
 topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stride, int K, TopkPlan plan,
             TopkWs ws, int32_t* __restrict__ out_ids, float* __restrict__ out_lp, float* __restrict__ out_lse) {
   typedef TopkTraits<DT> T;
   constexpr int EPV = T::EPV;
+  constexpr int NW = TOPK_THREADS / 32;
+  constexpr int NWE = TOPK_EXP_WARPS;                 // warps 0..NWE-1: exp-sum; the rest: selection
+  constexpr int SEL_THREADS = TOPK_THREADS - 32 * NWE;
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ uint32_t hist[256];
   __shared__ int bcast[4];
-  __shared__ uint32_t red_u[TOPK_THREADS / 32];
-  __shared__ uint32_t red_w[TOPK_THREADS / 32];
-  __shared__ double red_d[TOPK_THREADS / 32];
+  __shared__ uint32_t red_u[NW];
+  __shared__ uint32_t red_w[NW];
+  __shared__ double red_d[NWE];
   __shared__ double s_tab[64];
   __shared__ int s_count;
+  __shared__ int s_ncl;
   __shared__ int s_last;
 
   const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.x / plan.cpr;
   const int c = blockIdx.x - row * plan.cpr;
   const long long c0 = (long long)c * plan.chunk;
@@ -184,13 +203,39 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   const int kloc = K < len ? K : len;
   if (tid < 64) s_tab[tid] = EXP64_TABLE[tid];
   for (int i = tid; i < 256; i += TOPK_THREADS) hist[i] = 0;
+  if (tid == 0) { s_count = 0; s_ncl = 0; }
 
-  // ---- streaming load: every vector of this thread in flight at once, then staged in shared memory ----
+  // ---- streaming load: every vector of this thread in flight at once; the
+  //      thread maximum is taken from the registers, then the chunk is staged ----
   const unsigned char* base = (const unsigned char*)logits + ((long long)row * row_stride + c0) * (16 / EPV);
   const int nvec_full = len / EPV;
   const int tail = len - nvec_full * EPV;          // ragged end (V not a multiple of the vector width)
   const int nvec = nvec_full + (tail > 0 ? 1 : 0);
   uint4* chunk_s = reinterpret_cast<uint4*>(smem_raw);
+  // candidate list of the selection warps (bf16): value key << 16 | chunk-local index
+  uint32_t* clist = reinterpret_cast<uint32_t*>(smem_raw + topk_stage_bytes(plan));
+  // bf16: fp32 max of the widened halves (fmaxf skips NaN, the magnitude maxima
+  // detect it); fp32: max of the order keys.  tkey: the thread maximum's key.
+  float mx = -INFINITY;
+  uint32_t tkey = 0, mag = 0;
+  bool nan_seen = false;
+  auto take_vec = [&](const uint4& v, int valid) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t w = u32_at(v, q);
+      if (DT == DDTREE_BF16) {
+        const float lo = 2 * q < valid ? __uint_as_float(w << 16) : -INFINITY;
+        const float hi = 2 * q + 1 < valid ? __uint_as_float(w & 0xFFFF0000u) : -INFINITY;
+        mx = fmaxf(mx, fmaxf(lo, hi));
+        if (2 * q < valid) mag = max(mag, w & 0x7FFFu);
+        if (2 * q + 1 < valid) mag = max(mag, (w >> 16) & 0x7FFFu);
+      } else if (q < valid) {
+        const float f = __uint_as_float(w);
+        nan_seen |= f != f;
+        tkey = max(tkey, key32_of_f32(f));
+      }
+    }
+  };
   {
     uint4 vec[VPT];
 #pragma unroll
@@ -201,18 +246,33 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
 #pragma unroll
     for (int v = 0; v < VPT; ++v) {
       const int vi = v * TOPK_THREADS + tid;
-      if (vi < nvec_full) chunk_s[vi] = vec[v];
+      if (vi < nvec_full) {
+        take_vec(vec[v], EPV);
+        chunk_s[vi] = vec[v];
+      }
     }
   }
   if (tail > 0 && tid == 0) {
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    uint4 tv = make_uint4(0u, 0u, 0u, 0u);
     for (int j = 0; j < tail; ++j) {
-      if (DT == DDTREE_BF16) w[j >> 1] |= (uint32_t)((const uint16_t*)(base + (size_t)nvec_full * 16))[j] << (16 * (j & 1));
-      else w[j] = ((const uint32_t*)(base + (size_t)nvec_full * 16))[j];
+      uint32_t x;
+      int q;
+      if (DT == DDTREE_BF16) {
+        x = (uint32_t)((const uint16_t*)(base + (size_t)nvec_full * 16))[j] << (16 * (j & 1));
+        q = j >> 1;
+      } else {
+        x = ((const uint32_t*)(base + (size_t)nvec_full * 16))[j];
+        q = j;
+      }
+      if (q == 0) tv.x |= x; else if (q == 1) tv.y |= x; else if (q == 2) tv.z |= x; else tv.w |= x;
     }
-    chunk_s[nvec_full] = make_uint4(w[0], w[1], w[2], w[3]);
+    take_vec(tv, tail);
+    chunk_s[nvec_full] = tv;
   }
-  __syncthreads();
+  if (DT == DDTREE_BF16) {
+    nan_seen = mag > 0x7F80u;
+    tkey = mx > -INFINITY ? key32_of_f32(mx) >> 16 : 0u;
+  }
 
   // Element e of vector vi is logit c0 + vi*EPV + e; its order key is 0 past the chunk end.
   // bf16 keys are computed two at a time with 16-bit SIMD integer ops.
@@ -232,248 +292,197 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
     }
   };
 
-  // ---- NaN check and chunk maximum ----
-  uint32_t kmax = 0;
-  bool nan_seen = false;
+  // ---- chunk maximum; bf16: lower bound of the K'-th largest logit ----
+  if (__any_sync(0xffffffffu, nan_seen) && lane == 0) flag_status(DDTREE_STATUS_NONFINITE);
   if (DT == DDTREE_BF16) {
-    // bf16 widens to fp32 with a shift: the maximum is an fp32 max (fmaxf
-    // skips NaN; the magnitude maxima detect it); past-the-end elements of
-    // the ragged vector count as -inf
-    float mx = -INFINITY;
-    uint32_t mag_lo = 0, mag_hi = 0;
-    for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
-      const uint4 v = chunk_s[vi];
-      const int valid = len - vi * EPV;
+    // The thread maxima are distinct elements, so if every warp contributes
+    // its r-th largest thread maximum (r = ceil(K'/warps)), at least K'
+    // logits are >= the smallest of those.  Only logits above that bound
+    // enter the window histogram and the candidate list.
+    const int r = (kloc + NW - 1) / NW;
+    uint32_t wk = 0;
+    if (r <= 32) {
+      uint32_t x = tkey;                        // 0: none
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t w = u32_at(v, q);
-        const float lo = 2 * q < valid ? __uint_as_float(w << 16) : -INFINITY;
-        const float hi = 2 * q + 1 < valid ? __uint_as_float(w & 0xFFFF0000u) : -INFINITY;
-        mx = fmaxf(mx, fmaxf(lo, hi));
-        mag_lo = max(mag_lo, w & 0x7FFFu);
-        mag_hi = max(mag_hi, w & 0x7FFF0000u);
-      }
-    }
-    nan_seen = mag_lo > 0x7F80u || mag_hi > 0x7F800000u;
-    // the order key of the maximum (any element equal to it has this key)
-    kmax = mx > -INFINITY ? key32_of_f32(mx) >> 16 : 0u;
-    // Lower bound of the chunk's K'-th largest logit: the thread maxima are
-    // distinct elements, so if every warp contributes its r-th largest thread
-    // maximum (r = ceil(K'/warps)), at least K' logits are >= the smallest of
-    // those.  Only logits above the bound enter the window histogram.
-    {
-      constexpr int NW = TOPK_THREADS / 32;
-      const int r = (kloc + NW - 1) / NW;
-      uint32_t wk = 0;
-      if (r <= 32) {
-        uint32_t x = kmax;                      // this thread's maximum (0: none)
-        const int lane = tid & 31;
+      for (int k = 2; k <= 32; k <<= 1) {       // bitonic sort across the warp, descending
 #pragma unroll
-        for (int k = 2; k <= 32; k <<= 1) {     // bitonic sort across the warp, descending
-#pragma unroll
-          for (int j = k >> 1; j > 0; j >>= 1) {
-            const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
-            const bool lower = (lane & j) == 0;
-            const bool desc = (lane & k) == 0 || k == 32;
-            x = (lower == desc) ? max(x, y) : min(x, y);
-          }
+        for (int j = k >> 1; j > 0; j >>= 1) {
+          const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
+          const bool lower = (lane & j) == 0;
+          const bool desc = (lane & k) == 0 || k == 32;
+          x = (lower == desc) ? max(x, y) : min(x, y);
         }
-        wk = __shfl_sync(0xffffffffu, x, r - 1);
       }
-      if ((tid & 31) == 0) red_w[tid >> 5] = wk;
+      wk = __shfl_sync(0xffffffffu, x, r - 1);
     }
-    if (mx == -INFINITY) {                      // only -inf (or nothing) here: key of -inf if present
-      for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
-        uint32_t k[EPV];
-        keys_of(vi, k);
-#pragma unroll
-        for (int j = 0; j < EPV; ++j) kmax = k[j] > kmax ? k[j] : kmax;
-      }
-    }
-  } else {
-    for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
-      uint32_t k[EPV];
-      keys_of(vi, k);
-      const uint4 v = chunk_s[vi];
-#pragma unroll
-      for (int j = 0; j < EPV; ++j) {
-        const float f = __uint_as_float(u32_at(v, j));
-        nan_seen |= f != f;
-        kmax = k[j] > kmax ? k[j] : kmax;
-      }
-    }
+    if (lane == 0) red_w[warp] = wk;
   }
-  if (__any_sync(0xffffffffu, nan_seen) && (tid & 31) == 0) flag_status(DDTREE_STATUS_NONFINITE);
-  kmax = __reduce_max_sync(0xffffffffu, kmax);
-  if ((tid & 31) == 0) red_u[tid >> 5] = kmax;
+  uint32_t kmax = __reduce_max_sync(0xffffffffu, tkey);
+  if (lane == 0) red_u[warp] = kmax;
   __syncthreads();
   kmax = red_u[0];
 #pragma unroll
-  for (int i = 1; i < TOPK_THREADS / 32; ++i) kmax = red_u[i] > kmax ? red_u[i] : kmax;
+  for (int i = 1; i < NW; ++i) kmax = red_u[i] > kmax ? red_u[i] : kmax;
   const float m = key_value<DT>(kmax);
   const double md = (double)m;
-
-  // ---- fp64 sum of exp(z - m); bf16: max-anchored window histogram ----
-  double s0 = 0.0, s1 = 0.0;
   const bool m_finite = m > -INFINITY;
-  if (DT == DDTREE_BF16) {
-    // values below the window's lowest bin, or below the K'-th value's lower
-    // bound, skip the histogram with one compare
-    uint32_t wbound = red_w[0];
+
+  uint32_t tval = 0;
+  int above = 0, eq = 0;
+  if (warp < NWE) {
+    // ================= exp warps: fp64 sum of exp(z - m) =================
+    double s0 = 0.0, s1 = 0.0;
+    if (m_finite) {
+      for (int vi = tid; vi < nvec; vi += 32 * NWE) {
+        const uint4 v = chunk_s[vi];
+        const int valid = len - vi * EPV;
 #pragma unroll
-    for (int i = 1; i < TOPK_THREADS / 32; ++i) wbound = red_w[i] < wbound ? red_w[i] : wbound;
-    const uint32_t wkey = max(wbound, kmax >= 255u ? kmax - 255u : 0u);
-    const float wlow = wkey > 0u ? bf16_of_key16(wkey) : -INFINITY;
-    for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
-      const uint4 v = chunk_s[vi];
-      const int valid = len - vi * EPV;
-#pragma unroll
-      for (int j = 0; j < EPV; ++j) {
-        if (j < valid) {
-          const uint32_t bits = elem_bits<DT>(v, j);
-          const float z = bf16_bits_to_f32((uint16_t)bits);
-          const double e = m_finite ? exp64((double)z - md, s_tab) : 0.0;
-          if (j & 1) s1 += e; else s0 += e;
-          if (z >= wlow) {
-            const uint32_t d = kmax - key16_of_bf16((uint16_t)bits);
-            if (d < 256u) atomicAdd(&hist[d], 1u);
+        for (int j = 0; j < EPV; ++j) {
+          if (j < valid) {
+            const float z = DT == DDTREE_BF16 ? bf16_bits_to_f32((uint16_t)elem_bits<DT>(v, j))
+                                              : __uint_as_float(u32_at(v, j));
+            const double e = exp64((double)z - md, s_tab);
+            if (j & 1) s1 += e; else s0 += e;
           }
         }
       }
     }
+    double sum = s0 + s1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) red_d[warp] = sum;
   } else {
-    for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
-      uint32_t k[EPV];
-      keys_of(vi, k);
+    // ================= selection warps: threshold and emission =================
+    const int gtid = tid - 32 * NWE;
+    auto gsync = [] { named_sync(1, SEL_THREADS); };
+    bool found = false, use_list = false;
+    if (DT == DDTREE_BF16) {
+      // max-anchored window histogram (bin b: the value kmax - b) of the logits
+      // above the bound; the same logits enter the candidate list
+      uint32_t wbound = red_w[0];
 #pragma unroll
-      for (int j = 0; j < EPV; ++j) {
-        if (k[j] != 0) {
-          const double e = m_finite ? exp64((double)key_value<DT>(k[j]) - md, s_tab) : 0.0;
-          if (j & 1) s1 += e; else s0 += e;
+      for (int i = 1; i < NW; ++i) wbound = red_w[i] < wbound ? red_w[i] : wbound;
+      const uint32_t wkey = max(wbound, kmax >= 255u ? kmax - 255u : 0u);
+      const float wlow = wkey > 0u ? bf16_of_key16(wkey) : -INFINITY;
+      for (int vi = gtid; vi < nvec; vi += SEL_THREADS) {
+        const uint4 v = chunk_s[vi];
+        const int valid = len - vi * EPV;
+#pragma unroll
+        for (int j = 0; j < EPV; ++j) {
+          const uint32_t bits = elem_bits<DT>(v, j);
+          if (j < valid && bf16_bits_to_f32((uint16_t)bits) >= wlow) {
+            const uint32_t key = key16_of_bf16((uint16_t)bits);
+            const uint32_t d = kmax - key;
+            if (d < 256u) atomicAdd(&hist[d], 1u);
+            const int slot = atomicAdd(&s_ncl, 1);
+            if (slot < TOPK_LIST_CAP) clist[slot] = (key << 16) | (uint32_t)(vi * EPV + j);
+          }
         }
       }
-    }
-  }
-  double s = s0 + s1;
+      gsync();
+      if (gtid < 32) {
+        uint32_t cbin[8];
+        uint32_t mine = 0;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if ((tid & 31) == 0) red_d[tid >> 5] = s;
-  __syncthreads();
+        for (int j = 0; j < 8; ++j) { cbin[j] = hist[8 * gtid + j]; mine += cbin[j]; }
+        uint32_t incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (gtid >= o) incl += v;
+        }
+        const uint32_t before = incl - mine;
+        const unsigned msk = __ballot_sync(0xffffffffu, before < (uint32_t)kloc && (uint32_t)kloc <= incl);
+        if (gtid == 0) bcast[3] = msk ? 1 : 0;
+        if (msk && gtid == __ffs(msk) - 1) {
+          uint32_t acc = before, cb = cbin[0];
+          int j0 = 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (acc + cbin[j] >= (uint32_t)kloc) { j0 = j; cb = cbin[j]; break; }
+            acc += cbin[j];
+          }
+          bcast[0] = 8 * gtid + j0;
+          bcast[1] = (int)acc;
+          bcast[2] = (int)cb;
+        }
+      }
+      gsync();
+      if (bcast[3]) {
+        found = true;
+        tval = kmax - (uint32_t)bcast[0];
+        above = bcast[1];
+        eq = bcast[2];
+      }
+      // every logit >= the threshold is in the list when it did not overflow
+      use_list = found && s_ncl <= TOPK_LIST_CAP;
+      gsync();
+    }
+    if (!found) {
+      auto each = [&](auto f) {
+        for (int vi = gtid; vi < nvec; vi += SEL_THREADS) {
+          uint32_t k[EPV];
+          keys_of(vi, k);
+#pragma unroll
+          for (int j = 0; j < EPV; ++j) f(k[j]);
+        }
+      };
+      const RadixOut<uint32_t> ro = radix_kth_g<uint32_t>(each, T::KEY_BITS, kloc, hist, bcast, gtid, SEL_THREADS, gsync);
+      tval = ro.t;
+      above = ro.above;
+      eq = ro.eq;
+    }
+    const int ncl = use_list ? s_ncl : 0;
 
-  // ---- threshold value of the chunk's K'-th largest logit ----
-  uint32_t tval = 0;
-  int above = 0, eq = 0;
-  bool found = false;
-  if (DT == DDTREE_BF16) {
-    if (tid < 32) {     // bin b holds the value kmax - b
-      uint32_t cbin[8];
-      uint32_t mine = 0;
+    // ---- emit candidates: every key >= tval, or cut the ties at tval by lowest id ----
+    const bool all_ties = above + eq <= plan.cap;
+    uint32_t lid_thr = 0;
+    if (!all_ties) {
+      auto each_lid = [&](auto f) {
+        if (use_list) {
+          for (int i = gtid; i < ncl; i += SEL_THREADS) {
+            const uint32_t e = clist[i];
+            f((e >> 16) == tval ? (LID_MASK - (e & 0xFFFFu)) : 0u);
+          }
+        } else {
+          for (int vi = gtid; vi < nvec; vi += SEL_THREADS) {
+            uint32_t k[EPV];
+            keys_of(vi, k);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) { cbin[j] = hist[8 * tid + j]; mine += cbin[j]; }
-      uint32_t incl = mine;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (tid >= o) incl += v;
-      }
-      const uint32_t before = incl - mine;
-      const unsigned msk = __ballot_sync(0xffffffffu, before < (uint32_t)kloc && (uint32_t)kloc <= incl);
-      if (tid == 0) bcast[3] = msk ? 1 : 0;
-      if (msk && tid == __ffs(msk) - 1) {
-        uint32_t acc = before, cb = cbin[0];
-        int j0 = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (acc + cbin[j] >= (uint32_t)kloc) { j0 = j; cb = cbin[j]; break; }
-          acc += cbin[j];
+            for (int j = 0; j < EPV; ++j) f(k[j] == tval ? (LID_MASK - (uint32_t)(vi * EPV + j)) : 0u);
+          }
         }
-        bcast[0] = 8 * tid + j0;
-        bcast[1] = (int)acc;
-        bcast[2] = (int)cb;
+      };
+      lid_thr = radix_kth_g<uint32_t>(each_lid, LID_BITS, kloc - above, hist, bcast, gtid, SEL_THREADS, gsync).t;
+    }
+    unsigned long long* cand = ws.cand + (size_t)row * plan.cand + (size_t)c * plan.cap;
+    auto emit = [&](uint32_t key, uint32_t lid) {
+      const bool take = key != 0 && (key > tval || (key == tval && (all_ties || (LID_MASK - lid) >= lid_thr)));
+      if (take) {
+        const int slot = atomicAdd(&s_count, 1);
+        const uint32_t gid = (uint32_t)(c0 + lid);
+        if (slot < plan.cap)
+          cand[slot] = ((unsigned long long)key << TOPK_ID_BITS) | (unsigned long long)(TOPK_ID_MASK - gid);
       }
-    }
-    __syncthreads();
-    if (bcast[3]) {
-      found = true;
-      tval = kmax - (uint32_t)bcast[0];
-      above = bcast[1];
-      eq = bcast[2];
-    }
-    __syncthreads();
-  }
-  if (!found) {
-    auto each = [&](auto f) {
-      for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
+    };
+    if (use_list) {
+      for (int i = gtid; i < ncl; i += SEL_THREADS) {
+        const uint32_t e = clist[i];
+        emit(e >> 16, e & 0xFFFFu);
+      }
+    } else {
+      for (int vi = gtid; vi < nvec; vi += SEL_THREADS) {
         uint32_t k[EPV];
         keys_of(vi, k);
 #pragma unroll
-        for (int j = 0; j < EPV; ++j) f(k[j]);
-      }
-    };
-    const RadixOut<uint32_t> ro = radix_kth<uint32_t>(each, T::KEY_BITS, kloc, hist, bcast);
-    tval = ro.t;
-    above = ro.above;
-    eq = ro.eq;
-  }
-
-  // ---- emit candidates: every key >= tval, or cut the ties at tval by lowest id ----
-  const bool all_ties = above + eq <= plan.cap;
-  uint32_t lid_thr = 0;
-  if (!all_ties) {
-    auto each_lid = [&](auto f) {
-      for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
-        uint32_t k[EPV];
-        keys_of(vi, k);
-#pragma unroll
-        for (int j = 0; j < EPV; ++j) f(k[j] == tval ? (LID_MASK - (uint32_t)(vi * EPV + j)) : 0u);
-      }
-    };
-    lid_thr = radix_kth<uint32_t>(each_lid, LID_BITS, kloc - above, hist, bcast).t;
-  }
-  if (tid == 0) s_count = 0;
-  __syncthreads();
-  unsigned long long* cand_row = ws.cand + (size_t)row * plan.cand;
-  unsigned long long* cand = cand_row + (size_t)c * plan.cap;
-  if (DT == DDTREE_BF16 && all_ties) {
-    // every logit >= the threshold value: one fp32 compare per logit (-0.0 == +0.0)
-    const float tf = bf16_of_key16(tval);
-    for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
-      const uint4 v = chunk_s[vi];
-      const int valid = len - vi * EPV;
-#pragma unroll
-      for (int j = 0; j < EPV; ++j) {
-        const uint32_t bits = elem_bits<DT>(v, j);
-        if (j < valid && bf16_bits_to_f32((uint16_t)bits) >= tf) {
-          const int slot = atomicAdd(&s_count, 1);
-          const uint32_t gid = (uint32_t)(c0 + vi * EPV + j);
-          if (slot < plan.cap)
-            cand[slot] = ((unsigned long long)key16_of_bf16((uint16_t)bits) << TOPK_ID_BITS) |
-                         (unsigned long long)(TOPK_ID_MASK - gid);
-        }
-      }
-    }
-  } else {
-    for (int vi = tid; vi < nvec; vi += TOPK_THREADS) {
-      uint32_t k[EPV];
-      keys_of(vi, k);
-#pragma unroll
-      for (int j = 0; j < EPV; ++j) {
-        const int lid = vi * EPV + j;
-        const bool take =
-            k[j] != 0 && (k[j] > tval || (k[j] == tval && (all_ties || (LID_MASK - (uint32_t)lid) >= lid_thr)));
-        if (take) {
-          const int slot = atomicAdd(&s_count, 1);
-          const uint32_t gid = (uint32_t)(c0 + lid);
-          if (slot < plan.cap)
-            cand[slot] = ((unsigned long long)k[j] << TOPK_ID_BITS) | (unsigned long long)(TOPK_ID_MASK - gid);
-        }
+        for (int j = 0; j < EPV; ++j) emit(k[j], (uint32_t)(vi * EPV + j));
       }
     }
   }
   __syncthreads();
   if (tid == 0) {
     double tot = 0.0;
-    for (int i = 0; i < TOPK_THREADS / 32; ++i) tot += red_d[i];
+    for (int i = 0; i < NWE; ++i) tot += red_d[i];
     ws.stats[(size_t)row * plan.cpr + c] = make_double2(md, tot);
     ws.count[(size_t)row * plan.cpr + c] = s_count < plan.cap ? s_count : plan.cap;
     ws.thr[(size_t)row * plan.cpr + c] = tval;
@@ -489,6 +498,7 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   __threadfence();
 
   // =================== merge (last CTA of this row; the staged chunk is dead) ===================
+  const unsigned long long* cand_row = ws.cand + (size_t)row * plan.cand;
   unsigned long long* sc = (unsigned long long*)smem_raw;   // [plan.cand]
   int kpow = 1;
   while (kpow < K) kpow <<= 1;
@@ -498,7 +508,6 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   __shared__ double s_lse;
   __shared__ uint32_t s_floor;
   __shared__ int s_m;
-  const int lane = tid & 31;
   // Every chunk emitted at least min(K, its length) logits at or above its
   // threshold value, so the row's K-th best value is at least the largest
   // chunk threshold: candidates below it cannot be selected.
@@ -645,7 +654,7 @@ inline size_t topk_smem_bytes(const TopkPlan& p, int K) {
   int kpow = 1;
   while (kpow < K) kpow <<= 1;
   const size_t merge = (size_t)(p.cand + (kpow > TOPK_MERGE_SMALL ? kpow : TOPK_MERGE_SMALL)) * 8;
-  const size_t chunk = (size_t)(p.chunk + 16) * 4;    // worst case fp32 elements, + one ragged vector
+  const size_t chunk = topk_stage_bytes(p) + (size_t)TOPK_LIST_CAP * 4;   // staged chunk + candidate list
   return merge > chunk ? merge : chunk;
 }
 

@@ -173,6 +173,19 @@ __device__ __forceinline__ float key_value(uint32_t key) {
   return DT == DDTREE_BF16 ? bf16_of_key16(key) : f32_of_key32(key);
 }
 
+// Warp-aggregated append of `key` to dst[*counter] where `take` holds; every
+// lane of the warp calls it.
+__device__ __forceinline__ void append_to(unsigned long long* dst, int* counter, bool take, unsigned long long key,
+                                          int lane) {
+  const unsigned bal = __ballot_sync(0xffffffffu, take);
+  if (bal) {
+    int base = 0;
+    if (lane == 0) base = atomicAdd(counter, __popc(bal));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (take) dst[base + __popc(bal & ((1u << lane) - 1u))] = key;
+  }
+}
+
 template <int DT, int VPT>
 __global__ void __launch_bounds__(TOPK_THREADS, 1)
 topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stride, int K, TopkPlan plan,
@@ -336,15 +349,18 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
       for (int vi = tid; vi < nvec; vi += 32 * NWE) {
         const uint4 v = chunk_s[vi];
         const int valid = len - vi * EPV;
+        // branch-free over the vector (the exps are independent chains); the
+        // past-the-end elements of the ragged vector are computed and dropped
+        double e[EPV];
 #pragma unroll
         for (int j = 0; j < EPV; ++j) {
-          if (j < valid) {
-            const float z = DT == DDTREE_BF16 ? bf16_bits_to_f32((uint16_t)elem_bits<DT>(v, j))
-                                              : __uint_as_float(u32_at(v, j));
-            const double e = exp64((double)z - md, s_tab);
-            if (j & 1) s1 += e; else s0 += e;
-          }
+          const float z = DT == DDTREE_BF16 ? bf16_bits_to_f32((uint16_t)elem_bits<DT>(v, j))
+                                            : __uint_as_float(u32_at(v, j));
+          e[j] = exp64((double)z - md, s_tab);
+          e[j] = j < valid ? e[j] : 0.0;
         }
+#pragma unroll
+        for (int j = 0; j < EPV; j += 2) { s0 += e[j]; s1 += e[j + 1]; }
       }
     }
     double sum = s0 + s1;
@@ -506,13 +522,20 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   __shared__ int s_cnt[TOPK_MAX_CPR];
   __shared__ double2 s_st[TOPK_MAX_CPR];
   __shared__ double s_lse;
-  __shared__ uint32_t s_floor;
   __shared__ int s_m;
+  // One round of loads: the chunks' counts, statistics and thresholds, and
+  // (speculatively, before the counts are known) the first candidate slots.
+  constexpr int UNR = 4;
+  const int slots = plan.cpr * plan.cap;
+  unsigned long long v[UNR];
+#pragma unroll
+  for (int u = 0; u < UNR; ++u) {
+    const int sl = tid + u * TOPK_THREADS;
+    v[u] = sl < slots ? __ldcg(cand_row + sl) : 0ull;
+  }
   // Every chunk emitted at least min(K, its length) logits at or above its
   // threshold value, so the row's K-th best value is at least the largest
   // chunk threshold: candidates below it cannot be selected.
-  if (tid == 0) { s_floor = 0; s_count = 0; s_m = 0; }
-  __syncthreads();
   uint32_t tmax = 0;
   for (int i = tid; i < plan.cpr; i += TOPK_THREADS) {
     s_cnt[i] = __ldcg(&ws.count[(size_t)row * plan.cpr + i]);
@@ -521,9 +544,43 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
     if (li >= K) tmax = max(tmax, __ldcg(&ws.thr[(size_t)row * plan.cpr + i]));
   }
   tmax = __reduce_max_sync(0xffffffffu, tmax);
-  if (lane == 0 && tmax) atomicMax(&s_floor, tmax);
+  if (lane == 0) red_u[warp] = tmax;
+  if (tid == 0) { s_count = 0; s_m = 0; }
   __syncthreads();
-  if (tid < 32) {   // lse from the chunk statistics, combined across the lanes of warp 0
+  uint32_t floor_v = red_u[0];
+#pragma unroll
+  for (int i = 1; i < NW; ++i) floor_v = red_u[i] > floor_v ? red_u[i] : floor_v;
+  const unsigned long long floor_key = (unsigned long long)floor_v << TOPK_ID_BITS;
+  // gather the candidates at or above the floor (one shared atomic per warp and round)
+  auto append = [&](bool take, unsigned long long key) {
+    const unsigned bal = __ballot_sync(0xffffffffu, take);
+    if (bal) {
+      int base = 0;
+      if (lane == 0) base = atomicAdd(&s_count, __popc(bal));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (take) sc[base + __popc(bal & ((1u << lane) - 1u))] = key;
+    }
+  };
+#pragma unroll
+  for (int u = 0; u < UNR; ++u) {
+    const int sl = tid + u * TOPK_THREADS;
+    const int ci = sl / plan.cap, j = sl - ci * plan.cap;
+    append(sl < slots && j < s_cnt[ci] && v[u] >= floor_key, v[u]);
+  }
+  for (int s0 = UNR * TOPK_THREADS + (tid & ~31); s0 < slots; s0 += UNR * TOPK_THREADS) {   // warp-uniform
+    unsigned long long w[UNR];
+    bool ok[UNR];
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const int sl = s0 + lane + u * TOPK_THREADS;
+      const int ci = sl / plan.cap, j = sl - ci * plan.cap;
+      ok[u] = sl < slots && j < s_cnt[ci];
+      w[u] = ok[u] ? __ldcg(cand_row + sl) : 0ull;
+    }
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) append(ok[u] && w[u] >= floor_key, w[u]);
+  }
+  if (warp == NW - 1) {   // lse from the chunk statistics, combined across the lanes of the last warp
     double M = -INFINITY;
     for (int i = lane; i < plan.cpr; i += 32) M = fmax(M, s_st[i].x);
 #pragma unroll
@@ -537,57 +594,80 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
     if (lane == 0) {
       s_lse = M + log(S);
       ws.ticket[row] = 0;   // leave the workspace ready for the next call
-    }
-  }
-  // gather the candidates at or above the floor (one shared atomic per warp and round)
-  const unsigned long long floor_key = (unsigned long long)s_floor << TOPK_ID_BITS;
-  {
-    constexpr int UNR = 4;   // issue several candidate loads before storing any
-    const int slots = plan.cpr * plan.cap;
-    for (int s0 = tid & ~31; s0 < slots; s0 += UNR * TOPK_THREADS) {   // warp-uniform trip count
-      unsigned long long v[UNR];
-      bool ok[UNR];
-#pragma unroll
-      for (int u = 0; u < UNR; ++u) {
-        const int sl = s0 + lane + u * TOPK_THREADS;
-        const int ci = sl / plan.cap, j = sl - ci * plan.cap;
-        ok[u] = sl < slots && j < s_cnt[ci];
-        v[u] = ok[u] ? __ldcg(cand_row + sl) : 0ull;
-      }
-#pragma unroll
-      for (int u = 0; u < UNR; ++u) {
-        const bool take = ok[u] && v[u] >= floor_key;
-        const unsigned bal = __ballot_sync(0xffffffffu, take);
-        if (bal) {
-          int base = 0;
-          if (lane == 0) base = atomicAdd(&s_count, __popc(bal));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          if (take) sc[base + __popc(bal & ((1u << lane) - 1u))] = v[u];
-        }
-      }
+      // order key of the row maximum (the largest chunk maximum)
+      bcast[3] = M > -INFINITY ? (int)value_key<DT>(DT == DDTREE_BF16 ? (uint32_t)(__float_as_uint((float)M) >> 16)
+                                                                     : __float_as_uint((float)M))
+                               : 0;
     }
   }
   __syncthreads();
   const int ncand = s_count;   // <= plan.cand: every chunk wrote at most cap slots
   const double lse = s_lse;
+  const uint32_t vkmax = (uint32_t)bcast[3];
   const int per = (ncand + TOPK_THREADS - 1) / TOPK_THREADS;
-  // the K-th largest value among the candidates: every key above it and the
-  // ties at it form the set that holds the row's top K
-  auto veach = [&](auto f) {
-    for (int i = 0; i < per; ++i) {
-      const int idx = i * TOPK_THREADS + tid;
-      f(idx < ncand ? (uint32_t)(sc[idx] >> TOPK_ID_BITS) : 0u);
+  // The K-th largest value among the candidates: every key above it and the
+  // ties at it form the set that holds the row's top K.  bf16: one
+  // max-anchored 256-bin histogram when the value lies within 256 steps of
+  // the row maximum, else a radix select.
+  RadixOut<uint32_t> vt{0u, 0, 0};
+  bool vfound = false;
+  if (DT == DDTREE_BF16) {
+    for (int i = tid; i < 256; i += TOPK_THREADS) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < ncand; i += TOPK_THREADS) {
+      const uint32_t d = vkmax - (uint32_t)(sc[i] >> TOPK_ID_BITS);
+      if (d < 256u) atomicAdd(&hist[d], 1u);
     }
-  };
-  const RadixOut<uint32_t> vt = radix_kth<uint32_t>(veach, T::KEY_BITS, K, hist, bcast);
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t cbin[8];
+      uint32_t mine = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { cbin[j] = hist[8 * lane + j]; mine += cbin[j]; }
+      uint32_t incl = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t before = incl - mine;
+      const unsigned msk = __ballot_sync(0xffffffffu, before < (uint32_t)K && (uint32_t)K <= incl);
+      if (lane == 0) bcast[3] = msk ? 1 : 0;
+      if (msk && lane == __ffs(msk) - 1) {
+        uint32_t acc = before, cb = cbin[0];
+        int j0 = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (acc + cbin[j] >= (uint32_t)K) { j0 = j; cb = cbin[j]; break; }
+          acc += cbin[j];
+        }
+        bcast[0] = 8 * lane + j0;
+        bcast[1] = (int)acc;
+        bcast[2] = (int)cb;
+      }
+    }
+    __syncthreads();
+    if (bcast[3]) {
+      vfound = true;
+      vt = RadixOut<uint32_t>{vkmax - (uint32_t)bcast[0], bcast[1], bcast[2]};
+    }
+    __syncthreads();
+  }
+  if (!vfound) {
+    auto veach = [&](auto f) {
+      for (int i = 0; i < per; ++i) {
+        const int idx = i * TOPK_THREADS + tid;
+        f(idx < ncand ? (uint32_t)(sc[idx] >> TOPK_ID_BITS) : 0u);
+      }
+    };
+    vt = radix_kth<uint32_t>(veach, T::KEY_BITS, K, hist, bcast);
+  }
   const int nsel = vt.above + vt.eq;
   if (nsel <= TOPK_MERGE_SMALL) {
-    for (int i = 0; i < per; ++i) {
-      const int idx = i * TOPK_THREADS + tid;
-      if (idx < ncand) {
-        const unsigned long long k = sc[idx];
-        if ((uint32_t)(k >> TOPK_ID_BITS) >= vt.t) win[atomicAdd(&s_m, 1)] = k;
-      }
+    for (int i0 = 0; i0 < ncand; i0 += TOPK_THREADS) {   // block-uniform trip count
+      const int idx = i0 + tid;
+      const unsigned long long k = idx < ncand ? sc[idx] : 0ull;
+      append_to(win, &s_m, idx < ncand && (uint32_t)(k >> TOPK_ID_BITS) >= vt.t, k, lane);
     }
     __syncthreads();
     // rank by counting (keys are unique): g threads share one key's count
@@ -598,7 +678,16 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
     int rank = 0;
     if (q < nsel) {
       k = win[q];
-      for (int j = part; j < nsel; j += g) rank += win[j] > k;
+      int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+      int j = part;
+      for (; j + 3 * g < nsel; j += 4 * g) {
+        r0 += win[j] > k;
+        r1 += win[j + g] > k;
+        r2 += win[j + 2 * g] > k;
+        r3 += win[j + 3 * g] > k;
+      }
+      for (; j < nsel; j += g) r0 += win[j] > k;
+      rank = (r0 + r1) + (r2 + r3);
     }
     for (int o = g >> 1; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
     if (q < nsel && part == 0 && rank < K) {

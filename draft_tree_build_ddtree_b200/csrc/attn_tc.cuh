@@ -536,7 +536,8 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
               (m_used + log2f(l)) * 0.6931471805599453f;
       } else {
         const size_t slot = (size_t)unit * p.splits + split;
-        float* wo = p.ws_o + (slot * TC_BM + row) * TC_D;
+        // [slot][D/4][128 rows] float4: a warp's 32 rows write 512 contiguous bytes per store
+        float4* wo = reinterpret_cast<float4*>(p.ws_o) + slot * (TC_D / 4) * TC_BM + row;
 #pragma unroll 1
         for (int c = 0; c < TC_D / 32; ++c) {
           float o[32];
@@ -544,7 +545,7 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(wo + c * 32 + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+            wo[(size_t)((c * 32 + e) / 4) * TC_BM] = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
         }
         p.ws_ml[slot * TC_BM + row] = make_float2(m_used, l);
       }
@@ -565,16 +566,16 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 }
 
 // Merge the key splits of every (unit, row): O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
-// One CTA per (unit, group of 8 rows); 16 threads share a row, each owning 8
-// consecutive dims, so every split's partial row is read with coalesced
-// 16-byte loads.
-constexpr int TC_COMBINE_ROWS = 8;
+// One CTA per (unit, 8 dims), one thread per M row: the partials are stored
+// row-innermost, so every load is a coalesced run over the rows; each thread
+// requests all splits' data before combining.
 constexpr int TC_MAX_SPLITS = 16;
 
+template <int S>   // capacity for the number of splits (>= p.splits)
 __global__ void __launch_bounds__(128)
 tree_attn_combine_kernel(const TcParams p) {
   const AttnGeom& g = p.g;
-  const int groups = TC_BM / TC_COMBINE_ROWS;
+  const int groups = TC_D / 8;
   int u = blockIdx.x / groups;
   const int rg = blockIdx.x - u * groups;
   const int unit = u;
@@ -588,34 +589,40 @@ tree_attn_combine_kernel(const TcParams p) {
   const int P = p.prefix_len[r];
   const long long cap = g.paged ? (long long)g.max_blocks * DDTREE_PAGE : (long long)g.s_max;
   if (P < 0 || (long long)P + nn > cap) return;
-  const int row = rg * TC_COMBINE_ROWS + (threadIdx.x >> 4);
-  const int d0 = (threadIdx.x & 15) * 8;
+  const int row = threadIdx.x;                   // one M row per thread, 8 dims per CTA
+  const int d0 = rg * 8;
   const int node = node0 + row / p.G;
   if (node >= nn) return;
   const int hq = kvh * p.G + row % p.G;
-  float2 ml[TC_MAX_SPLITS];
-  float M = -INFINITY;
+  // every split's statistics and partial row are requested before any is used
+  float2 ml[S];
+  float4 pa[S], pb[S];
 #pragma unroll
-  for (int s = 0; s < TC_MAX_SPLITS; ++s) {
+  for (int s = 0; s < S; ++s) {
     if (s < p.splits) {
-      ml[s] = p.ws_ml[((size_t)unit * p.splits + s) * TC_BM + row];
-      M = fmaxf(M, ml[s].x);
+      const size_t slot = (size_t)unit * p.splits + s;
+      ml[s] = p.ws_ml[slot * TC_BM + row];
+      // partial O layout: [slot][D/4][128 rows] float4, so consecutive rows are consecutive
+      const float4* wo = reinterpret_cast<const float4*>(p.ws_o) + (slot * (TC_D / 4) + d0 / 4) * TC_BM + row;
+      pa[s] = wo[0];
+      pb[s] = wo[TC_BM];
     }
   }
+  float M = -INFINITY;
+#pragma unroll
+  for (int s = 0; s < S; ++s)
+    if (s < p.splits) M = fmaxf(M, ml[s].x);
   float wsum = 0.f;
   float acc[8];
 #pragma unroll
   for (int d = 0; d < 8; ++d) acc[d] = 0.f;
 #pragma unroll
-  for (int s = 0; s < TC_MAX_SPLITS; ++s) {
+  for (int s = 0; s < S; ++s) {
     if (s < p.splits && ml[s].x != -INFINITY) {
       const float w = exp2f(ml[s].x - M);
       wsum += w * ml[s].y;
-      const float4* wo =
-          reinterpret_cast<const float4*>(p.ws_o + (((size_t)unit * p.splits + s) * TC_BM + row) * TC_D + d0);
-      const float4 a = wo[0], b = wo[1];
-      acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
-      acc[4] += w * b.x; acc[5] += w * b.y; acc[6] += w * b.z; acc[7] += w * b.w;
+      acc[0] += w * pa[s].x; acc[1] += w * pa[s].y; acc[2] += w * pa[s].z; acc[3] += w * pa[s].w;
+      acc[4] += w * pb[s].x; acc[5] += w * pb[s].y; acc[6] += w * pb[s].z; acc[7] += w * pb[s].w;
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
@@ -738,7 +745,10 @@ inline int tc_attn_launch(const void* q, const void* kc, const void* vc, const i
   tree_attn_tc_kernel<<<(unsigned)grid, TC_THREADS, TC_SMEM_BYTES, stream>>>(mq, mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return DDTREE_ERR_CUDA;
   if (pl.splits > 1) {
-    tree_attn_combine_kernel<<<pl.units * (TC_BM / TC_COMBINE_ROWS), 128, 0, stream>>>(p);
+    if (pl.splits <= 8)
+      tree_attn_combine_kernel<8><<<pl.units * (TC_D / 8), TC_BM, 0, stream>>>(p);
+    else
+      tree_attn_combine_kernel<TC_MAX_SPLITS><<<pl.units * (TC_D / 8), TC_BM, 0, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return DDTREE_ERR_CUDA;
   }
   return DDTREE_OK;

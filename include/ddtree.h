@@ -163,6 +163,10 @@ size_t ddtree_attn_workspace_bytes(const ddtree_kv_desc* kv, int B);
  *            in anc[i].  Rows of absent nodes are not written.
  * out_lse    device float [layers][n_req][B+1][Hq] natural-log sum-exp of the
  *            scaled scores (may be NULL).
+ * ws         device scratch of ddtree_attn_workspace_bytes(kv, B) bytes
+ *            (16-byte aligned; NULL when that is 0).  It must be zero-filled
+ *            before its first use; every call leaves its counters at zero.
+ *            Calls that share a workspace must not overlap.
  * bf16: tcgen05 tensor-core path for D = 128 (fp32 accumulation, P rounded
  * to bf16 for the PV product); fp32 and D = 64: CUDA-core fp32 path.
  */

@@ -458,6 +458,22 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         m_new = m_tile;
         rescale = true;
       }
+      // P = exp2(s*sl2 - m) as packed bf16 in registers first (exp2(-inf) = 0
+      // masks), so the exponentials overlap the previous tile's PV product
+      const float m_eff = rescale ? m_new : m_used;
+      const float mneg = (m_eff == -INFINITY) ? 0.f : -m_eff;
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[TC_BN / 2];
+#pragma unroll
+      for (int ch = 0; ch < TC_BN / 8; ++ch) {       // 8 keys at a time
+        float e[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) e[t] = exp2f(fmaf(s[ch * 8 + t], sl2, mneg));
+#pragma unroll
+        for (int t = 0; t < 4; ++t) pk[ch * 4 + t] = pack_bf16x2(e[2 * t], e[2 * t + 1]);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) ls4[t & 3] += e[t];
+      }
       // P buffer and O are free once the previous PV has retired
       if (jj > 0) {
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_pvdone, (jj - 1) & 1, abort))) { ok = false; break; }
@@ -480,26 +496,15 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         if (rescale) m_used = m_new;
       }
-      // P = exp2(s*sl2 - m) as bf16 into the swizzled K-major tile (exp2(-inf) = 0 masks)
-      const float mneg = (m_used == -INFINITY) ? 0.f : -m_used;
-      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+      l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+      // into the swizzled K-major P tile
       unsigned char* prow = sm.p + row * 128;
 #pragma unroll
-      for (int ch = 0; ch < TC_BN / 8; ++ch) {       // 16-byte chunks of 8 keys
-        float e[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) e[t] = exp2f(fmaf(s[ch * 8 + t], sl2, mneg));
-        uint4 pk;
-        pk.x = pack_bf16x2(e[0], e[1]);
-        pk.y = pack_bf16x2(e[2], e[3]);
-        pk.z = pack_bf16x2(e[4], e[5]);
-        pk.w = pack_bf16x2(e[6], e[7]);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) ls4[t & 3] += e[t];
+      for (int ch = 0; ch < TC_BN / 8; ++ch) {
         const int atom = ch >> 3, c16 = ch & 7;
-        *reinterpret_cast<uint4*>(prow + atom * TC_ATOM + ((c16 ^ (row & 7)) << 4)) = pk;
+        *reinterpret_cast<uint4*>(prow + atom * TC_ATOM + ((c16 ^ (row & 7)) << 4)) =
+            make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
       }
-      l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
       mbar_arrive(&sm.bar_pfull);

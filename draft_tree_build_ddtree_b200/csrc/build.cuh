@@ -102,13 +102,14 @@ struct BuildSmem {
   float* nd_score;
 };
 
+// node arrays (16n bytes), the lp table (padded to 16 bytes), keys (8n), slot score, parent score, metadata (12n)
 __host__ __device__ inline size_t build_smem_bytes(int L, int kc, int B) {
   const size_t n = (size_t)B + 1;
-  return (size_t)L * kc * 4 + n * (8 + 4 + 4 + 4) + n * 4 * 4;
+  return n * 16 + (((size_t)L * kc * 4 + 15) & ~(size_t)15) + n * (8 + 4 + 4 + 4);
 }
-inline size_t enum_smem_bytes();
+__host__ __device__ inline size_t enum_smem_bytes();
 // with the enumeration arrays after the heap's
-inline size_t build_smem_bytes_enum(int L, int kc, int B) {
+__host__ __device__ inline size_t build_smem_bytes_enum(int L, int kc, int B) {
   return ((build_smem_bytes(L, kc, B) + 15) & ~(size_t)15) + enum_smem_bytes();
 }
 
@@ -338,7 +339,7 @@ struct EnumSmem {
   uint16_t* pos;                // [ENUM_CAP] node index of an entry (0: not selected)
 };
 
-inline size_t enum_smem_bytes() { return (size_t)ENUM_CAP * (4 + 4 + 8 + 2 + 2) + (ENUM_CAP + 1) * 4; }
+__host__ __device__ inline size_t enum_smem_bytes() { return (size_t)ENUM_CAP * (4 + 4 + 8 + 2 + 2) + (ENUM_CAP + 1) * 4; }
 
 // Lexicographic tuple comparison of two enumerated entries (a proper prefix
 // is smaller): lift the deeper entry, then walk both up to a common parent.
@@ -413,13 +414,57 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
   __syncthreads();
   uint32_t t = 1u;                                // every finite or -inf score
   if ((long long)L * kc >= B) {
-    auto each = [&](auto f) {
-      for (int i = tid; i < L * kc; i += BUILD_THREADS) {
-        const int d = i / kc;
-        f(score_key(__fadd_rn(chain[d], sm.lp[i])));
+    // One histogram over the family's key range [kmin, kmax] in 256 equal
+    // bins; the lower edge of the bin where the count from the top reaches B
+    // is a threshold that at least B prefixes reach (a lower bound of the
+    // B-th best, within one bin).  The largest family score is lp[0][0]
+    // (chains only fall); the smallest is the last rank at some depth.
+    const uint32_t kmax = score_key(sm.lp[0]);
+    if (tid < 32) {
+      uint32_t kmin = 0xFFFFFFFFu;
+      for (int d = tid; d < L; d += 32) kmin = min(kmin, score_key(__fadd_rn(chain[d], sm.lp[d * kc + kc - 1])));
+      kmin = __reduce_min_sync(0xffffffffu, kmin);
+      if (tid == 0) bcast[0] = (int)kmin;
+    }
+    for (int i = tid; i < 256; i += BUILD_THREADS) hist[i] = 0;
+    __syncthreads();
+    const uint32_t kmin = (uint32_t)bcast[0];
+    int shift = 0;
+    while (((kmax - kmin) >> shift) >= 256u) ++shift;
+    for (int i = tid; i < L * kc; i += BUILD_THREADS) {
+      const int d = i / kc;
+      const uint32_t key = score_key(__fadd_rn(chain[d], sm.lp[i]));
+      atomicAdd(&hist[(key - kmin) >> shift], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) {   // lane l holds bins 255-8l .. 248-8l (descending)
+      uint32_t c[8];
+      uint32_t mine = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { c[j] = hist[255 - 8 * tid - j]; mine += c[j]; }
+      uint32_t incl = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += y;
       }
-    };
-    t = radix_kth<uint32_t>(each, 32, B, hist, bcast).t;
+      const uint32_t before = incl - mine;
+      const unsigned m = __ballot_sync(0xffffffffu, before < (uint32_t)B && (uint32_t)B <= incl);
+      if (tid == __ffs(m) - 1) {
+        uint32_t acc = before;
+        int jb = 7;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          acc += c[j];
+          if (acc >= (uint32_t)B) { jb = j; break; }
+        }
+        bcast[1] = 255 - 8 * tid - jb;
+      }
+      if (m == 0 && tid == 0) bcast[1] = 0;        // cannot happen (L*kc >= B); keep every key
+    }
+    __syncthreads();
+    t = kmin + ((uint32_t)bcast[1] << shift);
+    if (t == 0u) t = 1u;
   }
   // ---- 2. every prefix with score key >= t, level by level ----
   // depth 1: children of the root
@@ -490,8 +535,27 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
     while (g > 1 && total * g > BUILD_THREADS) g >>= 1;
     const int q = tid / g, part = tid - q * g;
     int rank = 0;
-    if (q < total)
-      for (int j = part; j < total; j += g) rank += (j != q && e_before(j, q, es)) ? 1 : 0;
+    if (q < total) {
+      // 64-bit keys first (four independent counts); equal keys (identical
+      // score and leading ranks) are settled by the tuple walk
+      const unsigned long long kq = es.key[q];
+      int r0 = 0, r1 = 0, r2 = 0, r3 = 0, ties = 0;
+      int j = part;
+      for (; j + 3 * g < total; j += 4 * g) {
+        const unsigned long long k0 = es.key[j], k1 = es.key[j + g], k2 = es.key[j + 2 * g], k3 = es.key[j + 3 * g];
+        r0 += k0 > kq; r1 += k1 > kq; r2 += k2 > kq; r3 += k3 > kq;
+        ties += (k0 == kq) + (k1 == kq) + (k2 == kq) + (k3 == kq);
+      }
+      for (; j < total; j += g) {
+        const unsigned long long kj = es.key[j];
+        r0 += kj > kq;
+        ties += kj == kq;
+      }
+      rank = (r0 + r1) + (r2 + r3);
+      if (ties > (part == (q % g) ? 1 : 0))       // another entry shares the key
+        for (int jj = part; jj < total; jj += g)
+          if (jj != q && es.key[jj] == kq && e_tuple_less(jj, q, es.meta)) ++rank;
+    }
     for (int o = g >> 1; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
     if (q < total && part == 0) es.pos[q] = (uint16_t)(rank < npop ? rank + 1 : 0);
   } else {
@@ -501,14 +565,37 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
     __syncthreads();
     for (int size = 2; size <= P; size <<= 1) {
       for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int i = tid; i < P / 2; i += BUILD_THREADS) {
-          const int lo = 2 * stride * (i / stride) + (i % stride);
-          const int hi = lo + stride;
-          const bool up = (lo & size) == 0;       // this run sorts in pop order
-          const uint16_t a = es.ord[lo], b = es.ord[hi];
-          // b before a (pads last)
-          const bool b_first = b != 0xFFFFu && (a == 0xFFFFu || e_before(b, a, es));
-          if (b_first == up) { es.ord[lo] = b; es.ord[hi] = a; }
+        // up to four compare-exchanges per thread, their loads issued together
+        for (int i0 = tid; i0 < P / 2; i0 += 4 * BUILD_THREADS) {
+          int lo[4], hi[4];
+          uint16_t a[4], b[4];
+          unsigned long long ka[4], kb[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * BUILD_THREADS;
+            lo[u] = 2 * stride * (i / stride) + (i % stride);
+            hi[u] = lo[u] + stride;
+            const bool in = i < P / 2;
+            a[u] = in ? es.ord[lo[u]] : 0xFFFFu;
+            b[u] = in ? es.ord[hi[u]] : 0xFFFFu;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            ka[u] = a[u] != 0xFFFFu ? es.key[a[u]] : 0ull;
+            kb[u] = b[u] != 0xFFFFu ? es.key[b[u]] : 0ull;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (i0 + u * BUILD_THREADS >= P / 2) continue;
+            const bool up = (lo[u] & size) == 0;   // this run sorts in pop order
+            // b before a (pads last)
+            bool b_first;
+            if (b[u] == 0xFFFFu) b_first = false;
+            else if (a[u] == 0xFFFFu) b_first = true;
+            else if (ka[u] != kb[u]) b_first = kb[u] > ka[u];
+            else b_first = e_tuple_less(b[u], a[u], es.meta);
+            if (b_first == up) { es.ord[lo[u]] = b[u]; es.ord[hi[u]] = a[u]; }
+          }
         }
         __syncthreads();
       }
@@ -546,16 +633,17 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
 
   BuildSmem sm;
   {
+    // the node arrays first: everything after them is dead once the pops are known
     unsigned char* p = smem_raw;
-    sm.key = (uint2*)p;     p += (size_t)n * 8;
-    sm.lp = (float*)p;      p += (size_t)L * kc * 4;
-    sm.sc = (float*)p;      p += (size_t)n * 4;
-    sm.ps = (float*)p;      p += (size_t)n * 4;
-    sm.mt = (uint32_t*)p;   p += (size_t)n * 4;
     sm.nd_parent = (int*)p; p += (size_t)n * 4;
     sm.nd_rank = (int*)p;   p += (size_t)n * 4;
     sm.nd_depth = (int*)p;  p += (size_t)n * 4;
-    sm.nd_score = (float*)p;
+    sm.nd_score = (float*)p; p += (size_t)n * 4;
+    sm.lp = (float*)p;      p += ((size_t)L * kc * 4 + 15) & ~(size_t)15;   // 16-byte aligned
+    sm.key = (uint2*)p;     p += (size_t)n * 8;
+    sm.sc = (float*)p;      p += (size_t)n * 4;
+    sm.ps = (float*)p;      p += (size_t)n * 4;
+    sm.mt = (uint32_t*)p;
   }
   EnumSmem es;
   {
@@ -576,9 +664,28 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
 
   // stage the lp table (only ranks < kc can ever be popped)
   const float* lpr = lp + (size_t)r * L * K;
-  for (int i = tid; i < L * kc; i += BUILD_THREADS) {
-    const int d = i / kc, k = i - d * kc;
-    sm.lp[i] = lpr[(size_t)d * K + k];
+  if ((kc & 3) == 0 && (K & 3) == 0 && ((uintptr_t)lpr & 15) == 0) {
+    // 16-byte loads, all of a thread's issued before any is stored
+    const int q4 = kc >> 2, total4 = L * q4;
+    for (int i0 = tid; i0 < total4; i0 += 4 * BUILD_THREADS) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * BUILD_THREADS;
+        const int d = i / q4, k4 = i - d * q4;
+        if (i < total4) v[u] = *reinterpret_cast<const float4*>(lpr + (size_t)d * K + 4 * k4);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * BUILD_THREADS;
+        if (i < total4) reinterpret_cast<float4*>(sm.lp)[i] = v[u];
+      }
+    }
+  } else {
+    for (int i = tid; i < L * kc; i += BUILD_THREADS) {
+      const int d = i / kc, k = i - d * kc;
+      sm.lp[i] = lpr[(size_t)d * K + k];
+    }
   }
   __syncthreads();
 
@@ -606,6 +713,51 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
   const int nn = s_pops + 1;
   const size_t ro = (size_t)r * n;
   const int32_t* idr = ids + (size_t)r * L * K;
+  // Ancestor rows for wide masks: built in shared memory one depth level at a
+  // time (row i = row parent(i) | bit i, a warp per row, lanes over words),
+  // then written out with 16-byte stores.  Needs n*W words of the dead area.
+  const size_t dead = (use_enum ? build_smem_bytes_enum(L, kc, B) : build_smem_bytes(L, kc, B)) - (size_t)n * 16;
+  const bool smem_rows = W >= 4 && (size_t)n * (W + 1) * 4 <= dead;
+  if (smem_rows) {
+    uint32_t* rows = reinterpret_cast<uint32_t*>(smem_raw + (size_t)n * 16);   // [n][W]
+    int* order = reinterpret_cast<int*>(rows + (size_t)n * W);                  // [n] nodes sorted by depth
+    __shared__ int s_dcnt[66];
+    for (int i = tid; i < 66; i += BUILD_THREADS) s_dcnt[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < nn; i += BUILD_THREADS) atomicAdd(&s_dcnt[sm.nd_depth[i] + 1], 1);
+    __syncthreads();
+    if (tid == 0)
+      for (int d = 1; d < 66; ++d) s_dcnt[d] += s_dcnt[d - 1];   // s_dcnt[d]: first slot of depth d
+    __syncthreads();
+    for (int i = tid; i < nn; i += BUILD_THREADS) order[atomicAdd(&s_dcnt[sm.nd_depth[i]], 1)] = i;
+    __syncthreads();
+    // after the scatter s_dcnt[d] is the end of depth d: depth d spans [s_dcnt[d-1], s_dcnt[d])
+    const int lane = tid & 31, wrp = tid >> 5;
+    for (int w = lane; w < W; w += 32) rows[w] = (w == 0) ? 1u : 0u;   // the root row
+    __syncthreads();
+    for (int d = 1; d <= L; ++d) {
+      const int b0 = s_dcnt[d - 1], b1 = s_dcnt[d];
+      if (b0 >= b1) break;
+      for (int k = b0 + wrp; k < b1; k += BUILD_THREADS / 32) {
+        const int i = order[k];
+        const int pi = sm.nd_parent[i];
+        for (int w = lane; w < W; w += 32)
+          rows[(size_t)i * W + w] = rows[(size_t)pi * W + w] | ((i >> 5) == w ? (1u << (i & 31)) : 0u);
+      }
+      __syncthreads();
+    }
+    for (int i = nn * W + tid; i < n * W; i += BUILD_THREADS) rows[i] = 0u;   // absent nodes
+    __syncthreads();
+    uint32_t* arow0 = anc + ro * W;
+    const int words = n * W;
+    if (((uintptr_t)arow0 & 15) == 0) {
+      for (int i = tid; i < words / 4; i += BUILD_THREADS)
+        reinterpret_cast<uint4*>(arow0)[i] = reinterpret_cast<const uint4*>(rows)[i];
+      for (int i = (words & ~3) + tid; i < words; i += BUILD_THREADS) arow0[i] = rows[i];
+    } else {
+      for (int i = tid; i < words; i += BUILD_THREADS) arow0[i] = rows[i];
+    }
+  }
   for (int i = tid; i < n; i += BUILD_THREADS) {
     const bool live = i < nn;
     const int d = live ? sm.nd_depth[i] : -1;
@@ -615,6 +767,7 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
     if (depth) depth[ro + i] = d;
     if (node_rank) node_rank[ro + i] = rk;
     if (score) score[ro + i] = live ? sm.nd_score[i] : -INFINITY;
+    if (smem_rows) continue;
     // ancestor-or-self bitmask: walk up the chain, words from high to low
     uint32_t* arow = anc + ro * W + (size_t)i * W;
     int j = live ? i : -1;

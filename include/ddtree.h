@@ -271,7 +271,7 @@ int ddtree_round(const ddtree_round_args* a, cudaStream_t stream);
  *    loaded, held until the process exits).  A request whose scratch need,
  *    ddtree_topk_workspace_bytes(rows, V, K), exceeds it is rejected with
  *    DDTREE_ERR_SCRATCH_LIMIT before anything is launched (at V = 151936
- *    and bf16 logits: up to 573 rows at K = 64, 145 at K = 256, 48 at
+ *    and bf16 logits: up to 571 rows at K = 64, 145 at K = 256, 48 at
  *    K = 1024 on a 148-SM B200).
  *  - The first call on a device looks up the array's device address on the
  *    current device; make that first call before any stream capture.

@@ -80,6 +80,27 @@ int set_smem(F* kernel, size_t bytes) {
 }
 
 // ------------------------------------------------------------------ topk
+// The exp(z) table of every bf16 value is built once per device, on the
+// first bf16 top-K call, which then synchronizes its stream once (inside a
+// stream capture the build is captured instead: it is idempotent).
+constexpr int EXP_TABLE_MAX_DEVICES = 64;
+bool g_exp_table_ready[EXP_TABLE_MAX_DEVICES];
+
+int ensure_exp_table(cudaStream_t s) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= EXP_TABLE_MAX_DEVICES) return DDTREE_ERR_CUDA;
+  if (g_exp_table_ready[dev]) return DDTREE_OK;
+  exp_bf16_table_kernel<<<65536 / 256, 256, 0, s>>>();
+  if (cudaGetLastError() != cudaSuccess) return DDTREE_ERR_CUDA;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return DDTREE_ERR_CUDA;
+  if (cs == cudaStreamCaptureStatusNone) {
+    if (cudaStreamSynchronize(s) != cudaSuccess) return DDTREE_ERR_CUDA;
+    g_exp_table_ready[dev] = true;
+  }
+  return DDTREE_OK;
+}
+
 int topk_check(const void* logits, int dtype, int rows, int V, long long row_stride, int K,
                const void* ids, const void* lp) {
   if (!logits || !ids || !lp) return DDTREE_ERR_INVALID_ARG;
@@ -107,6 +128,7 @@ int topk_launch(const void* logits, int dtype, int rows, int V, long long row_st
   const long long grid = (long long)rows * p.cpr;
   if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
   if (dtype == DDTREE_BF16) {
+    if ((st = ensure_exp_table(s))) return st;
     switch (p.vpt) {
 #define DDT_TOPK_CASE(VP)                                                                                   \
   case VP:                                                                                                  \

@@ -122,8 +122,9 @@ inline TopkWs topk_ws_carve(void* ws, int rows, const TopkPlan& p) {
   return w;
 }
 
-// exp(x) in fp64 for x <= 0 (table-driven; relative error ~1e-16).  x is
-// clamped at -700, where exp is ~1e-304 and the result stays normal.  The
+// exp(x) in fp64 for -700 <= x <= 700 (table-driven; relative error ~1e-16).
+// x is clamped at -700 from below, where exp is ~1e-304 and the result
+// stays normal.  The
 // reduction k = round(x * 64/ln2) rounds with the 1.5*2^52 shifter (k lands in
 // the low word), r = x - k*ln2/64 in two exact-product steps, then
 // 2^(k/64) * exp(r) = 2^(k>>6) * T[k&63] * (1 + p(r)).
@@ -144,6 +145,28 @@ __device__ __forceinline__ double exp64(double x, const double* tab) {
   const double y = fma(tj, p, tj);          // 2^(j/64) * exp(r), in [0.99, 2.02)
   return __hiloint2double(__double2hiint(y) + ((k >> 6) << 20), __double2loint(y));
 }
+
+// exp(z) in fp64 for every bf16 bit pattern z with |z| <= 700 (others 0),
+// built once per device by exp_bf16_table_kernel.  With it a chunk's sum of
+// exp(z - m) is one cached table load and one fp64 add per logit, scaled by
+// exp(-m) once: the fp64 exponential, which B200 runs at a small fraction of
+// its fp32 rate, is paid per distinct value instead of per logit.
+__device__ double g_exp_bf16[65536];
+
+__global__ void exp_bf16_table_kernel() {
+  __shared__ double tab[64];
+  if (threadIdx.x < 64) tab[threadIdx.x] = EXP64_TABLE[threadIdx.x];
+  __syncthreads();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < 65536) {
+    const float z = __uint_as_float((uint32_t)i << 16);
+    const double zd = (double)z;
+    g_exp_bf16[i] = (z == z && fabs(zd) <= 700.0) ? exp64(zd, tab) : 0.0;
+  }
+}
+
+// A chunk uses the table when its maximum keeps every scaled sum in range.
+constexpr double EXP_TABLE_MAX_M = 600.0;
 
 
 template <int DT>
@@ -339,6 +362,7 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   const float m = key_value<DT>(kmax);
   const double md = (double)m;
   const bool m_finite = m > -INFINITY;
+  const bool use_table = DT == DDTREE_BF16 && md <= EXP_TABLE_MAX_M && md >= -EXP_TABLE_MAX_M;
 
   uint32_t tval = 0;
   int above = 0, eq = 0;
@@ -354,10 +378,14 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
         double e[EPV];
 #pragma unroll
         for (int j = 0; j < EPV; ++j) {
-          const float z = DT == DDTREE_BF16 ? bf16_bits_to_f32((uint16_t)elem_bits<DT>(v, j))
-                                            : __uint_as_float(u32_at(v, j));
-          e[j] = exp64((double)z - md, s_tab);
-          e[j] = j < valid ? e[j] : 0.0;
+          if (use_table) {
+            e[j] = j < valid ? __ldg(&g_exp_bf16[elem_bits<DT>(v, j)]) : 0.0;   // exp(z); scaled below
+          } else {
+            const float z = DT == DDTREE_BF16 ? bf16_bits_to_f32((uint16_t)elem_bits<DT>(v, j))
+                                              : __uint_as_float(u32_at(v, j));
+            e[j] = exp64((double)z - md, s_tab);
+            e[j] = j < valid ? e[j] : 0.0;
+          }
         }
 #pragma unroll
         for (int j = 0; j < EPV; j += 2) { s0 += e[j]; s1 += e[j + 1]; }
@@ -499,6 +527,7 @@ topk_kernel(const void* __restrict__ logits, int rows, int V, long long row_stri
   if (tid == 0) {
     double tot = 0.0;
     for (int i = 0; i < NWE; ++i) tot += red_d[i];
+    if (use_table) tot *= exp64(-md, s_tab);           // sum of exp(z) -> sum of exp(z - m)
     ws.stats[(size_t)row * plan.cpr + c] = make_double2(md, tot);
     ws.count[(size_t)row * plan.cpr + c] = s_count < plan.cap ? s_count : plan.cap;
     ws.thr[(size_t)row * plan.cpr + c] = tval;

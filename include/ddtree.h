@@ -106,7 +106,9 @@ size_t ddtree_topk_workspace_bytes(int rows, int V, int K);
  * NaN logits set DDTREE_STATUS_NONFINITE; -inf is allowed and ranks last;
  * -0.0 ranks equal to +0.0.
  * lp is the fp64 value z - lse rounded once to fp32 (the sum of exp is taken
- * in fp64).
+ * in fp64).  The first bf16 call on a device builds a 512 KiB table of
+ * exp(z) for every bf16 value in static device memory and synchronizes
+ * `stream` once; make it before any stream capture.
  */
 int ddtree_topk(const void* logits, int dtype, int rows, int V, long long row_stride,
                 int K, int32_t* ids, float* lp, float* lse,
@@ -274,7 +276,9 @@ int ddtree_round(const ddtree_round_args* a, cudaStream_t stream);
  *    and bf16 logits: up to 571 rows at K = 64, 145 at K = 256, 48 at
  *    K = 1024 on a 148-SM B200).
  *  - The first call on a device looks up the array's device address on the
- *    current device; make that first call before any stream capture.
+ *    current device (and, for bf16, builds the exp table as ddtree_topk
+ *    does, synchronizing `stream` once); make that first call before any
+ *    stream capture.
  *  - Every call on a device shares the one array and leaves its contents
  *    behind; each call clears the counters it needs at its start.  Calls
  *    that overlap on the GPU (other streams, other host threads) race on the

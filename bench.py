@@ -334,30 +334,41 @@ def run_ours(a):
     value = aggregate_rate(a.steps, world, ms_max / 1e3)
     status = dd.device_status()
 
-    # ---- per-stage kernel times (graphs of one launch per input set) ----
-    stage_ms = {}
-    reps = max(3, min(200, a.steps // R))
-    for name in ("topk", "build", "attn", "accept"):
-        fns = [stage_calls(w, rb)[name] for rb in sets]
-        for f in fns:
-            f()
-        torch.cuda.synchronize()
+    # ---- per-stage kernel times, with cold caches as in the rounds: a graph of
+    #      (L2 flush, stage on set k) for every set, minus the same graph of
+    #      flushes alone ----
+    names = ("topk", "build", "attn", "accept")
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
+
+    def timed(fn, n):
         if use_graph:
-            g = capture(lambda fns=fns: [f() for f in fns], side)
+            g = capture(fn, side)
             run = g.replay
         else:
-            def run(fns=fns):
-                for f in fns:
-                    f()
+            run = fn
         run()
         torch.cuda.synchronize()
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        for _ in range(reps):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(n):
             run()
-        s1.record(stream)
+        t1.record(stream)
         torch.cuda.synchronize()
-        stage_ms[name] = s0.elapsed_time(s1) / (reps * R)
+        return t0.elapsed_time(t1)
+
+    reps = max(3, min(20, a.steps // R))
+    t_flush = timed(lambda: [flush_buf.zero_() for _ in range(R)], reps)
+    stage_ms = {}
+    for name in names:
+        fns = [stage_calls(w, rb)[name] for rb in sets]
+
+        def flushed(fns=fns):
+            for f in fns:
+                flush_buf.zero_()
+                f()
+
+        stage_ms[name] = max(0.0, timed(flushed, reps) - t_flush) / (reps * R)
+    del flush_buf
     # restore the caches the stage runs compacted are irrelevant: sizes do not change
 
     work = algorithmic_work(w, sets[0])

@@ -44,12 +44,24 @@ namespace ddt {
 
 constexpr int TC_THREADS = 192;
 constexpr int TC_BM = 128;        // rows per M-tile
-constexpr int TC_BN = 128;        // keys per tile
 constexpr int TC_D = 128;         // head dim
 constexpr int TC_ATOM = TC_BM * 64 * 2;     // one [128][64] bf16 swizzle-128B atom column: 16 KB
-constexpr int TC_TILE = 2 * TC_ATOM;        // [128][128] bf16: 32 KB
+constexpr int TC_TILE = 2 * TC_ATOM;        // [128][128] bf16: 32 KB (Q)
+constexpr int TC_MIN_SPLIT_TILES = 4;
+constexpr int TC_SHORT_TILES = 6;
+
+// Key-tile variants: 128 keys per tile, one CTA per SM (short, split key
+// ranges: fewer tiles per CTA), or 64 keys (one KV page) per tile, two CTAs
+// per SM (long key ranges: the two CTAs' softmax and MMAs interleave).
+template <int BN>
+struct TcCfg {
+  static constexpr int KATOM = BN * 64 * 2;     // one [BN keys][64 dims] bf16 atom
+  static constexpr int KTILE = 2 * KATOM;       // a K or V tile [BN keys][128 dims]
+  static constexpr int PTILE = TC_BM * BN * 2;  // P [128 rows][BN keys] bf16
+  static constexpr int CTAS = BN == 64 ? 2 : 1; // CTAs per SM
+};
 constexpr int TC_STAGES = 2;
-constexpr uint32_t TC_TMEM_COLS = 256;      // S: cols [0,128), O: cols [128,256)
+constexpr uint32_t TC_TMEM_COLS = 256;      // S: cols [0,64), O: cols [64,192); two CTAs per SM
 constexpr float TC_RESCALE_LOG2 = 8.0f;
 
 inline bool tc_attn_supported(int group) { return group >= 1 && group <= TC_BM && (TC_BM % group) == 0; }
@@ -202,12 +214,13 @@ struct TcParams {
   float2* ws_ml;       // [units*splits][128] (max in log2 units, sum)
 };
 
+template <int BN>
 struct TcSmem {
   // 1024-byte aligned tiles first
   unsigned char q[TC_TILE];
-  unsigned char k[TC_STAGES][TC_TILE];
-  unsigned char v[TC_STAGES][TC_TILE];
-  unsigned char p[TC_TILE];
+  unsigned char k[TC_STAGES][TcCfg<BN>::KTILE];
+  unsigned char v[TC_STAGES][TcCfg<BN>::KTILE];
+  unsigned char p[TcCfg<BN>::PTILE];
   uint64_t bar_q, bar_kf[TC_STAGES], bar_ke[TC_STAGES], bar_vf[TC_STAGES], bar_ve[TC_STAGES];
   uint64_t bar_sfull, bar_sfree, bar_pfull, bar_pvdone;
   uint32_t tmem_base;
@@ -215,14 +228,26 @@ struct TcSmem {
   int blk[2];
 };
 
-constexpr size_t TC_SMEM_BYTES = sizeof(TcSmem) + 1024;   // + alignment slack
+// Two CTAs share an SM, so there is no room for alignment slack: the
+// dynamic shared memory (no static shared memory in the kernel) starts at
+// shared address 0, which the kernel checks.
+template <int BN>
+constexpr size_t tc_smem_bytes() { return sizeof(TcSmem<BN>); }
 
 // ---------------------------------------------------------------- the kernel
-__global__ void __launch_bounds__(TC_THREADS, 1)
+template <int BN>
+__global__ void __launch_bounds__(TC_THREADS, TcCfg<BN>::CTAS)
 tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const TcParams p) {
-  extern __shared__ unsigned char smem_dyn[];
-  TcSmem& sm = *reinterpret_cast<TcSmem*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~(uintptr_t)1023);
+  extern __shared__ __align__(1024) unsigned char smem_dyn[];
+  constexpr int TC_BN = BN;
+  constexpr int TC_KATOM = TcCfg<BN>::KATOM;
+  constexpr int TC_KTILE = TcCfg<BN>::KTILE;
+  TcSmem<BN>& sm = *reinterpret_cast<TcSmem<BN>*>(smem_dyn);
+  if ((smem_u32(smem_dyn) & 1023u) != 0u) {       // the 128B-swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) flag_status(DDTREE_STATUS_TIMEOUT);
+    return;
+  }
   const AttnGeom& g = p.g;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -288,8 +313,8 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t tmem_s = tmem;              // cols [0,128)
-  const uint32_t tmem_o = tmem + 128;        // cols [128,256)
+  const uint32_t tmem_s = tmem;              // cols [0,64)
+  const uint32_t tmem_o = tmem + TC_BN;      // cols [BN, BN+128)
   volatile int* abort = &sm.abort;
   const float sl2 = g.scale * 1.4426950408889634f;   // scale * log2(e)
 
@@ -306,37 +331,35 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int st = jj % TC_STAGES;
         const int use = jj / TC_STAGES;
         const int k0 = j * TC_BN;
+        // KV pages of this tile (paged: their blocks through the block table; a
+        // 128-key tile whose second page lies past the validated range reuses
+        // the first, whose keys are masked)
         int b0 = 0, b1 = 0;
         if (g.paged) {
           const int pg = k0 / DDTREE_PAGE;
           const int maxpg = (T + DDTREE_PAGE - 1) / DDTREE_PAGE;   // validated blocks
           b0 = p.block_table[(size_t)r * g.max_blocks + pg];
-          b1 = (pg + 1 < maxpg) ? p.block_table[(size_t)r * g.max_blocks + pg + 1] : b0;
+          b1 = (BN > DDTREE_PAGE && pg + 1 < maxpg) ? p.block_table[(size_t)r * g.max_blocks + pg + 1] : b0;
         }
+        auto load_tile = [&](const CUtensorMap* map, unsigned char* tile, uint64_t* bar) {
+          mbar_expect_tx(bar, TC_KTILE);
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t dst = smem_u32(tile + h * TC_KATOM);
+            if (!g.paged) {
+              tma_load_4d(dst, map, bar, 64 * h, kvh, k0, layer * g.n_req + r);
+            } else {
+              tma_load_4d(dst, map, bar, 64 * h, kvh, 0, layer * g.num_blocks + b0);
+              if (BN > DDTREE_PAGE)
+                tma_load_4d(dst + TC_KATOM / 2, map, bar, 64 * h, kvh, 0, layer * g.num_blocks + b1);
+            }
+          }
+        };
         // K tile
         if (use > 0 && !mbar_wait(&sm.bar_ke[st], (use - 1) & 1, abort)) break;
-        mbar_expect_tx(&sm.bar_kf[st], TC_TILE);
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t dst = smem_u32(sm.k[st] + h * TC_ATOM);
-          if (!g.paged) {
-            tma_load_4d(dst, &tm_k, &sm.bar_kf[st], 64 * h, kvh, k0, layer * g.n_req + r);
-          } else {
-            tma_load_4d(dst, &tm_k, &sm.bar_kf[st], 64 * h, kvh, 0, layer * g.num_blocks + b0);
-            tma_load_4d(dst + TC_ATOM / 2, &tm_k, &sm.bar_kf[st], 64 * h, kvh, 0, layer * g.num_blocks + b1);
-          }
-        }
+        load_tile(&tm_k, sm.k[st], &sm.bar_kf[st]);
         // V tile
         if (use > 0 && !mbar_wait(&sm.bar_ve[st], (use - 1) & 1, abort)) break;
-        mbar_expect_tx(&sm.bar_vf[st], TC_TILE);
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t dst = smem_u32(sm.v[st] + h * TC_ATOM);
-          if (!g.paged) {
-            tma_load_4d(dst, &tm_v, &sm.bar_vf[st], 64 * h, kvh, k0, layer * g.n_req + r);
-          } else {
-            tma_load_4d(dst, &tm_v, &sm.bar_vf[st], 64 * h, kvh, 0, layer * g.num_blocks + b0);
-            tma_load_4d(dst + TC_ATOM / 2, &tm_v, &sm.bar_vf[st], 64 * h, kvh, 0, layer * g.num_blocks + b1);
-          }
-        }
+        load_tile(&tm_v, sm.v[st], &sm.bar_vf[st]);
         issued = jj + 1;
       }
       // copies in flight must land before the CTA exits
@@ -366,8 +389,9 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const uint32_t k_addr = smem_u32(sm.k[st]);
 #pragma unroll
           for (int kk = 0; kk < TC_D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * TC_ATOM + (kk & 3) * 32;
-            umma_f16(tmem_s, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
+            const uint32_t qoff = (kk >> 2) * TC_ATOM + (kk & 3) * 32;
+            const uint32_t koff = (kk >> 2) * TC_KATOM + (kk & 3) * 32;
+            umma_f16(tmem_s, smem_desc_sw128(q_addr + qoff, 16, 1024), smem_desc_sw128(k_addr + koff, 16, 1024),
                      IDESC_QK, kk > 0);
           }
           umma_commit(&sm.bar_sfull);
@@ -382,9 +406,9 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const uint32_t v_addr = smem_u32(sm.v[st]);
 #pragma unroll
           for (int kk = 0; kk < TC_BN / 16; ++kk) {
-            const uint32_t a_off = (kk >> 2) * TC_ATOM + (kk & 3) * 32;
+            const uint32_t a_off = (kk >> 2) * TC_ATOM + (kk & 3) * 32;   // P: 64-key atoms
             umma_f16(tmem_o, smem_desc_sw128(p_addr + a_off, 16, 1024),
-                     smem_desc_sw128(v_addr + kk * 16 * 128, TC_ATOM, 1024), IDESC_PV, (pj > 0 || kk > 0));
+                     smem_desc_sw128(v_addr + kk * 16 * 128, TC_KATOM, 1024), IDESC_PV, (pj > 0 || kk > 0));
           }
           umma_commit(&sm.bar_pvdone);
           umma_commit(&sm.bar_ve[st]);
@@ -644,7 +668,7 @@ tree_attn_combine_kernel(const TcParams p) {
 
 // ---------------------------------------------------------------- host side
 struct TcPlan {
-  int G, mtiles, splits, units;
+  int G, mtiles, splits, units, bn;
 };
 
 inline TcPlan tc_plan(const AttnGeom& g, int num_sms) {
@@ -652,15 +676,32 @@ inline TcPlan tc_plan(const AttnGeom& g, int num_sms) {
   pl.G = g.Hq / g.Hkv;
   pl.mtiles = (g.n * pl.G + TC_BM - 1) / TC_BM;
   pl.units = g.layers * g.n_req * g.Hkv * pl.mtiles;
-  // split the key range only when the units alone leave SMs idle; a split
-  // must keep at least a few key tiles to amortise its set-up
-  int splits = 1;
-  if (pl.units < num_sms) {
-    splits = num_sms / pl.units;
-    if (splits > TC_MAX_SPLITS) splits = TC_MAX_SPLITS;
-    if (splits < 1) splits = 1;
+  // Split the key range only when the units alone leave CTA slots idle; a
+  // split keeps at least TC_MIN_SPLIT_TILES key tiles to amortise its
+  // set-up.  64-key tiles (two CTAs per SM) unless the split 128-key plan
+  // leaves each CTA fewer than TC_SHORT_TILES tiles (short prefixes).
+  const long long cap = g.paged ? (long long)g.max_blocks * DDTREE_PAGE : (long long)g.s_max;
+  auto plan_splits = [&](int bn, int ctas, int min_tiles) {
+    const int slots = num_sms * ctas;
+    const long long tiles_cap = (cap + bn - 1) / bn;
+    int splits = 1;
+    if (pl.units < slots) {
+      splits = slots / pl.units;
+      if (splits > TC_MAX_SPLITS) splits = TC_MAX_SPLITS;
+      if ((long long)splits * min_tiles > tiles_cap) splits = (int)(tiles_cap / min_tiles);
+      if (splits < 1) splits = 1;
+    }
+    return splits;
+  };
+  const int s128 = plan_splits(128, TcCfg<128>::CTAS, 1);
+  const long long t128 = (cap + 127) / 128;
+  if (pl.units < num_sms && t128 / s128 < TC_SHORT_TILES) {
+    pl.bn = 128;
+    pl.splits = s128;
+  } else {
+    pl.bn = 64;
+    pl.splits = plan_splits(64, TcCfg<64>::CTAS, TC_MIN_SPLIT_TILES);
   }
-  pl.splits = splits;
   return pl;
 }
 
@@ -730,8 +771,8 @@ inline int tc_attn_launch(const void* q, const void* kc, const void* vc, const i
                    (uint32_t)(TC_BM / pl.G)))
     return DDTREE_ERR_CUDA;
   if (!g.paged) {
-    if (!make_map_4d(&mk, kc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, TC_BN)) return DDTREE_ERR_CUDA;
-    if (!make_map_4d(&mv, vc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, TC_BN)) return DDTREE_ERR_CUDA;
+    if (!make_map_4d(&mk, kc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, pl.bn)) return DDTREE_ERR_CUDA;
+    if (!make_map_4d(&mv, vc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, pl.bn)) return DDTREE_ERR_CUDA;
   } else {
     if (!make_map_4d(&mk, kc, g.Hkv, DDTREE_PAGE, (uint64_t)g.layers * g.num_blocks, 1, DDTREE_PAGE))
       return DDTREE_ERR_CUDA;
@@ -740,14 +781,19 @@ inline int tc_attn_launch(const void* q, const void* kc, const void* vc, const i
   }
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(tree_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)TC_SMEM_BYTES) != cudaSuccess)
+    if (cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tc_smem_bytes<128>()) != cudaSuccess ||
+        cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tc_smem_bytes<64>()) != cudaSuccess)
       return DDTREE_ERR_CUDA;
     attr_set = true;
   }
   const long long grid = (long long)pl.units * pl.splits;
   if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
-  tree_attn_tc_kernel<<<(unsigned)grid, TC_THREADS, TC_SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  if (pl.bn == 64)
+    tree_attn_tc_kernel<64><<<(unsigned)grid, TC_THREADS, tc_smem_bytes<64>(), stream>>>(mq, mk, mv, p);
+  else
+    tree_attn_tc_kernel<128><<<(unsigned)grid, TC_THREADS, tc_smem_bytes<128>(), stream>>>(mq, mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return DDTREE_ERR_CUDA;
   if (pl.splits > 1) {
     if (pl.splits <= 8)

@@ -78,6 +78,7 @@ _SIGS = {
                            ctypes.POINTER(KVDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "ddtree_round_workspace_bytes": (_sz, [ctypes.POINTER(RoundArgs)]),
     "ddtree_round": (_i, [ctypes.POINTER(RoundArgs), _vp]),
+    "ddtree_round_launch_count": (_i, [ctypes.POINTER(RoundArgs)]),
     "ddtree_status_string": (ctypes.c_char_p, [_i]),
     "ddtree_device_status": (_i, [_vp, ctypes.POINTER(ctypes.c_uint)]),
     "ddtree_version": (_i, []),
@@ -379,6 +380,15 @@ def ddtree_round(rb: RoundBuffers, args: Optional[RoundArgs] = None):
     a = rb.args() if args is None else args
     _check(lib().ddtree_round(ctypes.byref(a), _stream()), "ddtree_round")
     return rb
+
+
+def ddtree_round_launch_count(rb: RoundBuffers, args: Optional[RoundArgs] = None) -> int:
+    """Kernel launches one ddtree_round call makes with these buffers."""
+    a = rb.args() if args is None else args
+    n = lib().ddtree_round_launch_count(ctypes.byref(a))
+    if n < 0:
+        raise DDTreeError("invalid round geometry")
+    return n
 
 
 def default_scale(D: int) -> float:

@@ -11,11 +11,12 @@
 // wave of resident 256-thread CTAs; every thread keeps its running best
 // (value, lowest index) over batches of 16-byte loads.  Each CTA reduces its
 // chunk to one 64-bit composite (order key of the logit, then the
-// complemented token id, so lower ids win ties), merges it with atomicMax
-// into the row's workspace slot, and the last CTA of the row (atomic ticket)
-// publishes the argmax and resets the slot.  When the walk is fused, the
-// CTA that publishes a request's last live row runs that request's walk and
-// compaction itself (nobody waits: a second ticket counts published rows).
+// complemented token id, so lower ids win ties) and merges it with atomicMax
+// into the row's workspace slot.  One ticket per request counts its finished
+// CTAs; the last one (nobody waits) reads every live row's slot, publishes
+// the argmax and resets the slot, and when the walk is fused it loads the
+// tree in the same round of loads and runs the request's walk and
+// compaction itself.
 // Kernel 2 (walk + compaction, for caches with many layers): one CTA per
 // (request, layer, K/V).
 // The walk: node j is the accepted child of its parent iff its token equals
@@ -41,25 +42,22 @@ constexpr int WALK_FUSE_MAX_LAYERS = 2;   // compaction by the argmax kernel up 
 constexpr int WALK_MAX_N = 1025;   // B + 1 <= 1025
 
 struct ArgmaxWs {
-  unsigned long long* best;  // [rows]
-  uint32_t* ticket;          // [rows] chunks finished
+  unsigned long long* best;  // [rows] running composite maximum
   int32_t* argmax;           // [rows]
-  uint32_t* req_done;        // [n_req] rows published
+  uint32_t* req_ticket;      // [n_req] CTAs finished
 };
 
 inline size_t argmax_ws_bytes(int rows, int n_req) {
-  return align256((size_t)rows * 8) + 2 * align256((size_t)rows * 4) + align256((size_t)n_req * 4);
+  return align256((size_t)rows * 8) + align256((size_t)rows * 4) + align256((size_t)n_req * 4);
 }
 inline ArgmaxWs argmax_ws_carve(void* ws, int rows) {
   char* b = (char*)ws;
   ArgmaxWs w;
   w.best = (unsigned long long*)b;
   b += align256((size_t)rows * 8);
-  w.ticket = (uint32_t*)b;
-  b += align256((size_t)rows * 4);
   w.argmax = (int32_t*)b;
   b += align256((size_t)rows * 4);
-  w.req_done = (uint32_t*)b;
+  w.req_ticket = (uint32_t*)b;
   return w;
 }
 
@@ -88,28 +86,40 @@ struct WalkArgs {
 
 struct WalkSmem {
   int* nxt;     // [n]
-  int* targ;    // [n]
+  int* targ;    // [n] target argmax of every node
+  int* par;     // [n] parent
+  int* tok;     // [n] token
   int* path;    // [33]
   int* k;
   int* ok;
 };
 
+// Request r's tree (parent, token of every node slot) and target argmax in
+// shared memory, all with one round of loads; next[] cleared.
+__device__ __forceinline__ void walk_load(const WalkArgs& a, int r, const WalkSmem& ws) {
+  const size_t ro = (size_t)r * a.n;
+  for (int i = threadIdx.x; i < a.n; i += blockDim.x) {
+    const int p = __ldcg(a.parent + ro + i);
+    const int t = __ldcg(a.node_token + ro + i);
+    const int g = __ldcg(a.argmax_ws + ro + i);
+    ws.par[i] = p;
+    ws.tok[i] = t;
+    ws.targ[i] = g;
+    ws.nxt[i] = -1;
+  }
+}
+
 // Walk of request r, then compaction of its (layer, K/V) pairs lk0..lk1-1
 // (lk = layer * 2 + (0: K, 1: V)); the pair lk == 0 also writes the walk's
 // outputs.  All threads of the CTA call it.
-__device__ void walk_request(const WalkArgs& a, int r, int lk0, int lk1, const WalkSmem& ws) {
+// The tree and argmax are in `ws` (walk_load, or the argmax kernel's last
+// CTA), followed by a barrier; nn live nodes, committed prefix P.
+__device__ void walk_request(const WalkArgs& a, int r, int nn, int P, int lk0, int lk1, const WalkSmem& ws) {
   const int tid = threadIdx.x, nth = blockDim.x;
-  const int nn = min(a.n_nodes[r], a.n);
-  const int P = a.prefix_len[r];
   const size_t ro = (size_t)r * a.n;
-  for (int i = tid; i < nn; i += nth) {
-    ws.nxt[i] = -1;
-    ws.targ[i] = __ldcg(a.argmax_ws + ro + i);
-  }
-  __syncthreads();
   for (int j = 1 + tid; j < nn; j += nth) {
-    const int p = a.parent[ro + j];
-    if (p >= 0 && p < j && a.node_token[ro + j] == ws.targ[p]) ws.nxt[p] = j;
+    const int p = ws.par[j];
+    if (p >= 0 && p < j && ws.tok[j] == ws.targ[p]) ws.nxt[p] = j;
   }
   __syncthreads();
   if (tid == 0) {
@@ -206,9 +216,11 @@ argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_strid
               const int32_t* __restrict__ n_nodes, int cpr, int chunk, ArgmaxWs ws, WalkArgs wa, int fuse_walk) {
   constexpr int EPV = (DT == DDTREE_BF16) ? 8 : 4;
   __shared__ unsigned long long red[ARGMAX_THREADS / 32];
-  __shared__ int s_walk;
+  __shared__ int s_last;
   __shared__ int s_nxt[WALK_MAX_N];
   __shared__ int s_targ[WALK_MAX_N];
+  __shared__ int s_par[WALK_MAX_N];
+  __shared__ int s_tok[WALK_MAX_N];
   __shared__ int s_path[33];
   __shared__ int s_k, s_ok;
   const int tid = threadIdx.x;
@@ -286,38 +298,53 @@ argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_strid
     for (int i = 1; i < ARGMAX_THREADS / 32; ++i) b = red[i] > b ? red[i] : b;
     atomicMax(&ws.best[row], b);
     __threadfence();
-    int walk = 0;
-    const unsigned t = atomicAdd(&ws.ticket[row], 1u);
-    if (t == (unsigned)(cpr - 1)) {
-      __threadfence();
-      const unsigned long long fin = atomicExch(&ws.best[row], 0ull);   // read and reset
-      ws.argmax[row] = (int32_t)(TOPK_ID_MASK - (uint32_t)(fin & TOPK_ID_MASK));
-      ws.ticket[row] = 0;
-      if (fuse_walk) {
-        __threadfence();
-        const unsigned d = atomicAdd(&ws.req_done[req], 1u);
-        if (d == (unsigned)(live - 1)) {
-          ws.req_done[req] = 0;
-          __threadfence();
-          walk = 1;
-        }
-      }
-    }
-    s_walk = walk;
+    const unsigned t = atomicAdd(&ws.req_ticket[req], 1u);
+    s_last = (t == (unsigned)(live * cpr - 1));
   }
   __syncthreads();
-  if (s_walk) {
-    const WalkSmem sm{s_nxt, s_targ, s_path, &s_k, &s_ok};
-    walk_request(wa, req, 0, wa.k_cache ? 2 * wa.layers : 1, sm);
+  if (!s_last) return;
+  __threadfence();
+  // The request's last CTA: every live row's argmax (read and reset) and,
+  // for the fused walk, the tree, in one round of loads.
+  const size_t ro = (size_t)req * n;
+  const int P = fuse_walk ? wa.prefix_len[req] : 0;
+  for (int i = tid; i < n; i += ARGMAX_THREADS) {
+    unsigned long long fin = 0ull;
+    int p = -1, tk = -1;
+    if (i < live) fin = __ldcg(&ws.best[ro + i]);
+    if (fuse_walk) {
+      p = __ldcg(wa.parent + ro + i);
+      tk = __ldcg(wa.node_token + ro + i);
+    }
+    if (i < live) {
+      const int32_t am = (int32_t)(TOPK_ID_MASK - (uint32_t)(fin & TOPK_ID_MASK));
+      ws.best[ro + i] = 0ull;
+      ws.argmax[ro + i] = am;
+      s_targ[i] = am;
+    }
+    s_par[i] = p;
+    s_tok[i] = tk;
+    s_nxt[i] = -1;
   }
+  if (tid == 0) ws.req_ticket[req] = 0;   // ready for the next call
+  if (!fuse_walk) return;
+  __syncthreads();
+  const WalkSmem sm{s_nxt, s_targ, s_par, s_tok, s_path, &s_k, &s_ok};
+  walk_request(wa, req, live, P, 0, wa.k_cache ? 2 * wa.layers : 1, sm);
 }
 
 __global__ void __launch_bounds__(WALK_THREADS) walk_compact_kernel(WalkArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(16) unsigned char smem_raw[];   // [4][n] ints
   __shared__ int s_path[33];
   __shared__ int s_k, s_ok;
-  const WalkSmem sm{(int*)smem_raw, (int*)smem_raw + a.n, s_path, &s_k, &s_ok};
-  walk_request(a, blockIdx.x, blockIdx.y, blockIdx.y + 1, sm);
+  int* sw = (int*)smem_raw;
+  const WalkSmem sm{sw, sw + a.n, sw + 2 * a.n, sw + 3 * a.n, s_path, &s_k, &s_ok};
+  const int r = blockIdx.x;
+  const int nn = min(a.n_nodes[r], a.n);
+  const int P = a.prefix_len[r];
+  walk_load(a, r, sm);
+  __syncthreads();
+  walk_request(a, r, nn, P, blockIdx.y, blockIdx.y + 1, sm);
 }
 
 }  // namespace ddt

@@ -349,7 +349,7 @@ int accept_launch(const void* target_logits, int dtype, int V, long long row_str
                                                                        p.cpr, p.chunk, w, a, fuse);
   int st = launch_status();
   if (st || fuse) return st;
-  const size_t smem = (size_t)n * 8;
+  const size_t smem = (size_t)n * 16;   // next, argmax, parent, token
   dim3 grid2(n_req, a.layers * 2);
   walk_compact_kernel<<<grid2, WALK_THREADS, smem, s>>>(a);
   return launch_status();
@@ -422,6 +422,16 @@ static size_t round_parts(const ddtree_round_args* a, size_t* off_attn, size_t* 
 size_t ddtree_round_workspace_bytes(const ddtree_round_args* a) {
   if (!a || a->n_req < 1 || a->L < 1 || a->V < 1 || a->K < 1 || a->B < 0 || kv_check(&a->kv)) return 0;
   return round_parts(a, nullptr, nullptr);
+}
+
+int ddtree_round_launch_count(const ddtree_round_args* a) {
+  if (!a || a->n_req < 1 || a->L < 1 || a->V < 1 || a->K < 1 || a->B < 0 || kv_check(&a->kv)) return -1;
+  int n = 2;                                                             // top-K, build
+  n += 1;                                                                // attention
+  if (use_tc_attn(a->dtype, &a->kv) && tc_attn_ws_bytes(geom_of(&a->kv, a->B), num_sms()) > 0) n += 1;   // combine
+  n += 1;                                                                // argmax (+ walk)
+  if (a->kv.layers > WALK_FUSE_MAX_LAYERS) n += 1;                       // walk and compaction
+  return n;
 }
 
 int ddtree_round(const ddtree_round_args* a, cudaStream_t stream) {

@@ -247,12 +247,20 @@ typedef struct {
   void* ws; size_t ws_bytes;
 } ddtree_round_args;
 
+/* Bytes of a->ws the round needs (0 for an invalid geometry).  The
+ * workspace holds the stages' counters and tickets: it must be zero-filled
+ * before its first use, and every call leaves them at zero again. */
 size_t ddtree_round_workspace_bytes(const ddtree_round_args* a);
 
 /* Stage order topk -> build -> tree_attn -> accept on `stream`; ids, lp,
  * node_token, parent, depth, anc, n_nodes and new_prefix_len are required,
  * the other outputs may be NULL. */
 int ddtree_round(const ddtree_round_args* a, cudaStream_t stream);
+
+/* Number of kernel launches one ddtree_round call with these arguments
+ * makes on the current device (the one-time exp table build excluded), or
+ * -1 for an invalid geometry.  Host only: no device work. */
+int ddtree_round_launch_count(const ddtree_round_args* a);
 
 /* ---------------------------------------------------------------------- */
 /* Top-K without a caller workspace (no counterpart in the paper: an      */

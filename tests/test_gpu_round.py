@@ -106,6 +106,44 @@ def test_round_batched_paged_sampled():
     check_round(w, rb, h, nodes=[0, 3, 64], heads=[0, 31])
 
 
+@pytest.mark.parametrize("cfg,over", [
+    (1, dict(N=3)),                      # 12 rows of 512 logits: one chunk per row
+    (2, dict(N=2, V=32768)),             # 32 rows, 4 chunks each: 128 CTAs
+    (2, dict(N=2, V=32768, B=0)),        # root-only trees
+])
+def test_round_multi_request(cfg, over):
+    """Several requests in one round, each with exactly its own tree, and a
+    second round on the same workspace (tickets back at zero) repeats it."""
+    w = datagen.workload(cfg, **over)
+    rb, h = make_round(w)
+    args = rb.args()
+    k0, v0 = rb.k_cache.clone(), rb.v_cache.clone()
+    dd.ddtree_round(rb, args)
+    torch.cuda.synchronize()
+    check_round(w, rb, h, nodes=sorted({0, min(1, w.B), w.B // 2, w.B}), heads=[0, w.Hq - 1])
+    # the per-request tickets are back at zero: a second round builds the same trees
+    first = [x.clone() for x in (rb.tree.parent, rb.tree.anc, rb.tree.n_nodes, rb.acc.path)]
+    rb.k_cache.copy_(k0)
+    rb.v_cache.copy_(v0)
+    dd.ddtree_round(rb, args)
+    torch.cuda.synchronize()
+    assert dd.device_status() == 0
+    for a, b in zip(first, (rb.tree.parent, rb.tree.anc, rb.tree.n_nodes, rb.acc.path)):
+        assert torch.equal(a, b)
+
+
+def test_round_launch_count():
+    """The launch plan the round reports: top-K, build, attention (+ the
+    combine when b64_p2k splits its key range), argmax (+ a separate walk
+    and compaction launch above two cache layers)."""
+    rb2, _ = make_round(datagen.workload(2))
+    assert dd.ddtree_round_launch_count(rb2) == 5
+    rb1, _ = make_round(datagen.workload(1))
+    assert dd.ddtree_round_launch_count(rb1) == 4
+    rb1l, _ = make_round(datagen.workload(1, layers=3))
+    assert dd.ddtree_round_launch_count(rb1l) == 5
+
+
 def test_round_repeats_are_identical():
     w = datagen.workload(2)
     rb, h = make_round(w)

@@ -212,6 +212,7 @@ struct TcParams {
   float* out_lse;
   float* ws_o;         // [units*splits][128][128] partial O (splits > 1)
   float2* ws_ml;       // [units*splits][128] (max in log2 units, sum)
+  int lpt;             // 1: requests taken longest key range first (unsplit only)
 };
 
 template <int BN>
@@ -226,6 +227,7 @@ struct TcSmem {
   uint32_t tmem_base;
   int abort;
   int blk[2];
+  int lpt_r;
 };
 
 // Two CTAs share an SM, so there is no room for alignment slack: the
@@ -258,8 +260,25 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const int unit = u;
   const int mt = u % p.mtiles; u /= p.mtiles;
   const int kvh = u % g.Hkv; u /= g.Hkv;
-  const int r = u % g.n_req; u /= g.n_req;
+  int r = u % g.n_req; u /= g.n_req;
   const int layer = u;
+  if (p.lpt) {
+    // Ragged batch: request slot r takes the request of rank r in the order
+    // of key count (prefix + nodes) descending, ties by index, so the
+    // longest units are dispatched first and the last wave holds short ones.
+    const int r_slot = r;
+    for (int i = tid; i < g.n_req; i += TC_THREADS) {
+      const int ki = p.prefix_len[i] + p.n_nodes[i];
+      int rank = 0;
+      for (int j = 0; j < g.n_req; ++j) {
+        const int kj = p.prefix_len[j] + p.n_nodes[j];
+        rank += (kj > ki) || (kj == ki && j < i);
+      }
+      if (rank == r_slot) sm.lpt_r = i;
+    }
+    __syncthreads();
+    r = sm.lpt_r;
+  }
   const int nodes_per_tile = TC_BM / p.G;
   const int node0 = mt * nodes_per_tile;
   const int nn = p.n_nodes[r];
@@ -599,6 +618,7 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 // row-innermost, so every load is a coalesced run over the rows; each thread
 // requests all splits' data before combining.
 constexpr int TC_MAX_SPLITS = 16;
+constexpr int TC_LPT_MAX_REQ = 128;   // longest-first request order up to this batch (each CTA ranks them all)
 
 template <int S>   // capacity for the number of splits (>= p.splits)
 __global__ void __launch_bounds__(128)
@@ -761,6 +781,7 @@ inline int tc_attn_launch(const void* q, const void* kc, const void* vc, const i
   p.out_lse = out_lse;
   p.ws_o = nullptr;
   p.ws_ml = nullptr;
+  p.lpt = (pl.splits == 1 && g.n_req > 1 && g.n_req <= TC_LPT_MAX_REQ) ? 1 : 0;
   if (pl.splits > 1) {
     const size_t slots = (size_t)pl.units * pl.splits;
     p.ws_o = (float*)ws;

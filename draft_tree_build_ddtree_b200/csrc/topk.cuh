@@ -42,7 +42,7 @@ constexpr int TOPK_THREADS = 512;
 constexpr int TOPK_MAX_VPT = 6;            // 16-byte vectors per thread
 constexpr int TOPK_MAX_CAND = 16384;       // merge capacity (candidates per row)
 constexpr int TOPK_MAX_CPR = 128;          // chunks per row
-constexpr int TOPK_EXP_WARPS = 6;          // warps of a CTA that sum exp while the others select (4, 8, 10, 12 measured slower)
+constexpr int TOPK_EXP_WARPS = 6;          // warps of a CTA that sum exp while the others select (4, 5, 7, 8, 10, 12 measured slower)
 constexpr int TOPK_LIST_CAP = 4096;        // bf16 candidate list entries per chunk
 constexpr int TOPK_MERGE_SMALL = 512;      // merge ranks by counting up to this many keys >= the K-th value
 constexpr int TOPK_ID_BITS = 20;           // V <= 2^20

@@ -87,3 +87,26 @@ def test_cpu_tensors_are_refused():
     import torch
     with pytest.raises(dd.DDTreeError):
         dd.ddtree_topk(torch.zeros(2, 64), 4)
+
+
+def test_round_launch_count_is_host_only(lib):
+    """The round's launch plan is computed on the host from sizes alone (no
+    pointer is read): top-K, build, attention (+ combine when the key range
+    is split), argmax (+ walk launch above two cache layers)."""
+    def args(layers, P, dtype=0, n_req=1, B=64, D=128):
+        a = dd.RoundArgs()
+        a.n_req, a.L, a.V, a.K, a.B = n_req, 16, 151936, 64, B
+        a.dtype = dtype
+        a.kv = dd.kv_desc(layers, n_req, 32, 4, D, s_max=(P + B + 1 + 63) // 64 * 64)
+        return a
+
+    def count(a):
+        return lib.ddtree_round_launch_count(ctypes.byref(a))
+
+    # without a device the library plans for 148 SMs; these plans hold for any B200
+    assert count(args(1, 2048)) == 5            # b64_p2k: 20 units split over the SMs -> combine
+    assert count(args(48, 8192, B=256)) == 5    # 3264 units fill the GPU (no combine); 48 layers -> walk launch
+    assert count(args(1, 2048, dtype=1)) == 4   # fp32: SIMT attention, no split
+    bad = args(1, 2048)
+    bad.n_req = 0
+    assert count(bad) == -1

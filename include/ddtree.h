@@ -274,7 +274,7 @@ int ddtree_round_launch_count(const ddtree_round_args* a);
  * It is meant for callers that cannot allocate device memory while they
  * run rounds: serving engines that hand all free device memory to their KV
  * cache pool at start-up, where a cudaMalloc at decode time can synchronize
- * the device or fail because the pool already holds the memory.
+ * the device or fail because that pool already holds the memory.
  *
  * Limits and behaviour:
  *  - The built-in scratch is 4 MiB per device (allocated when the library is

@@ -192,6 +192,13 @@ def workload_from_args(a):
     return datagen.workload(a.config)
 
 
+def workload_label(w) -> str:
+    """The workload's name and sizes, as both arms report it."""
+    return (f"{w.name}: L={w.L} V={w.V} K={w.K} B={w.B} Hq={w.Hq} Hkv={w.Hkv} "
+            f"D={w.D} P={w.P or f'U[{w.P_lo},{w.P_hi}]'} layers={w.layers} "
+            f"n_req={w.N}{' paged' if w.paged else ''}")
+
+
 def set_bytes(w) -> int:
     es = 2 if w.dtype == "bf16" else 4
     prefix = datagen.prefix_lengths(w)
@@ -451,9 +458,7 @@ def run_ours(a):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms_max / a.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": f"{w.name}: L={w.L} V={w.V} K={w.K} B={w.B} Hq={w.Hq} Hkv={w.Hkv} "
-                                   f"D={w.D} P={w.P or f'U[{w.P_lo},{w.P_hi}]'} layers={w.layers} "
-                                   f"n_req={w.N}{' paged' if w.paged else ''}",
+            "config": {"workload": workload_label(w),
                        "config_id": w.cfg, "n_req": w.N, "parallelism": f"replicas x{world}",
                        "l2": f"{R} rotating input sets of {per_set / 1e6:.1f} MB (> 2x L2)",
                        "launch": "cuda graph per round" if use_graph else "eager"},
@@ -588,7 +593,7 @@ def run_reference(a):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": total / a.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": w.name, "config_id": w.cfg, "n_req": w.N},
+            "data": "synthetic", "config": {"workload": workload_label(w), "config_id": w.cfg, "n_req": w.N},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": f"each step: {desc}; numpy/BLAS limited to 1 thread"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

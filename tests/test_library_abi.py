@@ -110,3 +110,37 @@ def test_round_launch_count_is_host_only(lib):
     bad = args(1, 2048)
     bad.n_req = 0
     assert count(bad) == -1
+
+
+def _align256(x):
+    return (x + 255) // 256 * 256
+
+
+def test_launch_plans_from_sizes(lib):
+    """The host-side plans (148 SMs without a device) behind the workspace
+    sizes: b64_p2k top-K cuts each of its 16 bf16 rows into 9 chunks (one
+    wave of 144 CTAs) with K + K candidate slots each; the b64_p2k attention splits
+    its 20 units (4 KV heads x 5 M-tiles) 7 ways over 128-key tiles; the
+    48-layer and 32-request workloads fill the GPU unsplit."""
+    rows, V, K = 16, 151936, 64
+    cap = 2 * K
+
+    def topk_ws(cpr):
+        return (_align256(rows * 4) + _align256(rows * cpr * 16) + 2 * _align256(rows * cpr * 4)
+                + _align256(rows * cpr * cap * 8))
+    # the query covers either dtype: bf16 rows take 9 chunks (one wave of
+    # 144 CTAs); fp32 rows need 13 (at most 6 x 512 x 16 bytes staged per CTA)
+    assert lib.ddtree_topk_workspace_bytes(rows, V, K) == max(topk_ws(9), topk_ws(13)) == topk_ws(13)
+
+    kv2 = dd.kv_desc(1, 1, 32, 4, 128, s_max=2176)
+    slots = 20 * 7
+    assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv2), 64) == \
+        _align256(slots * 128 * 128 * 4) + _align256(slots * 128 * 8)
+    kv3 = dd.kv_desc(48, 1, 32, 4, 128, s_max=8512)
+    assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv3), 256) == 0
+    kv4 = dd.kv_desc(1, 32, 32, 4, 128, paged=True, num_blocks=4096, max_blocks=258)
+    assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv4), 64) == 0
+    # accept: composite slots, argmax, one ticket per request
+    n = 65
+    assert lib.ddtree_accept_workspace_bytes(32, 64, V) == \
+        _align256(32 * n * 8) + _align256(32 * n * 4) + _align256(32 * 4)

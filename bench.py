@@ -65,7 +65,7 @@ def parse():
 CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "draft_tree_build_ddtree_b200", "csrc")
 TRAFFIC = {
     ("b64_p2k", "topk"): (5069568, ("topk.cuh", "common.cuh", "exp64_table.h"), "4c480e2f4cca5119"),
-    ("b256_p8k_48l", "attn"): (1057939712, ("attn_tc.cuh", "attn_simt.cuh", "common.cuh"), "ac35819ac895c730"),
+    ("b256_p8k_48l", "attn"): (1057939712, ("attn_tc.cuh", "attn_simt.cuh", "common.cuh"), "673c3d78fa774a8f"),
 }
 
 

@@ -12,7 +12,7 @@
 // loads in one box from q[layer][req][node][head][D].  One CTA handles one
 // (layer, request, KV head, M-tile, key split).
 //
-// Per 128-key tile:  S = Q K^T (tcgen05.mma kind::f16, A and B K-major from
+// Per key tile (64 or 128 keys, TcCfg):  S = Q K^T (tcgen05.mma kind::f16, A and B K-major from
 // 128B-swizzled shared memory, fp32 accumulator in TMEM), then the softmax
 // warps read S from TMEM (one thread per row = TMEM lane), apply the
 // ancestor mask only on tiles that reach the tree slots, update the running
@@ -32,6 +32,8 @@
 //
 // When the key range is split across CTAs, each split writes its unnormalised
 // O, running max and sum to the workspace and a combine kernel merges them.
+// Unsplit launches over a ragged batch take the requests longest key range
+// first, so the longest units start in the first wave.
 #pragma once
 
 #include <cuda.h>

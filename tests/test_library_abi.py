@@ -144,3 +144,11 @@ def test_launch_plans_from_sizes(lib):
     n = 65
     assert lib.ddtree_accept_workspace_bytes(32, 64, V) == \
         _align256(32 * n * 8) + _align256(32 * n * 4) + _align256(32 * 4)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No CPU fallback: without libddtree.so every call raises."""
+    monkeypatch.setattr(dd, "_LIB_PATH", str(tmp_path / "libddtree.so"))
+    monkeypatch.setattr(dd, "_lib", None)
+    with pytest.raises(dd.DDTreeError):
+        dd.lib()

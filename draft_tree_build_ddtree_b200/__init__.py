@@ -30,7 +30,7 @@ __all__ = [
 ]
 
 BF16, F32 = 0, 1
-STATUS_NONFINITE, STATUS_TIMEOUT, STATUS_CAPACITY = 1, 2, 4
+STATUS_NONFINITE, STATUS_TIMEOUT, STATUS_CAPACITY, STATUS_SETUP = 1, 2, 4, 8
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libddtree.so")
 _lib = None
 
@@ -63,13 +63,16 @@ class RoundArgs(ctypes.Structure):
                 ("target_argmax", _vp), ("path", _vp), ("accept_len", _vp),
                 ("next_bonus", _vp), ("src_slot", _vp), ("dst_slot", _vp),
                 ("new_prefix_len", _vp),
-                ("ws", _vp), ("ws_bytes", _sz)]
+                ("ws", _vp), ("ws_bytes", _sz),
+                ("gain_floor", _vp)]
 
 
 _SIGS = {
     "ddtree_topk_workspace_bytes": (_sz, [_i, _i, _i]),
     "ddtree_topk": (_i, [_vp, _i, _i, _i, _ll, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "ddtree_build": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "ddtree_build_ex": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i,
+                             _vp, _vp]),
     "ddtree_attn_workspace_bytes": (_sz, [ctypes.POINTER(KVDesc), _i]),
     "ddtree_tree_attn": (_i, [_vp, _vp, _vp, _i, ctypes.POINTER(KVDesc), _vp, _vp, _vp, _vp, _i,
                               _vp, _vp, _vp, _sz, _vp]),
@@ -83,6 +86,7 @@ _SIGS = {
     "ddtree_device_status": (_i, [_vp, ctypes.POINTER(ctypes.c_uint)]),
     "ddtree_version": (_i, []),
     "ddtree_topk_static_ws": (_i, [_vp, _i, _i, _i, _ll, _i, _vp, _vp, _vp, _vp]),
+    "ddtree_debug_attn_timeout": (_i, [ctypes.c_ulonglong, _i]),
 }
 
 
@@ -205,17 +209,40 @@ def alloc_tree(n_req: int, B: int, device) -> Tree:
                 torch.empty((n_req, n, W), **i32), torch.empty((n_req,), **i32))
 
 
+BUILD_FORCE_HEAP = 0x1
+BUILD_PATH_NAMES = {0: "enumeration", 1: "heap_registers_3", 2: "heap_registers_9", 3: "heap_tournament"}
+
+
 def ddtree_build(ids: torch.Tensor, lp: torch.Tensor, root_token: torch.Tensor, B: int,
-                 out: Optional[Tree] = None) -> Tree:
-    """Best-first tree of ``B`` nodes per request from [n_req, L, K] top-K tables."""
+                 out: Optional[Tree] = None, gain_floor: Optional[torch.Tensor] = None,
+                 flags: int = 0, build_path: Optional[torch.Tensor] = None) -> Tree:
+    """Best-first tree of ``B`` nodes per request from [n_req, L, K] top-K tables.
+
+    ``gain_floor`` (float32 [n_req], optional): adaptive budget, keep only the
+    pops whose score exceeds it.  ``flags`` / ``build_path``: see
+    ddtree_build_ex in include/ddtree.h.
+    """
     for t, nm in ((ids, "ids"), (lp, "lp"), (root_token, "root_token")):
         _contig(t, nm)
     n_req, L, K = ids.shape
     t = alloc_tree(n_req, B, ids.device) if out is None else out
-    _check(lib().ddtree_build(_ptr(ids), _ptr(lp), _ptr(root_token), n_req, L, K, B,
-                              _ptr(t.node_token), _ptr(t.parent), _ptr(t.depth), _ptr(t.node_rank),
-                              _ptr(t.score), _ptr(t.anc), _ptr(t.n_nodes), _stream()),
-           "ddtree_build")
+    if gain_floor is None and flags == 0 and build_path is None:
+        _check(lib().ddtree_build(_ptr(ids), _ptr(lp), _ptr(root_token), n_req, L, K, B,
+                                  _ptr(t.node_token), _ptr(t.parent), _ptr(t.depth), _ptr(t.node_rank),
+                                  _ptr(t.score), _ptr(t.anc), _ptr(t.n_nodes), _stream()),
+               "ddtree_build")
+        return t
+    if gain_floor is not None:
+        _contig(gain_floor, "gain_floor")
+        if gain_floor.dtype != torch.float32 or gain_floor.numel() != n_req:
+            raise DDTreeError("gain_floor must be float32 [n_req]")
+    if build_path is not None:
+        _contig(build_path, "build_path")
+    _check(lib().ddtree_build_ex(_ptr(ids), _ptr(lp), _ptr(root_token), n_req, L, K, B,
+                                 _ptr(t.node_token), _ptr(t.parent), _ptr(t.depth), _ptr(t.node_rank),
+                                 _ptr(t.score), _ptr(t.anc), _ptr(t.n_nodes), _ptr(gain_floor), int(flags),
+                                 _ptr(build_path), _stream()),
+           "ddtree_build_ex")
     return t
 
 
@@ -328,6 +355,7 @@ class RoundBuffers:
     attn_lse: torch.Tensor = None
     acc: Accept = None
     ws: torch.Tensor = None
+    gain_floor: Optional[torch.Tensor] = None   # float32 [n_req]: adaptive-budget floor of the build
     _args: RoundArgs = None
 
     def allocate_outputs(self):
@@ -365,6 +393,7 @@ class RoundBuffers:
         a.target_argmax, a.path, a.accept_len = _ptr(c.target_argmax), _ptr(c.path), _ptr(c.accept_len)
         a.next_bonus, a.src_slot, a.dst_slot = _ptr(c.next_bonus), _ptr(c.src_slot), _ptr(c.dst_slot)
         a.new_prefix_len = _ptr(c.new_prefix_len)
+        a.gain_floor = _ptr(self.gain_floor)
         need = lib().ddtree_round_workspace_bytes(ctypes.byref(a))
         if need == 0:
             raise DDTreeError("invalid round geometry")

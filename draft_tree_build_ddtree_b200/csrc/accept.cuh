@@ -317,7 +317,8 @@ argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_strid
       tk = __ldcg(wa.node_token + ro + i);
     }
     if (i < live) {
-      const int32_t am = (int32_t)(TOPK_ID_MASK - (uint32_t)(fin & TOPK_ID_MASK));
+      // fin == 0: every logit of the row was NaN (flagged); -1 matches no token
+      const int32_t am = fin == 0ull ? -1 : (int32_t)(TOPK_ID_MASK - (uint32_t)(fin & TOPK_ID_MASK));
       ws.best[ro + i] = 0ull;
       ws.argmax[ro + i] = am;
       s_targ[i] = am;

@@ -26,7 +26,7 @@
 // Warp roles (192 threads): warps 0-3 softmax + epilogue (warp w reads TMEM
 // lanes 32w..32w+31), warp 4 the TMA producer, warp 5 TMEM allocation and
 // the single-thread MMA issue.  Every mbarrier wait is bounded (about one
-// second); on timeout the kernel sets DDTREE_STATUS_TIMEOUT, every role
+// second by default); on timeout the kernel sets DDTREE_STATUS_TIMEOUT, every role
 // leaves its loop, waits (bounded) for its copies and MMAs in flight, and
 // the TMEM is freed before exit.  No TMA multicast is used.
 //
@@ -99,15 +99,16 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 
 constexpr uint64_t TC_WAIT_NS = 1000000000ull;   // one second
 
-// Bounded wait for the phase of parity `parity`; false on timeout or when
-// another role already gave up (*abort set).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// Bounded wait for the phase of parity `parity`; false on timeout (after
+// limit_ns) or when another role already gave up (*abort set).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = TC_WAIT_NS) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
     if (mbar_test(bar, parity)) return true;
     if (*abort) return false;
-    if (global_ns() - t0 > TC_WAIT_NS) {
+    if (global_ns() - t0 > limit_ns) {
       *abort = 1;
       flag_status(DDTREE_STATUS_TIMEOUT);
       return false;
@@ -215,6 +216,8 @@ struct TcParams {
   float* ws_o;         // [units*splits][128][128] partial O (splits > 1)
   float2* ws_ml;       // [units*splits][128] (max in log2 units, sum)
   int lpt;             // 1: requests taken longest key range first (unsplit only)
+  uint64_t wait_ns;    // limit of the pipeline's bounded waits
+  int stop_tile;       // >= 0: the producer issues no key tile from this one on (timeout-path diagnostics)
 };
 
 template <int BN>
@@ -249,7 +252,7 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   constexpr int TC_KTILE = TcCfg<BN>::KTILE;
   TcSmem<BN>& sm = *reinterpret_cast<TcSmem<BN>*>(smem_dyn);
   if ((smem_u32(smem_dyn) & 1023u) != 0u) {       // the 128B-swizzled tiles need 1024-byte alignment
-    if (threadIdx.x == 0) flag_status(DDTREE_STATUS_TIMEOUT);
+    if (threadIdx.x == 0) flag_status(DDTREE_STATUS_SETUP);
     return;
   }
   const AttnGeom& g = p.g;
@@ -348,6 +351,7 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       tma_load_4d(smem_u32(sm.q + TC_ATOM), &tm_q, &sm.bar_q, 64, kvh * p.G, node0, qb);
       int issued = 0;
       for (int jj = 0; jj < nt; ++jj) {
+        if (jj == p.stop_tile) break;      // diagnostics: withhold the rest, a consumer wait runs out
         const int j = t_begin + jj;
         const int st = jj % TC_STAGES;
         const int use = jj / TC_STAGES;
@@ -376,15 +380,15 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           }
         };
         // K tile
-        if (use > 0 && !mbar_wait(&sm.bar_ke[st], (use - 1) & 1, abort)) break;
+        if (use > 0 && !mbar_wait(&sm.bar_ke[st], (use - 1) & 1, abort, p.wait_ns)) break;
         load_tile(&tm_k, sm.k[st], &sm.bar_kf[st]);
         // V tile
-        if (use > 0 && !mbar_wait(&sm.bar_ve[st], (use - 1) & 1, abort)) break;
+        if (use > 0 && !mbar_wait(&sm.bar_ve[st], (use - 1) & 1, abort, p.wait_ns)) break;
         load_tile(&tm_v, sm.v[st], &sm.bar_vf[st]);
         issued = jj + 1;
       }
       // copies in flight must land before the CTA exits
-      if (*abort) {
+      if (*abort || issued < nt) {
         mbar_wait(&sm.bar_q, 0, abort);
         for (int jj = max(0, issued - TC_STAGES); jj < issued; ++jj) {
           int z = 0;
@@ -399,13 +403,13 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(TC_BM, TC_BN, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(TC_BM, TC_D, false, true);
       const uint32_t q_addr = smem_u32(sm.q), p_addr = smem_u32(sm.p);
-      bool ok = mbar_wait(&sm.bar_q, 0, abort);
-      int committed_pv = 0;
+      bool ok = mbar_wait(&sm.bar_q, 0, abort, p.wait_ns);
+      int committed_pv = 0, committed_qk = 0;
       for (int jj = 0; ok && jj <= nt; ++jj) {
         if (jj < nt) {
           const int st = jj % TC_STAGES;
-          if (!mbar_wait(&sm.bar_kf[st], (jj / TC_STAGES) & 1, abort)) break;
-          if (jj > 0 && !mbar_wait(&sm.bar_sfree, (jj - 1) & 1, abort)) break;
+          if (!mbar_wait(&sm.bar_kf[st], (jj / TC_STAGES) & 1, abort, p.wait_ns)) break;
+          if (jj > 0 && !mbar_wait(&sm.bar_sfree, (jj - 1) & 1, abort, p.wait_ns)) break;
           tc_fence_after();
           const uint32_t k_addr = smem_u32(sm.k[st]);
 #pragma unroll
@@ -417,12 +421,13 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           }
           umma_commit(&sm.bar_sfull);
           umma_commit(&sm.bar_ke[st]);
+          committed_qk = jj + 1;
         }
         if (jj > 0) {
           const int pj = jj - 1;
           const int st = pj % TC_STAGES;
-          if (!mbar_wait(&sm.bar_pfull, pj & 1, abort)) break;
-          if (!mbar_wait(&sm.bar_vf[st], (pj / TC_STAGES) & 1, abort)) break;
+          if (!mbar_wait(&sm.bar_pfull, pj & 1, abort, p.wait_ns)) break;
+          if (!mbar_wait(&sm.bar_vf[st], (pj / TC_STAGES) & 1, abort, p.wait_ns)) break;
           tc_fence_after();
           const uint32_t v_addr = smem_u32(sm.v[st]);
 #pragma unroll
@@ -437,9 +442,10 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
       }
       // MMAs in flight must retire before TMEM is freed
-      if (*abort && committed_pv > 0) {
+      if (*abort) {
         int z = 0;
-        mbar_wait(&sm.bar_pvdone, (committed_pv - 1) & 1, (volatile int*)&z);
+        if (committed_qk > 0) mbar_wait(&sm.bar_sfull, (committed_qk - 1) & 1, (volatile int*)&z);
+        if (committed_pv > 0) mbar_wait(&sm.bar_pvdone, (committed_pv - 1) & 1, (volatile int*)&z);
       }
     }
   } else {
@@ -456,7 +462,7 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int j = t_begin + jj;
       const int k0 = j * TC_BN;
       // tcgen05.ld/st are warp-collective: every exit and branch around them is warp-uniform
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull, jj & 1, abort))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull, jj & 1, abort, p.wait_ns))) { ok = false; break; }
       tc_fence_after();
       float s[TC_BN];
 #pragma unroll
@@ -521,7 +527,7 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
       // P buffer and O are free once the previous PV has retired
       if (jj > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_pvdone, (jj - 1) & 1, abort))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_pvdone, (jj - 1) & 1, abort, p.wait_ns))) { ok = false; break; }
         tc_fence_after();
       }
       if (__any_sync(0xffffffffu, rescale)) {
@@ -556,7 +562,7 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
     // ---- epilogue ----
     bool fin = ok && nt > 0;
-    if (fin) fin = mbar_wait(&sm.bar_pvdone, (nt - 1) & 1, abort);
+    if (fin) fin = mbar_wait(&sm.bar_pvdone, (nt - 1) & 1, abort, p.wait_ns);
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
       const bool live = node < nn;
@@ -767,7 +773,8 @@ inline bool make_map_4d(CUtensorMap* m, const void* base, uint64_t d1, uint64_t 
 
 inline int tc_attn_launch(const void* q, const void* kc, const void* vc, const int32_t* block_table,
                           const int32_t* prefix_len, const uint32_t* anc, const int32_t* n_nodes, const AttnGeom& g,
-                          void* out, float* out_lse, void* ws, int num_sms, cudaStream_t stream) {
+                          void* out, float* out_lse, void* ws, int num_sms, cudaStream_t stream,
+                          uint64_t wait_ns = 0, int stop_tile = -1) {
   TcPlan pl = tc_plan(g, num_sms);
   TcParams p;
   p.g = g;
@@ -784,6 +791,8 @@ inline int tc_attn_launch(const void* q, const void* kc, const void* vc, const i
   p.ws_o = nullptr;
   p.ws_ml = nullptr;
   p.lpt = (pl.splits == 1 && g.n_req > 1 && g.n_req <= TC_LPT_MAX_REQ) ? 1 : 0;
+  p.wait_ns = wait_ns > 0 ? wait_ns : TC_WAIT_NS;
+  p.stop_tile = stop_tile;
   if (pl.splits > 1) {
     const size_t slots = (size_t)pl.units * pl.splits;
     p.ws_o = (float*)ws;

@@ -400,8 +400,10 @@ __device__ __forceinline__ int block_exclusive_scan(int* v, int m, int* warp_tot
 
 // Returns the number of pops, or -1 when the enumeration exceeds ENUM_CAP.
 // Block-uniform.  Fills sm.nd_* for nodes 1..pops.
+// kfloor > 0 raises the score threshold: only prefixes whose score key is
+// at least kfloor are listed (the adaptive budget's floor).
 __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B, int kc, TieCode tc,
-                          uint32_t* hist, int* bcast, int* warp_tot, float* chain, int* s_lev) {
+                          uint32_t* hist, int* bcast, int* warp_tot, float* chain, int* s_lev, uint32_t kfloor) {
   const int tid = threadIdx.x;
   // ---- 1. threshold: B-th best score among the one-deviation chain prefixes ----
   if (tid == 0) {
@@ -466,6 +468,7 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
     t = kmin + ((uint32_t)bcast[1] << shift);
     if (t == 0u) t = 1u;
   }
+  if (kfloor > t) t = kfloor;
   // ---- 2. every prefix with score key >= t, level by level ----
   // depth 1: children of the root
   if (tid == 0) {
@@ -622,9 +625,10 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
 __global__ void __launch_bounds__(BUILD_THREADS, 1)
 build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
              const int32_t* __restrict__ root_token, int L, int K, int B, int kc, TieCode tc, int use_enum,
-             int32_t* __restrict__ node_token, int32_t* __restrict__ parent,
+             const float* __restrict__ gain_floor, int32_t* __restrict__ node_token, int32_t* __restrict__ parent,
              int32_t* __restrict__ depth, int32_t* __restrict__ node_rank,
-             float* __restrict__ score, uint32_t* __restrict__ anc, int32_t* __restrict__ n_nodes) {
+             float* __restrict__ score, uint32_t* __restrict__ anc, int32_t* __restrict__ n_nodes,
+             int32_t* __restrict__ build_path) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int r = blockIdx.x;
   const int tid = threadIdx.x;
@@ -695,19 +699,52 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
     sm.nd_depth[0] = 0;
     sm.nd_score[0] = 0.f;
   }
-  int epops = -1;
-  if (use_enum && B > 0) epops = enum_build(sm, es, L, B, kc, tc, s_hist, s_bcast, s_warp_tot, s_chain, s_lev);
+  // Adaptive budget: only pops whose score exceeds the request's floor are
+  // kept (NaN keeps nothing).  Pops come in non-increasing score order, so
+  // the kept ones are a leading run of the pop sequence.
+  float floor_v = -INFINITY;
+  bool has_floor = false;
+  if (gain_floor != nullptr) {
+    floor_v = gain_floor[r];
+    if (floor_v != floor_v) floor_v = INFINITY;
+    has_floor = true;
+  }
+  // the smallest order key above the floor (scores compare by their keys)
+  const uint32_t kfloor = !has_floor ? 0u : (floor_v == INFINITY ? 0xFFFFFFFFu : score_key(floor_v) + 1u);
+  int epops = -1, how = 0;
+  if (use_enum && B > 0)
+    epops = enum_build(sm, es, L, B, kc, tc, s_hist, s_bcast, s_warp_tot, s_chain, s_lev, kfloor);
   if (epops >= 0) {
     if (tid == 0) s_pops = epops;
-  } else if (tid < 32) {
-    const int lane = tid;
-    int pops;
-    if (n <= 32 * 3) pops = heap_registers<3>(sm, L, B, kc, tc, lane);
-    else if (n <= 32 * 9) pops = heap_registers<9>(sm, L, B, kc, tc, lane);
-    else pops = heap_tournament(sm, L, B, kc, tc, lane);
-    if (lane == 0) s_pops = pops;
+  } else if (B > 0) {
+    how = n <= 32 * 3 ? 1 : (n <= 32 * 9 ? 2 : 3);
+    if (tid < 32) {
+      const int lane = tid;
+      int pops;
+      if (how == 1) pops = heap_registers<3>(sm, L, B, kc, tc, lane);
+      else if (how == 2) pops = heap_registers<9>(sm, L, B, kc, tc, lane);
+      else pops = heap_tournament(sm, L, B, kc, tc, lane);
+      if (lane == 0) s_pops = pops;
+    }
+  } else if (tid == 0) {
+    s_pops = 0;
   }
   __syncthreads();
+  if (has_floor) {
+    // count of the leading pops above the floor
+    __shared__ int s_keep;
+    if (tid == 0) s_keep = 0;
+    __syncthreads();
+    const int pops = s_pops;
+    int keep = 0;
+    for (int i = 1 + tid; i <= pops; i += BUILD_THREADS) keep += score_key(sm.nd_score[i]) >= kfloor ? 1 : 0;
+    keep = __reduce_add_sync(0xffffffffu, keep);
+    if ((tid & 31) == 0 && keep) atomicAdd(&s_keep, keep);
+    __syncthreads();
+    if (tid == 0) s_pops = s_keep;
+    __syncthreads();
+  }
+  if (build_path != nullptr && tid == 0) build_path[r] = how;
 
   // ---- outputs ----
   const int nn = s_pops + 1;

@@ -159,21 +159,25 @@ int topk_launch(const void* logits, int dtype, int rows, int V, long long row_st
 // ------------------------------------------------------------------ build
 int build_launch(const int32_t* ids, const float* lp, const int32_t* root_token, int n_req, int L, int K,
                  int B, int32_t* node_token, int32_t* parent, int32_t* depth, int32_t* node_rank,
-                 float* score, uint32_t* anc, int32_t* n_nodes, cudaStream_t s) {
+                 float* score, uint32_t* anc, int32_t* n_nodes, cudaStream_t s, int flags = 0,
+                 const float* gain_floor = nullptr, int32_t* build_path = nullptr) {
   if (!ids || !lp || !root_token || !parent || !anc || !n_nodes) return DDTREE_ERR_INVALID_ARG;
   if (n_req < 1 || n_req > MAX_REQ || L < 1 || L > MAX_L || K < 1 || K > MAX_K || B < 0 || B > MAX_B)
     return DDTREE_ERR_INVALID_ARG;
+  if (flags & ~DDTREE_BUILD_FORCE_HEAP) return DDTREE_ERR_INVALID_ARG;
   const int kc = B < K ? B : K;
   // the threshold enumeration when its arrays fit beside the heap's
   cudaFuncAttributes attr;
   if (cudaFuncGetAttributes(&attr, build_kernel) != cudaSuccess) return DDTREE_ERR_CUDA;
   const size_t smem_enum = build_smem_bytes_enum(L, kc, B);
-  const int use_enum = smem_enum + attr.sharedSizeBytes <= (size_t)max_smem_optin() ? 1 : 0;
+  const int use_enum =
+      (!(flags & DDTREE_BUILD_FORCE_HEAP) && smem_enum + attr.sharedSizeBytes <= (size_t)max_smem_optin()) ? 1 : 0;
   const size_t smem = use_enum ? smem_enum : build_smem_bytes(L, kc, B);
   int st = set_smem(build_kernel, smem);
   if (st) return st;
   build_kernel<<<n_req, BUILD_THREADS, smem, s>>>(ids, lp, root_token, L, K, B, kc, tie_code(kc, L), use_enum,
-                                                   node_token, parent, depth, node_rank, score, anc, n_nodes);
+                                                   gain_floor, node_token, parent, depth, node_rank, score, anc,
+                                                   n_nodes, build_path);
   return launch_status();
 }
 
@@ -209,6 +213,10 @@ AttnGeom geom_of(const ddtree_kv_desc* kv, int B) {
   return g;
 }
 
+// Diagnostics of the attention pipeline's timeout path (ddtree_debug_attn_timeout).
+unsigned long long g_attn_wait_ns = 0;   // 0: the default limit
+int g_attn_stop_tile = -1;
+
 bool use_tc_attn(int dtype, const ddtree_kv_desc* kv) {
   return dtype == DDTREE_BF16 && kv->D == 128 && tc_attn_supported(kv->Hq / kv->Hkv);
 }
@@ -234,7 +242,7 @@ int attn_launch(const void* q, const void* k_cache, const void* v_cache, int dty
     const size_t need = tc_attn_ws_bytes(g, num_sms());
     if (need && (!ws || !aligned16(ws) || ws_bytes < need)) return DDTREE_ERR_INVALID_ARG;
     return tc_attn_launch(q, k_cache, v_cache, block_table, prefix_len, anc, n_nodes, g, out, out_lse, ws,
-                          num_sms(), s);
+                          num_sms(), s, g_attn_wait_ns, g_attn_stop_tile);
   }
   const long long grid =
       (long long)g.layers * g.n_req * g.n * ((g.Hq + ATTN_SIMT_WARPS - 1) / ATTN_SIMT_WARPS);
@@ -380,6 +388,14 @@ int ddtree_build(const int32_t* ids, const float* lp, const int32_t* root_token,
                       n_nodes, stream);
 }
 
+int ddtree_build_ex(const int32_t* ids, const float* lp, const int32_t* root_token, int n_req, int L, int K, int B,
+                    int32_t* node_token, int32_t* parent, int32_t* depth, int32_t* node_rank, float* score,
+                    uint32_t* anc, int32_t* n_nodes, const float* gain_floor, int flags, int32_t* build_path,
+                    cudaStream_t stream) {
+  return build_launch(ids, lp, root_token, n_req, L, K, B, node_token, parent, depth, node_rank, score, anc,
+                      n_nodes, stream, flags, gain_floor, build_path);
+}
+
 size_t ddtree_attn_workspace_bytes(const ddtree_kv_desc* kv, int B) {
   if (kv_check(kv) || B < 0 || B > MAX_B) return 0;
   return attn_ws(kv, B, DDTREE_BF16);
@@ -446,7 +462,7 @@ int ddtree_round(const ddtree_round_args* a, cudaStream_t stream) {
                        a->lse, ws, off_attn, stream);
   if (st) return st;
   st = build_launch(a->ids, a->lp, a->root_token, a->n_req, a->L, a->K, a->B, a->node_token, a->parent, a->depth,
-                    a->node_rank, a->score, a->anc, a->n_nodes, stream);
+                    a->node_rank, a->score, a->anc, a->n_nodes, stream, 0, a->gain_floor, nullptr);
   if (st) return st;
   st = attn_launch(a->q, a->k_cache, a->v_cache, a->dtype, &a->kv, a->block_table, a->prefix_len, a->anc,
                    a->n_nodes, a->B, a->attn_out, a->attn_lse, ws + off_attn, off_acc - off_attn, stream);
@@ -455,6 +471,13 @@ int ddtree_round(const ddtree_round_args* a, cudaStream_t stream) {
                        a->n_req, a->L, a->B, a->prefix_len, a->new_prefix_len, a->k_cache, a->v_cache, &a->kv,
                        a->block_table, a->target_argmax, a->path, a->accept_len, a->next_bonus, a->src_slot,
                        a->dst_slot, ws + off_acc, need - off_acc, stream);
+}
+
+int ddtree_debug_attn_timeout(unsigned long long wait_ns, int withhold_tile) {
+  if (withhold_tile < -1) return DDTREE_ERR_INVALID_ARG;
+  g_attn_wait_ns = wait_ns;
+  g_attn_stop_tile = withhold_tile;
+  return DDTREE_OK;
 }
 
 const char* ddtree_status_string(int status) {

@@ -62,6 +62,7 @@ typedef enum {
 #define DDTREE_STATUS_NONFINITE 0x1u
 #define DDTREE_STATUS_TIMEOUT   0x2u
 #define DDTREE_STATUS_CAPACITY  0x4u
+#define DDTREE_STATUS_SETUP     0x8u   /* a kernel could not set up (misaligned shared memory) and did nothing */
 
 typedef enum { DDTREE_BF16 = 0, DDTREE_F32 = 1 } ddtree_dtype;
 
@@ -145,6 +146,43 @@ int ddtree_build(const int32_t* ids, const float* lp, const int32_t* root_token,
                  int32_t* node_rank, float* score, uint32_t* anc, int32_t* n_nodes,
                  cudaStream_t stream);
 
+/*
+ * ddtree_build_ex: ddtree_build with two options and a diagnostic output.
+ *
+ * gain_floor device float [n_req] or NULL.  Adaptive budget ("DDTree Deep
+ *            Dive" §10, cost-aware budgets; the autobench page's note that
+ *            a bigger tree is not faster: the budget has an optimum).  Each
+ *            pop adds its surrogate gain q(u) = exp(score) to the expected
+ *            accepted length (Proposition 1), and pops come in non-increasing
+ *            score order, so the tree that maximises sum q(u) - c*|T| among
+ *            trees of at most B nodes is the leading run of pops with
+ *            q(u) > c.  Request r keeps exactly the pops whose fp32 score is
+ *            strictly greater than gain_floor[r] = log(c_r) (c_r: the
+ *            verification cost of one more node, in accepted tokens); a NaN
+ *            floor keeps no node.  n_nodes[r] = 1 + the kept pops, and rows
+ *            past it are filled as for an exhausted tree.  NULL: no floor.
+ * flags      0, or DDTREE_BUILD_FORCE_HEAP: select by Proposition 3's heap
+ *            even when the threshold enumeration applies (same result;
+ *            diagnostics and tests).
+ * build_path device int32 [n_req] or NULL: which selection ran for the
+ *            request: DDTREE_BUILD_PATH_ENUM (threshold enumeration, or
+ *            B == 0), _HEAP_REG3 / _HEAP_REG9 (register-resident heap for
+ *            B+1 <= 96 / 288), _HEAP_TOURNAMENT (block tournament heap).
+ *            The enumeration falls back to the heap when more than 4096
+ *            prefixes reach its score threshold.
+ */
+#define DDTREE_BUILD_FORCE_HEAP 0x1
+#define DDTREE_BUILD_PATH_ENUM 0
+#define DDTREE_BUILD_PATH_HEAP_REG3 1
+#define DDTREE_BUILD_PATH_HEAP_REG9 2
+#define DDTREE_BUILD_PATH_HEAP_TOURNAMENT 3
+int ddtree_build_ex(const int32_t* ids, const float* lp, const int32_t* root_token,
+                    int n_req, int L, int K, int B,
+                    int32_t* node_token, int32_t* parent, int32_t* depth,
+                    int32_t* node_rank, float* score, uint32_t* anc, int32_t* n_nodes,
+                    const float* gain_floor, int flags, int32_t* build_path,
+                    cudaStream_t stream);
+
 /* ---------------------------------------------------------------------- */
 /* Stage 3: ancestor-only tree attention (Deep Dive §4).                  */
 /* ---------------------------------------------------------------------- */
@@ -194,10 +232,13 @@ size_t ddtree_accept_workspace_bytes(int n_req, int B, int V);
  *            may be NULL to skip compaction.
  * Outputs per request (temperature 0):
  *   target_argmax int32 [n_req][B+1] (may be NULL): argmax of each live
- *                 node's row, lowest id on ties (-0.0 equals +0.0)
+ *                 node's row, lowest id on ties (-0.0 equals +0.0); NaN
+ *                 entries are skipped (and flag DDTREE_STATUS_NONFINITE); a
+ *                 row of NaN only gives -1, which matches no child
  *   path       int32 [n_req][L+1]: accepted node ids root first, -1 after
  *   accept_len int32 [n_req]: accepted draft nodes + 1 (the new bonus)
- *   next_bonus int32 [n_req]: target argmax at the last accepted node
+ *   next_bonus int32 [n_req]: target argmax at the last accepted node (-1
+ *              when that node's row is NaN only)
  *   src_slot, dst_slot int32 [n_req][L+1]: P+path[j] -> P+j, -1 after
  * For every layer and both caches, slot P+path[j] is copied to slot P+j for
  * j = 0..accept_len-1; all sources are read before any destination is
@@ -245,6 +286,9 @@ typedef struct {
   int32_t* new_prefix_len;
   /* scratch */
   void* ws; size_t ws_bytes;
+  /* optional (NULL: none): per-request adaptive-budget floor of the build,
+   * device float [n_req], as gain_floor of ddtree_build_ex */
+  const float* gain_floor;
 } ddtree_round_args;
 
 /* Bytes of a->ws the round needs (0 for an invalid geometry).  The
@@ -277,16 +321,23 @@ int ddtree_round_launch_count(const ddtree_round_args* a);
  * the device or fail because that pool already holds the memory.
  *
  * Limits and behaviour:
- *  - The built-in scratch is 4 MiB per device (allocated when the library is
- *    loaded, held until the process exits).  A request whose scratch need,
- *    ddtree_topk_workspace_bytes(rows, V, K), exceeds it is rejected with
- *    DDTREE_ERR_SCRATCH_LIMIT before anything is launched (at V = 151936
- *    and bf16 logits: up to 571 rows at K = 64, 145 at K = 256, 48 at
- *    K = 1024 on a 148-SM B200).
- *  - The first call on a device looks up the array's device address on the
- *    current device (and, for bf16, builds the exp table as ddtree_topk
- *    does, synchronizing `stream` once); make that first call before any
- *    stream capture.
+ *  - The built-in scratch is 4 MiB per device, held until the process
+ *    exits.  A request whose scratch need for its own dtype exceeds it is
+ *    rejected with DDTREE_ERR_SCRATCH_LIMIT before anything is launched (at
+ *    V = 151936 and bf16 logits: up to 571 rows at K = 64, 145 at K = 256,
+ *    48 at K = 1024 on a 148-SM B200).  ddtree_topk_workspace_bytes(rows,
+ *    V, K) returns the larger of the bf16 and fp32 needs, so it bounds that
+ *    need from above: a request it puts within 4 MiB is always accepted,
+ *    but some it puts above 4 MiB are accepted too.
+ *  - With CUDA's default lazy module loading, the device memory of the
+ *    library's static arrays (this scratch and the 512 KiB exp table of
+ *    ddtree_topk) is allocated when the library's module is first loaded on
+ *    a device, which happens at the first call into it there.  Make one
+ *    warm-up call per device at start-up, before the KV pool takes the free
+ *    memory and before any stream capture: it performs that allocation,
+ *    looks up the array's device address on the current device and, for
+ *    bf16, builds the exp table (synchronizing `stream` once).  Later calls
+ *    allocate nothing.
  *  - Every call on a device shares the one array and leaves its contents
  *    behind; each call clears the counters it needs at its start.  Calls
  *    that overlap on the GPU (other streams, other host threads) race on the
@@ -304,6 +355,24 @@ const char* ddtree_status_string(int status);
 /* Synchronises `stream`, returns the device status word's bits in *bits and
  * clears it.  Returns DDTREE_OK or DDTREE_ERR_CUDA. */
 int ddtree_device_status(cudaStream_t stream, unsigned int* bits);
+
+/*
+ * Diagnostics of the tensor-core attention kernel's timeout path (no
+ * counterpart in the paper).  Every wait of that kernel's pipeline is
+ * bounded; on timeout the kernel sets DDTREE_STATUS_TIMEOUT, every role
+ * leaves its loop, waits (bounded by one second) for its own copies and
+ * tensor-core products in flight, frees its tensor memory and returns, so
+ * the context stays usable.  For tests of that path:
+ *   wait_ns        limit of the pipeline's waits (0: the default, 1 s);
+ *   withhold_tile  >= 0: the producer issues no key tile from this index
+ *                  (within each CTA's key range) on, so a consumer's wait
+ *                  runs out; -1: normal operation.
+ * The setting is process-wide and applies to later ddtree_tree_attn and
+ * ddtree_round calls until reset with (0, -1).  Outputs of a call that
+ * timed out are undefined.  Returns DDTREE_ERR_INVALID_ARG for
+ * withhold_tile < -1.
+ */
+int ddtree_debug_attn_timeout(unsigned long long wait_ns, int withhold_tile);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int ddtree_version(void);

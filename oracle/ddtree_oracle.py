@@ -43,6 +43,9 @@ R6  The whole committed prefix is visible to every tree node; no causal
 R7  Greedy verification (temperature 0): the target's argmax takes the
     lowest token id among equal maxima.  accept_len counts the accepted
     draft nodes plus the new bonus token (k + 1).
+R9  Adaptive budget: a node is worth adding while its gain q(u) exceeds the
+    cost c of verifying one more node (in accepted tokens); the build keeps
+    the pops whose score is strictly above log c.
 """
 from __future__ import annotations
 
@@ -138,7 +141,8 @@ def _order_key(score: np.float32, tup: Tuple[int, ...]):
     return (-float(score), tup)
 
 
-def build_tree(ids: np.ndarray, lp32: np.ndarray, root_token: int, B: int) -> Tree:
+def build_tree(ids: np.ndarray, lp32: np.ndarray, root_token: int, B: int,
+               gain_floor: Optional[float] = None) -> Tree:
     """Top-B prefixes by best-first search (Deep Dive §2, Proposition 3).
 
     ``ids`` and ``lp32`` are one request's [L, K] top-K table.  The frontier
@@ -147,6 +151,12 @@ def build_tree(ids: np.ndarray, lp32: np.ndarray, root_token: int, B: int) -> Tr
     sibling (same parent, rank + 1) and its first child (one position deeper,
     rank 0).  Proposition 2 says the B popped prefixes are the top-B set and
     form a prefix-closed tree.
+
+    ``gain_floor`` (reading R9, the adaptive budget of Deep Dive §10): a pop
+    adds q(u) = exp(score) to the expected acceptance (Proposition 1), so
+    popping stops at the first pop whose float32 score is not strictly above
+    ``gain_floor`` = log c, c being the verification cost of one more node in
+    accepted tokens; that pop is not kept.  A NaN floor keeps nothing.
     """
     L, K = lp32.shape
     t = _empty_tree(B)
@@ -154,6 +164,7 @@ def build_tree(ids: np.ndarray, lp32: np.ndarray, root_token: int, B: int) -> Tr
     t.depth[0] = 0
     t.score[0] = np.float32(0.0)
     t.tuples = [()]
+    floor = None if gain_floor is None else np.float32(gain_floor)
     # heap entries: (order key, parent node, depth d (1-based), rank r, score)
     heap = []
     s0 = np.float32(np.float32(0.0) + lp32[0, 0])
@@ -161,6 +172,8 @@ def build_tree(ids: np.ndarray, lp32: np.ndarray, root_token: int, B: int) -> Tr
     pops = 0
     while pops < B and heap:
         (_, tup), par, d, r, s = heapq.heappop(heap)
+        if floor is not None and not (s > floor):
+            break
         pops += 1
         node = pops
         t.node_token[node] = ids[d - 1, r]
@@ -196,9 +209,11 @@ def ancestor_mask(parent: np.ndarray, n_nodes: int, n: int) -> np.ndarray:
     return anc
 
 
-def build_trees(ids: np.ndarray, lp32: np.ndarray, root_token: Sequence[int], B: int) -> List[Tree]:
+def build_trees(ids: np.ndarray, lp32: np.ndarray, root_token: Sequence[int], B: int,
+                gain_floor: Optional[Sequence[float]] = None) -> List[Tree]:
     """``build_tree`` for each request of an [N, L, K] table."""
-    return [build_tree(ids[r], lp32[r], int(root_token[r]), B) for r in range(ids.shape[0])]
+    return [build_tree(ids[r], lp32[r], int(root_token[r]), B,
+                       None if gain_floor is None else float(gain_floor[r])) for r in range(ids.shape[0])]
 
 
 def stack_trees(trees: List[Tree]):

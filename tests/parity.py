@@ -92,3 +92,31 @@ def order_margin(lp32: np.ndarray, B: int) -> float:
                 continue
         margin = min(margin, gap)
     return float(margin)
+
+
+def raw_bits(t: torch.Tensor) -> np.ndarray:
+    """The tensor's bytes as integers of its element size (exact comparisons
+    and plain row copies without a float64 widening of large caches)."""
+    t = t.detach().to("cpu").contiguous()
+    if t.element_size() == 2:
+        return t.view(torch.int16).numpy().copy()
+    if t.element_size() == 4:
+        return t.view(torch.int32).numpy().copy()
+    return t.numpy().copy()
+
+
+def attention_ref(w, q, cache, prefix, anc, n_nodes, layers=None, reqs=None, nodes=None, heads=None):
+    """Oracle tree attention on sampled layers, widened to float64 one layer
+    at a time (the 48-layer caches would not fit in float64 at once).
+    Returns {(layer, req, node, head): out row} and the matching lse dict."""
+    table = None if cache.block_table is None else cache.block_table.numpy()
+    layers = range(q.shape[0]) if layers is None else layers
+    out, lse = {}, {}
+    for l in layers:
+        o, s = oracle.tree_attention(np64(q[l:l + 1]), np64(cache.k[l:l + 1]), np64(cache.v[l:l + 1]), prefix,
+                                     anc, n_nodes, datagen.default_scale(w), block_table=table, reqs=reqs,
+                                     nodes=nodes, heads=heads)
+        for (_, r, i, h), v in o.items():
+            out[(l, r, i, h)] = v
+            lse[(l, r, i, h)] = s[(0, r, i, h)]
+    return out, lse

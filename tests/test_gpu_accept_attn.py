@@ -241,3 +241,52 @@ def test_attention_budget_zero_is_decode():
     st, prefix, cache, q = _attn_case(w)
     out, lse = _gpu_attn(w, st, prefix, cache, q)
     _check_attn(w, st, prefix, cache, q, out, lse)
+
+
+def test_accept_nan_rows_give_sentinel():
+    """A target row of NaN only has no argmax: the kernel reports -1 (which
+    matches no child, so the walk stops there) and flags NONFINITE; a row
+    with some NaN entries takes the argmax of the others."""
+    w = datagen.workload(2, V=4096)
+    z, ids, lp32, lse32, root, trees, st = tree_inputs(w)
+    tgt = _target_for(w, z, st, plant_path=[_deepest(st, 0)])
+    c = int(st["parent"][0, _deepest(st, 0)])     # a node on the planted path
+    tgt[0, c, :] = float("nan")
+    tgt[0, 0, 5:4000:7] = float("nan")            # the root row keeps its planted maximum
+    acc = dd.ddtree_accept(_dev(tgt), _dev(st["node_token"]), _dev(st["parent"]), _dev(st["n_nodes"]), w.L,
+                           _dev(np.array([10])))
+    torch.cuda.synchronize()
+    assert dd.device_status() & dd.STATUS_NONFINITE
+    ta = acc.target_argmax[0].cpu().numpy()
+    assert ta[c] == -1
+    clean = tgt[0, 0].clone()
+    clean[torch.isnan(clean)] = -float("inf")
+    assert ta[0] == int(oracle.argmax_rows(clean.to(torch.float64).numpy()[None])[0])
+    path = [p for p in acc.path[0].tolist() if p >= 0]
+    assert path[-1] == c and int(acc.next_bonus[0]) == -1
+    assert int(acc.accept_len[0]) == len(path)
+
+
+def test_attention_wait_timeout_reports_and_recovers():
+    """The pipeline's bounded waits: with the producer withholding a key tile
+    and a 200 us limit, a consumer wait runs out, the kernel returns and sets
+    TIMEOUT (cleared by the status read), and the next call with the normal
+    settings matches the oracle."""
+    w = datagen.workload(2)
+    st, prefix, cache, q = _attn_case(w)
+    lib = dd.lib()
+    try:
+        assert lib.ddtree_debug_attn_timeout(200_000, 1) == 0
+        dev = _to_dev_cache(cache)
+        kv = dd.kv_desc_for(dev.k, w.N, w.Hq, dev.block_table)
+        dd.ddtree_tree_attn(q.to(CUDA), dev.k, dev.v, kv, _dev(prefix), _dev(st["anc"]), _dev(st["n_nodes"]), w.B)
+        torch.cuda.synchronize()
+        bits = dd.device_status()
+        assert bits & dd.STATUS_TIMEOUT, bits
+        assert not bits & dd.STATUS_SETUP
+        assert dd.device_status() == 0
+    finally:
+        assert lib.ddtree_debug_attn_timeout(0, -1) == 0
+    assert lib.ddtree_debug_attn_timeout(0, -2) != 0
+    out, lse = _gpu_attn(w, st, prefix, cache, q)
+    _check_attn(w, st, prefix, cache, q, out, lse)

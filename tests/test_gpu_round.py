@@ -1,10 +1,13 @@
 """GPU parity of the whole round (ddtree_round) against the oracle chain.
 
-The round feeds its own top-K table to its build.  Its log-probs are the
-fp64 log-softmax rounded once to fp32, like the oracle's, so the table is
-bit-identical in practice and every tree array is then compared bit for
-bit; every downstream integer output and the compacted cache are compared
-bit for bit, the attention output within tolerance.
+The round feeds its own top-K table to its build.  Its ids must equal the
+oracle's and its log-probs lie within the stated tolerance of them (in
+practice they are bit-identical: both are the fp64 log-softmax rounded once
+to fp32).  The tree is then compared, bit for bit, with the oracle's tree
+built from the round's own lp table ("DDTree Deep Dive" §2, Propositions 2
+and 3: the tree is a function of that table), and with the oracle's own tree
+when the tables agree.  Every downstream integer output and the compacted
+cache are compared bit for bit, the attention output within tolerance.
 """
 import numpy as np
 import pytest
@@ -14,14 +17,16 @@ import draft_tree_build_ddtree_b200 as dd
 import oracle
 from draft_tree_build_ddtree_b200 import datagen
 
-from parity import assert_topk, attn_close, np64, tree_inputs
+from parity import assert_topk, assert_tree, attention_ref, attn_close, np64, raw_bits, tree_inputs
 
 pytestmark = pytest.mark.gpu
 CUDA = "cuda:0"
 
 
-def make_round(w, rep=0):
+def make_round(w, rep=0, gain_floor=None):
     z, ids, lp32, lse32, root, trees, st = tree_inputs(w, rep)
+    if gain_floor is not None:
+        st = oracle.stack_trees(oracle.build_trees(ids, lp32, root, w.B, gain_floor=gain_floor))
     prefix = datagen.prefix_lengths(w, rep)
     cache = datagen.kv_cache(w, prefix, rep)
     q = datagen.queries(w, rep)
@@ -32,61 +37,52 @@ def make_round(w, rep=0):
         drafter_logits=z.to(CUDA), root_token=torch.from_numpy(root).to(CUDA), q=q.to(CUDA),
         k_cache=cache.k.to(CUDA), v_cache=cache.v.to(CUDA),
         block_table=None if cache.block_table is None else cache.block_table.to(CUDA),
-        prefix_len=prefix.to(CUDA), target_logits=tgt.to(CUDA)).allocate_outputs()
+        prefix_len=prefix.to(CUDA), target_logits=tgt.to(CUDA),
+        gain_floor=None if gain_floor is None else torch.from_numpy(np.asarray(gain_floor, np.float32)).to(CUDA),
+    ).allocate_outputs()
     host = dict(z=z, ids=ids, lp32=lp32, lse32=lse32, root=root, st=st, prefix=prefix.numpy(),
-                cache=cache, q=q, tgt=tgt)
+                cache=cache, q=q, tgt=tgt, gain_floor=gain_floor)
     return rb, host
 
 
-def _valid_tree(parent, anc, n_nodes):
-    for i in range(1, n_nodes):
-        assert 0 <= parent[i] < i
-    walk = oracle.ancestor_mask(parent, n_nodes, parent.shape[0])
-    assert np.array_equal(anc.view(np.uint32), walk)
-
-
-def check_round(w, rb, h, layers=None, nodes=None, heads=None):
+def check_round(w, rb, h, layers=None, nodes=None, heads=None, reqs=None):
     assert dd.device_status() == 0
     assert_topk(rb.ids.reshape(-1, w.K), rb.lp.reshape(-1, w.K), rb.lse, h["ids"].reshape(-1, w.K),
                 h["lp32"].reshape(-1, w.K), h["lse32"].reshape(-1))
+    # the oracle's tree from the round's own (ids, lp) table: bit for bit
+    g_ids = rb.ids.cpu().numpy()
+    g_lp = rb.lp.cpu().numpy()
+    own = oracle.stack_trees(oracle.build_trees(g_ids, g_lp, h["root"], w.B, gain_floor=h["gain_floor"]))
+    assert_tree(rb.tree, own)
     st = h["st"]
-    # The tree is a deterministic function of the (ids, lp) table, and the
-    # build stage alone is bit-exact on identical tables; so when the round's
-    # lp table is bit-identical to the oracle's, every tree array must be too.
-    lp_same = np.array_equal(rb.lp.cpu().numpy().reshape(h["lp32"].shape).view(np.uint32),
-                             h["lp32"].view(np.uint32))
-    t = rb.tree
-    if lp_same:
-        for name in ("node_token", "parent", "depth", "node_rank", "n_nodes"):
-            assert np.array_equal(getattr(t, name).cpu().numpy(), st[name]), name
-        assert np.array_equal(t.anc.cpu().numpy().view(np.uint32), st["anc"])
-        assert np.array_equal(t.score.cpu().numpy().view(np.uint32), st["score"].view(np.uint32))
+    if np.array_equal(g_lp.view(np.uint32), h["lp32"].view(np.uint32)):
+        assert_tree(rb.tree, st)
     else:
-        for r in range(w.N):
-            _valid_tree(t.parent[r].cpu().numpy(), t.anc[r].cpu().numpy(), int(t.n_nodes[r]))
-        pytest.skip("an lp value differs from the oracle's in its last bit: tree validity checked only")
-    # attention of the tree nodes
-    table = None if h["cache"].block_table is None else h["cache"].block_table.numpy()
-    ref, _ = oracle.tree_attention(np64(h["q"]), np64(h["cache"].k), np64(h["cache"].v), h["prefix"],
-                                   st["anc"], st["n_nodes"], datagen.default_scale(w), block_table=table,
-                                   layers=layers, nodes=nodes, heads=heads)
-    o = np64(rb.attn_out.cpu())
+        st = own
+    # attention of the tree nodes (sampled where asked)
+    ref, _ = attention_ref(w, h["q"], h["cache"], h["prefix"], st["anc"], st["n_nodes"], layers=layers,
+                           reqs=reqs, nodes=nodes, heads=heads)
+    o = rb.attn_out
     for (l, r, i, hh), v in ref.items():
-        ok, ex = attn_close(o[l, r, i, hh], v)
+        got = o[l, r, i, hh].to("cpu", torch.float64).numpy()
+        ok, ex = attn_close(got, v)
         assert ok, (l, r, i, hh, ex)
-    # walk and compaction
-    tg = h["tgt"].to(torch.float64).numpy()
-    kh, vh = np64(h["cache"].k), np64(h["cache"].v)
+    # walk, and the compaction of every layer's K and V, bit for bit
+    tg = h["tgt"]
+    table = None if h["cache"].block_table is None else h["cache"].block_table.numpy()
+    kh, vh = raw_bits(h["cache"].k), raw_bits(h["cache"].v)
     for r in range(w.N):
-        a = oracle.accept(tg[r], st["node_token"][r], st["parent"][r], int(st["n_nodes"][r]), w.L,
-                          int(h["prefix"][r]))
+        a = oracle.accept(tg[r].to(torch.float64).numpy(), st["node_token"][r], st["parent"][r],
+                          int(st["n_nodes"][r]), w.L, int(h["prefix"][r]))
         assert rb.acc.path[r].tolist() == a.path.tolist()
         assert int(rb.acc.accept_len[r]) == a.accept_len
         assert int(rb.acc.next_bonus[r]) == a.next_bonus
         assert int(rb.acc.new_prefix_len[r]) == a.new_prefix_len
+        assert rb.acc.src_slot[r].tolist() == a.src_slot.tolist()
+        assert rb.acc.dst_slot[r].tolist() == a.dst_slot.tolist()
         oracle.compact(kh, vh, r, a, block_table=table)
-    assert np.array_equal(np64(rb.k_cache.cpu()), kh)
-    assert np.array_equal(np64(rb.v_cache.cpu()), vh)
+    assert np.array_equal(raw_bits(rb.k_cache), kh)
+    assert np.array_equal(raw_bits(rb.v_cache), vh)
 
 
 @pytest.mark.parametrize("cfg", [1, 2])
@@ -98,12 +94,49 @@ def test_round_configs(cfg):
     check_round(w, rb, h)
 
 
+def test_round_48_layers_b256_p8k():
+    """b256_p8k_48l end to end: attention sampled over (layer, node, head),
+    the walk's compaction of all 48 layers compared bit for bit (the separate
+    walk + compaction launch)."""
+    w = datagen.workload(3)
+    rb, h = make_round(w)
+    dd.ddtree_round(rb)
+    torch.cuda.synchronize()
+    check_round(w, rb, h, layers=[0, 23, 47], nodes=[0, 1, 100, 255, 256], heads=[0, 9, 31])
+
+
+@pytest.mark.parametrize("sigma", [1.0, 8.0])
+def test_round_p32k_b1024(sigma):
+    """sweep_p32k at B = 1024: bushy (sigma 1) and chain-like (sigma 8) trees."""
+    w = datagen.workload(5, B=1024, sigma=sigma)
+    rb, h = make_round(w)
+    dd.ddtree_round(rb)
+    torch.cuda.synchronize()
+    check_round(w, rb, h, nodes=[0, 1, 17, 512, 1023, 1024], heads=[0, 13, 31])
+
+
 def test_round_batched_paged_sampled():
     w = datagen.workload(4)
     rb, h = make_round(w)
     dd.ddtree_round(rb)
     torch.cuda.synchronize()
     check_round(w, rb, h, nodes=[0, 3, 64], heads=[0, 31])
+
+
+@pytest.mark.parametrize("cfg", [2, 4])
+def test_round_adaptive_budget(cfg):
+    """A round with per-request gain floors (adaptive budget): the build
+    keeps the pops above each floor and every later stage works on that
+    smaller tree."""
+    w = datagen.workload(cfg)
+    z, ids, lp32, lse32, root, trees, st = tree_inputs(w)
+    floor = np.array([float(st["score"][r, (7 * r + 20) % w.n]) for r in range(w.N)], np.float32)
+    rb, h = make_round(w, gain_floor=floor)
+    dd.ddtree_round(rb)
+    torch.cuda.synchronize()
+    assert np.all(rb.tree.n_nodes.cpu().numpy() <= w.n)
+    check_round(w, rb, h, nodes=None if cfg == 2 else [0, 3, 64], heads=None if cfg == 2 else [0, 31],
+                reqs=None if cfg == 2 else [0, 5, 31])
 
 
 @pytest.mark.parametrize("cfg,over", [

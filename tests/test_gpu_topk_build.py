@@ -8,6 +8,7 @@ import pytest
 import torch
 
 import draft_tree_build_ddtree_b200 as dd
+import oracle
 from draft_tree_build_ddtree_b200 import datagen
 
 from parity import assert_topk, assert_tree, oracle_topk, oracle_trees, tree_inputs
@@ -164,3 +165,101 @@ def test_build_batched_config4():
     w = datagen.workload(4)
     z, ids, lp32, lse32, root, trees, st = tree_inputs(w)
     assert_tree(_gpu_build(ids, lp32, root, w.B), st)
+
+
+# ------------------------------------------------------------------ build: every selection path
+
+def _gpu_build_ex(ids, lp32, root, B, flags=0, floor=None):
+    N = ids.shape[0]
+    path = torch.full((N,), -7, dtype=torch.int32, device=CUDA)
+    fl = None if floor is None else torch.as_tensor(np.asarray(floor, np.float32)).to(CUDA)
+    t = dd.ddtree_build(torch.from_numpy(np.ascontiguousarray(ids)).to(CUDA),
+                        torch.from_numpy(np.ascontiguousarray(lp32)).to(CUDA),
+                        torch.from_numpy(np.ascontiguousarray(root).astype(np.int32)).to(CUDA), B,
+                        gain_floor=fl, flags=flags, build_path=path)
+    torch.cuda.synchronize()
+    return t, path.cpu().numpy()
+
+
+def _heap_kind(B):
+    n = B + 1
+    return 1 if n <= 96 else (2 if n <= 288 else 3)
+
+
+@pytest.mark.parametrize("cfg,over", [(1, {}), (2, {}), (3, {}), (4, {}), (5, dict(B=1024, K=1024)),
+                                      (5, dict(B=200, K=200))])
+def test_build_forced_heap_matches_oracle(cfg, over):
+    """Proposition 3's heap itself (all three queue variants), bit for bit."""
+    w = datagen.workload(cfg, **over)
+    z, ids, lp32, lse32, root, trees, st = tree_inputs(w)
+    t, path = _gpu_build_ex(ids, lp32, root, w.B, flags=dd.BUILD_FORCE_HEAP)
+    assert np.all(path == _heap_kind(w.B)), path
+    assert_tree(t, st)
+    # the default call takes the enumeration on these tables and agrees
+    t2, path2 = _gpu_build_ex(ids, lp32, root, w.B)
+    assert np.all(path2 == 0), path2
+    assert_tree(t2, st)
+
+
+def _tie_table(N, L, K, top_equal, seed):
+    """lp tables whose `top_equal` best ranks at every position are exactly
+    0.0 (the rest strictly negative): every prefix over those ranks scores
+    exactly 0, the largest possible score."""
+    g = torch.Generator().manual_seed(seed)
+    lp = -(torch.rand(N, L, K, generator=g) * 4 + 0.5)
+    lp[:, :, :top_equal] = 0.0
+    lp = -torch.sort(-lp, dim=-1).values
+    ids = torch.randint(0, 151936, (N, L, K), generator=g).to(torch.int32)
+    return ids.numpy(), lp.numpy().astype(np.float32)
+
+
+@pytest.mark.parametrize("B,K,top_equal", [(64, 64, 64), (95, 8, 8), (200, 64, 4), (287, 16, 16),
+                                           (1024, 1024, 1024), (1024, 64, 3)])
+def test_build_enumeration_overflow_takes_heap(B, K, top_equal):
+    """Tie-heavy tables overflow the enumeration: the kernel reports the heap
+    it fell back to, and the tree is the oracle's bit for bit.
+
+    Why the enumeration must overflow, from the oracle's side: the B-th pop
+    scores 0, the largest possible score, so any threshold that admits B
+    prefixes admits every prefix scoring 0, and there are
+    sum_d top_equal^d > 4096 of them."""
+    N, L = 3, 16
+    ids, lp32 = _tie_table(N, L, K, top_equal, seed=B + K)
+    root = np.arange(N, dtype=np.int32)
+    trees, st = oracle_trees(ids, lp32, root, B)
+    assert np.all(st["score"][:, B] == 0.0)
+    assert sum(top_equal ** d for d in range(1, L + 1)) > 4096
+    t, path = _gpu_build_ex(ids, lp32, root, B)
+    assert np.all(path == _heap_kind(B)), path
+    assert_tree(t, st)
+
+
+@pytest.mark.parametrize("cfg,over", [(1, {}), (2, {}), (3, {}), (5, dict(B=1024, K=1024, sigma=8.0))])
+@pytest.mark.parametrize("flags", [0, 1])
+def test_build_adaptive_floor_matches_oracle(cfg, over, flags):
+    """Adaptive budget (gain floor): the kept pops are the oracle's, bit for
+    bit, for floors at a node's exact score, between scores, and the edges."""
+    w = datagen.workload(cfg, **over)
+    z, ids, lp32, lse32, root, trees, st = tree_inputs(w)
+    s = st["score"][0]
+    nn = int(st["n_nodes"][0])
+    cases = [float(s[nn // 2]), float(np.float32(s[nn // 3]) - np.float32(1e-3)), -np.inf, np.inf, np.nan,
+             -1e30, 0.0]
+    for f in cases:
+        floor = np.full(w.N, f, np.float32)
+        ref = oracle.stack_trees(oracle.build_trees(ids, lp32, root, w.B, gain_floor=floor))
+        t, path = _gpu_build_ex(ids, lp32, root, w.B, flags=flags, floor=floor)
+        assert_tree(t, ref)
+
+
+def test_build_adaptive_floor_per_request():
+    """Each request keeps its own floor (batched workload, mixed floors)."""
+    w = datagen.workload(4)
+    z, ids, lp32, lse32, root, trees, st = tree_inputs(w)
+    g = np.random.default_rng(5)
+    floor = np.array([float(st["score"][r, g.integers(1, w.n)]) for r in range(w.N)], np.float32)
+    floor[3] = -np.inf
+    floor[7] = np.nan
+    ref = oracle.stack_trees(oracle.build_trees(ids, lp32, root, w.B, gain_floor=floor))
+    t, _ = _gpu_build_ex(ids, lp32, root, w.B, floor=floor)
+    assert_tree(t, ref)

@@ -148,6 +148,103 @@ def test_beam_and_chain_never_beat_heap():
     assert oracle.surrogate_value(chain, lp64_topk) <= v_heap + 1e-15
 
 
+def _brute_beam(lp32, width):
+    """Beam search written from the definition over the full prefix list:
+    at depth d, rank every length-d prefix whose parent is in the previous
+    beam by reading R4 and keep the ``width`` best."""
+    L, K = lp32.shape
+    prev = {()}
+    out = []
+    for d in range(1, L + 1):
+        cand = [u for u in itertools.product(range(K), repeat=d) if u[:-1] in prev]
+        cand.sort(key=lambda u: (-float(oracle.prefix_score(lp32, u)), u))
+        keep = cand[:width]
+        out.extend(keep)
+        prev = set(keep)
+    return out
+
+
+@pytest.mark.parametrize("width", [1, 2, 3, 5, 8])
+def test_beam_tree_equals_definition_config1(width):
+    w, z, ids, lp32, lse32, lp64 = _cfg1()
+    beam = oracle.beam_tree(lp32[0], width)
+    ref = _brute_beam(lp32[0], width)
+    assert beam == ref
+    # every depth keeps min(width, K * |previous beam|) prefixes
+    K, L = w.K, w.L
+    size, expect = 1, 0
+    for _ in range(L):
+        size = min(width, K * size)
+        expect += size
+    assert len(beam) == expect
+
+
+def test_beam_tree_extremes():
+    w, z, ids, lp32, lse32, lp64 = _cfg1()
+    # width 1 is the single drafted line (argmax at every position)
+    assert oracle.beam_tree(lp32[0], 1) == oracle.chain_tree(w.L)
+    # a width no depth can fill keeps every prefix
+    small = lp32[0][:3, :4]
+    allp = [u for d in range(1, 4) for u in itertools.product(range(4), repeat=d)]
+    assert sorted(oracle.beam_tree(small, 4 ** 3)) == sorted(allp)
+
+
+def _prefix_closed_subsets(prefixes):
+    """Every subset of ``prefixes`` whose members' parents are members."""
+    idx = {u: i for i, u in enumerate(prefixes)}
+    n = len(prefixes)
+    for mask in range(1 << n):
+        ok = True
+        for u, i in idx.items():
+            if (mask >> i) & 1 and len(u) > 1 and not (mask >> idx[u[:-1]]) & 1:
+                ok = False
+                break
+        if ok:
+            yield [u for u, i in idx.items() if (mask >> i) & 1]
+
+
+@pytest.mark.parametrize("L,K,seed", [(2, 3, 0), (2, 3, 1), (3, 2, 2), (3, 2, 5)])
+def test_adaptive_budget_equals_bruteforce_optimum(L, K, seed):
+    """Reading R9 (Deep Dive §10, cost-aware budgets): the adaptive tree is
+    the prefix-closed tree of at most B nodes that maximises
+    sum_{u in T} q(u) - c * |T|, found here by trying every prefix-closed set."""
+    g = torch.Generator().manual_seed(100 + seed)
+    z = (torch.randn(L, 6, generator=g, dtype=torch.float64) * 1.5).numpy()
+    ids, lp32, _, lp64 = oracle.topk(z, K)
+    q = {}
+    prefixes = [u for d in range(1, L + 1) for u in itertools.product(range(K), repeat=d)]
+    lpk = np.take_along_axis(lp64, ids.astype(np.int64), axis=-1)
+    for u in prefixes:
+        q[u] = float(np.exp(sum(lpk[d, r] for d, r in enumerate(u))))
+    vals = sorted(set(q.values()))
+    # costs in the gaps between distinct gains (no gain within 1e-4 relative of c)
+    costs = [0.5 * (a + b) for a, b in zip(vals, vals[1:]) if b - a > 1e-4 * b] + [vals[-1] * 1.5, vals[0] * 0.5]
+    subsets = list(_prefix_closed_subsets(prefixes))
+    for c in costs:
+        for B in (1, 3, len(prefixes)):
+            best = max((sum(q[u] for u in T) - c * len(T), sorted(T)) for T in subsets if len(T) <= B)
+            t = oracle.build_tree(ids, lp32, 0, B, gain_floor=math.log(c))
+            assert sorted(t.tuples[1:]) == best[1], (c, B)
+
+
+def test_adaptive_budget_floor_edges():
+    w, z, ids, lp32, lse32, lp64 = _cfg1()
+    full = oracle.build_tree(ids[0], lp32[0], 0, w.B)
+    # no floor and a floor below every score give the budgeted tree
+    low = oracle.build_tree(ids[0], lp32[0], 0, w.B, gain_floor=-1e30)
+    assert low.tuples == full.tuples
+    # a floor at or above the best score keeps the root only; so does NaN
+    for f in (0.0, float(full.score[1]), float("nan")):
+        t = oracle.build_tree(ids[0], lp32[0], 0, w.B, gain_floor=f)
+        assert t.n_nodes == 1 and t.tuples == [()]
+    # a floor equal to a node's score drops that node and everything after it
+    i = 7
+    t = oracle.build_tree(ids[0], lp32[0], 0, w.B, gain_floor=float(full.score[i]))
+    kept = [j for j in range(1, full.n_nodes) if full.score[j] > full.score[i]]
+    assert t.n_nodes == 1 + len(kept)
+    assert t.tuples == full.tuples[:t.n_nodes]
+
+
 def test_lemma1_topk_min_b_v_suffices():
     g = torch.Generator().manual_seed(3)
     V, L = 9, 3

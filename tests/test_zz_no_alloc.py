@@ -65,3 +65,48 @@ def test_static_scratch_rejects_requests_beyond_its_size():
                                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 7
     assert b"scratch" in dd.lib().ddtree_status_string(st)
+
+
+def test_static_scratch_largest_accepted_request_and_no_allocation():
+    """The largest request the 4 MiB scratch accepts (found through the call
+    itself: a rejected request launches nothing) runs like ddtree_topk and the
+    oracle on sampled rows; one row more is rejected; and a call after the
+    first leaves the device's free memory unchanged."""
+    import oracle
+    V, K = 151936, 64
+    g = torch.Generator().manual_seed(11)
+    big = (torch.randn(640, V, generator=g) * 4).to(torch.bfloat16).to(CUDA)
+    lo, hi = 1, 640                      # largest accepted row count in [lo, hi)
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        ids = torch.empty((mid, K), dtype=torch.int32, device=CUDA)
+        lp = torch.empty((mid, K), dtype=torch.float32, device=CUDA)
+        st = dd.lib().ddtree_topk_static_ws(ctypes.c_void_p(big.data_ptr()), dd.BF16, mid, V, V, K,
+                                            ctypes.c_void_p(ids.data_ptr()), ctypes.c_void_p(lp.data_ptr()), None,
+                                            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert st in (0, 7)
+        lo, hi = (mid, hi) if st == 0 else (lo, mid)
+    rows = lo
+    assert 500 <= rows < 640, rows     # about 571 rows on a 148-SM B200
+    x = big[:rows]
+    ref_ids, ref_lp, ref_lse = dd.ddtree_topk(x, K)
+    torch.cuda.synchronize()
+    ids, lp, lse = _static_topk(x, K)
+    free0 = torch.cuda.mem_get_info()[0]
+    ids2, lp2, lse2 = _static_topk(x, K)
+    free1 = torch.cuda.mem_get_info()[0]
+    assert free1 == free0
+    for a, b in ((ids, ref_ids), (ids2, ref_ids)):
+        assert torch.equal(a, b)
+    assert float((lp2 - ref_lp).abs().max()) <= LP_TOL
+    sample = [0, 1, rows // 2, rows - 1]
+    o_ids, o_lp, _, _ = oracle.topk(x[sample].to("cpu", torch.float64).numpy(), K)
+    assert np.array_equal(ids2[sample].cpu().numpy(), o_ids)
+    assert np.max(np.abs(lp2[sample].cpu().numpy().astype(np.float64) - o_lp)) <= LP_TOL
+    one_more = torch.empty((rows + 1, K), dtype=torch.int32, device=CUDA)
+    lp_more = torch.empty((rows + 1, K), dtype=torch.float32, device=CUDA)
+    st = dd.lib().ddtree_topk_static_ws(ctypes.c_void_p(big.data_ptr()), dd.BF16, rows + 1, V, V, K,
+                                        ctypes.c_void_p(one_more.data_ptr()), ctypes.c_void_p(lp_more.data_ptr()),
+                                        None, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 7
+    assert dd.device_status() == 0

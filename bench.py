@@ -6,21 +6,29 @@
 A step is one ddtree_round (top-K -> tree build -> tree attention over all
 of the workload's layers -> verifier walk + KV compaction) over one batch of
 synthetic inputs already resident in HBM.  Steps rotate over enough input
-sets that consecutive steps never find their inputs in L2.  Each rank runs
-its own independent rounds (replicas: the round of one request batch does
-not shard), timed with CUDA events and reduced as the max over ranks; rank
-0 prints one JSON line.
+sets that consecutive steps never find their inputs in L2.  The default
+workload is b256_p8k_48l (budget 256, 8k prefix, 48 layers: the largest
+single-GPU configuration); ``per_config`` adds b64_p2k, the 32-request
+paged batch and the 32k-prefix sweep at B = 64 and 256.
+
+Multi-GPU: ``--gpus N`` without a torchrun environment re-launches itself
+under ``torch.distributed.run`` with N ranks.  Batch-1 workloads run as
+independent replicas (weak scaling); the batched workload (config 4) is
+sharded by request (request r on rank r mod N, strong scaling) and each
+round ends with an NCCL all-gather of every request's accept length, next
+bonus token and new prefix length.  Times are CUDA events, max over ranks.
 
 ``--impl reference`` times the CPU oracle (the checker, plain numpy) on the
-host, each step a bounded sample of the same workload, extrapolated to the
-same metric.
+host, each step one bounded sample of the same workload.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -40,49 +48,57 @@ UNIT = "rounds/s"
 L2_BYTES = 126 * 1024 * 1024
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DEFAULT_CONFIG = 3
+PER_CONFIG = ((2, {}), (4, {}), (5, {"B": 64, "sigma": 4.0}), (5, {"B": 256, "sigma": 4.0}))
+SUSTAINED_AFTER_S = 1.0      # a timed region at least this long is graded against the sustained peak
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG)
     ap.add_argument("--budget", type=int, default=None, help="config 5: B")
     ap.add_argument("--sigma", type=float, default=None, help="config 5: drafter logit std-dev")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true", help="launch rounds eagerly instead of CUDA graphs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="profiling driver: one input set, warmup + steps eager rounds, no timing")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
 # ncu capture, with a hash of the kernel's sources at capture time: the value
 # is reported only while the sources are unchanged (summaries under profiles/).
-CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "draft_tree_build_ddtree_b200", "csrc")
+CSRC = os.path.join(ROOT, "draft_tree_build_ddtree_b200", "csrc")
 TRAFFIC = {
     ("b64_p2k", "topk"): (5069568, ("topk.cuh", "common.cuh", "exp64_table.h"), "4c480e2f4cca5119"),
     ("b256_p8k_48l", "attn"): (1057939712, ("attn_tc.cuh", "attn_simt.cuh", "common.cuh"), "673c3d78fa774a8f"),
 }
 
 
-def measured_traffic(workload: str, stage: str):
+def sources_digest(files) -> str:
     import hashlib
+    m = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            m.update(fh.read())
+    return m.hexdigest()[:16]
+
+
+def measured_traffic(workload: str, stage: str):
     entry = TRAFFIC.get((workload, stage))
     if entry is None:
         return None
     nbytes, files, digest = entry
-    m = hashlib.sha256()
     try:
-        for f in files:
-            with open(os.path.join(CSRC, f), "rb") as fh:
-                m.update(fh.read())
+        return nbytes if sources_digest(files) == digest else None
     except OSError:
         return None
-    return nbytes if m.hexdigest()[:16] == digest else None
 
 
 def load_peaks():
@@ -103,7 +119,10 @@ def dist_env():
 def init_dist(world: int, backend: str = "nccl"):
     if world > 1 and not torch.distributed.is_initialized():
         import datetime
-        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+        kw = {}
+        if backend == "nccl":
+            kw["device_id"] = torch.device("cuda", dist_env()[2])
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120), **kw)
 
 
 def max_over_ranks(x: float, device=None) -> float:
@@ -128,6 +147,20 @@ def aggregate_rate(units_per_rank: float, world: int, seconds_max: float) -> flo
     return units_per_rank * world / seconds_max
 
 
+def free_port() -> int:
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def relaunch_cmd(argv, n: int, port: int):
+    """The torchrun command that runs this script on n ranks of one node."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -141,7 +174,6 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
-        self.t0 = self.t1 = None
 
     def start(self):
         try:
@@ -186,10 +218,18 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- workload
 
+def workload_of(cfg: int, over=None):
+    over = dict(over or {})
+    if cfg == 5:
+        return datagen.workload(5, B=over.pop("B", 64), sigma=over.pop("sigma", 4.0), **over)
+    return datagen.workload(cfg, **over)
+
+
 def workload_from_args(a):
+    over = {}
     if a.config == 5:
-        return datagen.workload(5, B=a.budget if a.budget else 64, sigma=a.sigma if a.sigma else 4.0)
-    return datagen.workload(a.config)
+        over = {"B": a.budget or 64, "sigma": a.sigma or 4.0}
+    return workload_of(a.config, over)
 
 
 def workload_label(w) -> str:
@@ -207,34 +247,41 @@ def set_bytes(w) -> int:
     return (w.N * w.L * w.V + w.N * w.n * w.V) * es + w.layers * w.N * w.n * w.Hq * w.D * es + kv
 
 
-def make_sets(w, R, device):
-    """R independent input sets on the device, each a ready RoundBuffers."""
+def host_inputs(w, rep, device, shard=None):
+    """One input set on the host: drafter logits, prefix, cache, queries,
+    roots and the target logits (which follow the tree the library builds
+    from the drafter logits).  ``shard``: the request indices to keep."""
     import draft_tree_build_ddtree_b200 as dd
-    sets = []
-    for rep in range(R):
-        z = datagen.drafter_logits(w, rep)
-        prefix = datagen.prefix_lengths(w, rep)
-        cache = datagen.kv_cache(w, prefix, rep)
-        q = datagen.queries(w, rep)
-        root = datagen.root_tokens(w, rep)
-        zd = z.to(device)
-        rootd = root.to(device)
-        # the target logits follow the tree, which the library builds here
-        ids, lp, _ = dd.ddtree_topk(zd.reshape(-1, w.V), w.K)
-        tree = dd.ddtree_build(ids.reshape(w.N, w.L, w.K), lp.reshape(w.N, w.L, w.K), rootd, w.B)
-        tgt = datagen.target_logits(w, z, tree.depth.cpu(), tree.n_nodes.cpu(), rep)
-        rb = dd.RoundBuffers(
-            n_req=w.N, L=w.L, V=w.V, K=w.K, B=w.B,
-            kv=dd.kv_desc_for(cache.k, w.N, w.Hq, cache.block_table),
-            drafter_logits=zd, root_token=rootd, q=q.to(device),
-            k_cache=cache.k.to(device), v_cache=cache.v.to(device),
-            block_table=None if cache.block_table is None else cache.block_table.to(device),
-            prefix_len=prefix.to(device), target_logits=tgt.to(device)).allocate_outputs()
-        rb.args()
-        sets.append(rb)
-        del cache, tgt
-    torch.cuda.synchronize()
-    return sets
+    z = datagen.drafter_logits(w, rep)
+    prefix = datagen.prefix_lengths(w, rep)
+    cache = datagen.kv_cache(w, prefix, rep)
+    q = datagen.queries(w, rep)
+    root = datagen.root_tokens(w, rep)
+    ids, lp, _ = dd.ddtree_topk(z.to(device).reshape(-1, w.V), w.K)
+    tree = dd.ddtree_build(ids.reshape(w.N, w.L, w.K), lp.reshape(w.N, w.L, w.K), root.to(device), w.B)
+    tgt = datagen.target_logits(w, z, tree.depth.cpu(), tree.n_nodes.cpu(), rep)
+    if shard is not None:
+        idx = torch.tensor(shard, dtype=torch.long)
+        z, prefix, root, tgt, q = z[idx], prefix[idx], root[idx], tgt[idx], q[:, idx]
+        if cache.block_table is None:
+            cache = datagen.KVCache(cache.k[:, idx].contiguous(), cache.v[:, idx].contiguous(), None, cache.s_max)
+        else:
+            cache = datagen.KVCache(cache.k, cache.v, cache.block_table[idx].contiguous(), cache.s_max)
+    return dict(z=z, prefix=prefix, cache=cache, q=q.contiguous(), root=root, tgt=tgt.contiguous())
+
+
+def to_round(w, h, device):
+    import draft_tree_build_ddtree_b200 as dd
+    cache = h["cache"]
+    rb = dd.RoundBuffers(
+        n_req=w.N, L=w.L, V=w.V, K=w.K, B=w.B,
+        kv=dd.kv_desc_for(cache.k, w.N, w.Hq, cache.block_table),
+        drafter_logits=h["z"].to(device), root_token=h["root"].to(device), q=h["q"].to(device),
+        k_cache=cache.k.to(device), v_cache=cache.v.to(device),
+        block_table=None if cache.block_table is None else cache.block_table.to(device),
+        prefix_len=h["prefix"].to(device), target_logits=h["tgt"].to(device)).allocate_outputs()
+    rb.args()
+    return rb
 
 
 def algorithmic_work(w, rb):
@@ -313,69 +360,93 @@ def capture(fn, stream):
     return g
 
 
-def run_ours(a):
+def stage_report(w, work, stage_ms, peaks, long_region: bool):
+    """Per-stage µs, achieved bandwidth / flop rate and roof fractions."""
+    hbm = float(peaks["hbm_gbs"])
+    burst = float(peaks["bf16_tflops"])
+    sust = float(peaks.get("bf16_tflops_sustained", burst))
+    tensor_peak = sust if long_region else burst
+    ridge = tensor_peak * 1e12 / (hbm * 1e9)
+    stages = {}
+    for name, t in stage_ms.items():
+        wk = work[name]
+        d = {"us": t * 1e3, "bytes": wk["bytes"], "flops": wk["flops"], "gbs": wk["bytes"] / (t * 1e-3) / 1e9}
+        d["hbm_frac"] = d["gbs"] / hbm
+        if wk["flops"]:
+            d["tflops"] = wk["flops"] / (t * 1e-3) / 1e12
+            d["tensor_frac_burst"] = d["tflops"] / burst
+            d["tensor_frac_sustained"] = d["tflops"] / sust
+            d["intensity"] = wk["flops"] / wk["bytes"]
+            d["bound"] = "tensor" if d["intensity"] > ridge else "hbm"
+        else:
+            d["bound"] = "hbm" if name != "build" else "latency"
+        d["frac"] = (d["tflops"] / tensor_peak) if d["bound"] == "tensor" else d["hbm_frac"]
+        stages[name] = d
+    return stages, tensor_peak
+
+
+def measure(w, a, device, steps, warmup, shard=None, world=1, rank=0, clocks=None, gather=False, keep_host=False):
+    """Build the input sets of ``w`` (this rank's ``shard`` of requests),
+    time ``steps`` rounds and each stage; returns a result dict."""
     import draft_tree_build_ddtree_b200 as dd
-    rank, world, local = dist_env()
-    init_dist(world)
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    w = workload_from_args(a)
-    per_set = set_bytes(w)
+    from draft_tree_build_ddtree_b200 import serving
+    w_run = w if shard is None else dataclasses.replace(w, N=len(shard))
+    per_set = set_bytes(w_run)
     R = max(2, math.ceil(2 * L2_BYTES / per_set) + 1)
-    sets = make_sets(w, R, device)
+    hosts = [host_inputs(w, rep, device, shard) for rep in range(R)]
+    sets = [to_round(w_run, h, device) for h in hosts]
+    host0 = hosts[0] if keep_host else None
+    del hosts
+    torch.cuda.synchronize()
     stream = torch.cuda.current_stream(device)
     use_graph = not a.no_graph
-
-    # one warm eager round per set (one-time library set-up happens outside capture)
-    for rb in sets:
+    for rb in sets:                     # one eager round per set: one-time set-up outside any capture
         dd.ddtree_round(rb, rb._args)
     torch.cuda.synchronize()
+    side = torch.cuda.Stream(device)
     if use_graph:
-        side = torch.cuda.Stream(device)
         graphs = [capture(lambda rb=rb: dd.ddtree_round(rb, rb._args), side) for rb in sets]
-        step = [g.replay for g in graphs]
+        rounds = [g.replay for g in graphs]
     else:
-        step = [lambda rb=rb: dd.ddtree_round(rb, rb._args) for rb in sets]
+        rounds = [lambda rb=rb: dd.ddtree_round(rb, rb._args) for rb in sets]
 
-    for i in range(R):                   # every graph once: its upload happens before any timing
-        step[i]()
+    def step(i):
+        rounds[i % R]()
+        if gather:                      # the batch's per-request outcome, in request order, on every rank
+            rb = sets[i % R]
+            local = torch.stack([rb.acc.accept_len, rb.acc.next_bonus, rb.acc.new_prefix_len], dim=1)
+            serving.gather_by_request(local, w.N, world, rank)
+
+    for i in range(R):                  # every graph once: its upload happens before any timing
+        step(i)
     torch.cuda.synchronize()
-
-    for i in range(a.warmup):
-        step[i % R]()
+    for i in range(warmup):
+        step(i)
     torch.cuda.synchronize()
-
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
-    # ---- the timed region: exactly K steps ----
+    if clocks is not None:
+        clocks.start()
+        time.sleep(0.3)
     barrier(device)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(a.steps):
-        step[i % R]()
+    for i in range(steps):
+        step(i)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(device)
-    clocks.stop()
+    if clocks is not None:
+        clocks.stop()
     ms = e0.elapsed_time(e1)
     ms_max = max_over_ranks(ms, device)
-    value = aggregate_rate(a.steps, world, ms_max / 1e3)
     status = dd.device_status()
 
-    # ---- per-stage kernel times, with cold caches as in the rounds: a graph of
-    #      (L2 flush, stage on set k) for every set, minus the same graph of
-    #      flushes alone ----
-    names = ("topk", "build", "attn", "accept")
+    # per-stage times with cold caches as in the rounds: a graph of (L2 flush,
+    # stage on set k) for every set, minus the same graph of flushes alone
     flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
 
     def timed(fn, n):
-        if use_graph:
-            g = capture(fn, side)
-            run = g.replay
-        else:
-            run = fn
+        run = capture(fn, side).replay if use_graph else fn
         run()
         torch.cuda.synchronize()
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -386,91 +457,134 @@ def run_ours(a):
         torch.cuda.synchronize()
         return t0.elapsed_time(t1)
 
-    reps = max(3, min(20, a.steps // R))
+    reps = max(3, min(20, steps // R))
     t_flush = timed(lambda: [flush_buf.zero_() for _ in range(R)], reps)
     stage_ms = {}
-    for name in names:
-        fns = [stage_calls(w, rb)[name] for rb in sets]
+    for name in ("topk", "build", "attn", "accept"):
+        fns = [stage_calls(w_run, rb)[name] for rb in sets]
 
         def flushed(fns=fns):
             for f in fns:
                 flush_buf.zero_()
                 f()
 
-        stage_ms[name] = max(0.0, timed(flushed, reps) - t_flush) / (reps * R)
+        stage_ms[name] = max(1e-6, timed(flushed, reps) - t_flush) / (reps * R)
     del flush_buf
-    # restore the caches the stage runs compacted are irrelevant: sizes do not change
+    work = algorithmic_work(w_run, sets[0])
+    return dict(w=w_run, sets=sets, R=R, per_set=per_set, ms=ms_max, steps=steps, status=status,
+                stage_ms=stage_ms, work=work, use_graph=use_graph, host0=host0,
+                launches=dd.ddtree_round_launch_count(sets[0], sets[0]._args),
+                accept_len_mean=float(torch.cat([rb.acc.accept_len.float() for rb in sets]).mean().item()))
 
-    work = algorithmic_work(w, sets[0])
+
+def run_ours(a):
+    import draft_tree_build_ddtree_b200 as dd
+    from draft_tree_build_ddtree_b200 import serving
+    rank, world, local = dist_env()
+    if world != a.gpus:
+        raise SystemExit(f"bench.py: --gpus {a.gpus} but WORLD_SIZE is {world}")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    init_dist(world)
+    w = workload_from_args(a)
+    sharded = w.N > 1 and world > 1          # the batched workload splits by request
+    shard = serving.shard_of(w.N, world, rank) if sharded else None
+    clocks = ClockSampler(local)
+    m = measure(w, a, device, a.steps, a.warmup, shard=shard, world=world, rank=rank, clocks=clocks,
+                gather=sharded, keep_host=(rank == 0 and world == 1 and not a.no_cpu_baseline))
+    if sharded:
+        value = a.steps / (m["ms"] / 1e3)    # whole-batch rounds per second
+    else:
+        value = aggregate_rate(a.steps, world, m["ms"] / 1e3)
     peaks, peak_kind = load_peaks()
-    hbm = float(peaks["hbm_gbs"])
-    tflops = float(peaks["bf16_tflops"])
-    ridge = tflops * 1e12 / (hbm * 1e9)
-    stages = {}
-    for name, t in stage_ms.items():
-        wk = work[name]
-        d = {"us": t * 1e3, "bytes": wk["bytes"], "flops": wk["flops"],
-             "gbs": wk["bytes"] / (t * 1e-3) / 1e9}
-        d["hbm_frac"] = d["gbs"] / hbm
-        if wk["flops"]:
-            d["tflops"] = wk["flops"] / (t * 1e-3) / 1e12
-            d["tensor_frac"] = d["tflops"] / tflops
-            d["intensity"] = wk["flops"] / wk["bytes"]
-        stages[name] = d
+    long_region = m["ms"] / 1e3 >= SUSTAINED_AFTER_S
+    stages, tensor_peak = stage_report(m["w"], m["work"], m["stage_ms"], peaks, long_region)
     dom = max((n for n in stages if n != "build"), key=lambda n: stages[n]["us"])
     ds = stages[dom]
-    if dom == "attn" and ds["intensity"] > ridge:
-        roof = {"bound": "tensor", "achieved": ds["tflops"], "peak": tflops, "unit": "TFLOP/s",
-                "frac": ds["tflops"] / tflops}
+    if ds["bound"] == "tensor":
+        roof = {"bound": "tensor", "achieved": ds["tflops"], "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": ds["tflops"] / tensor_peak}
     else:
-        roof = {"bound": "hbm", "achieved": ds["gbs"], "peak": hbm, "unit": "GB/s", "frac": ds["gbs"] / hbm}
-    roof.update({"kernel": dom, "traffic": measured_traffic(w.name, dom), "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst)"
-                 if peak_kind == "measured" else "fallback"})
+        roof = {"bound": "hbm", "achieved": ds["gbs"], "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "frac": ds["gbs"] / float(peaks["hbm_gbs"])}
+    roof.update({"kernel": dom, "traffic": measured_traffic(w.name, dom),
+                 "peak_source": (f"of {peak_kind} (MEASURED_PEAKS.json "
+                                 f"{'sustained' if long_region and ds['bound'] == 'tensor' else 'burst'})")})
 
-    # ---- end to end through the host-buffer API ----
+    # ---- end to end through the C ABI's host-buffer round ----
     e2e = None
     if not a.no_e2e:
         from draft_tree_build_ddtree_b200 import host_api
-        hosts = [host_api.make_host_round(rb) for rb in sets]
-        k_e2e = max(3, min(a.steps, 200))
-        for i in range(2):
-            host_api.round_from_host(sets[i % R], hosts[i % R], sets[i % R]._args)
+        sets, R = m["sets"], m["R"]
+        hosts = [host_api.make_host_round(rb, rb._args) for rb in sets]
+        k_e2e = max(3, min(a.steps, 100))
+        stream = torch.cuda.current_stream(device)
+        for i in range(R):
+            host_api.round_from_host(sets[i], hosts[i], sets[i]._args)
         torch.cuda.synchronize()
         barrier(device)
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(stream)
         for i in range(k_e2e):
             host_api.round_from_host(sets[i % R], hosts[i % R], sets[i % R]._args)
+            if sharded:
+                rb = sets[i % R]
+                serving.gather_by_request(torch.stack([rb.acc.accept_len, rb.acc.next_bonus,
+                                                       rb.acc.new_prefix_len], dim=1), w.N, world, rank)
         f1.record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(f0.elapsed_time(f1), device)
-        e2e = {"value": aggregate_rate(k_e2e, world, e_ms / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": hosts[0].h2d_bytes, "d2h_bytes_per_step": hosts[0].d2h_bytes,
-               "steps": k_e2e}
+        e_val = k_e2e / (e_ms / 1e3) if sharded else aggregate_rate(k_e2e, world, e_ms / 1e3)
+        e2e = {"value": e_val, "unit": UNIT, "h2d_bytes_per_step": hosts[0].h2d_bytes,
+               "d2h_bytes_per_step": hosts[0].d2h_bytes, "steps": k_e2e,
+               "api": "ddtree_round_host (C ABI): pinned host inputs, round, host results"}
+        del hosts
 
-    launches_per_round = dd.ddtree_round_launch_count(sets[0], sets[0]._args)
+    per_config = None
+    if world == 1 and not a.no_per_config:
+        per_config = {}
+        for cfg, over in PER_CONFIG:
+            wc = workload_of(cfg, over)
+            if wc.name == w.name:
+                continue
+            mc = measure(wc, a, device, max(50, min(a.steps, 500)), max(3, a.warmup))
+            long_c = mc["ms"] / 1e3 >= SUSTAINED_AFTER_S
+            st_c, _ = stage_report(mc["w"], mc["work"], mc["stage_ms"], peaks, long_c)
+            per_config[wc.name] = {
+                "workload": workload_label(wc), "rounds_per_s": mc["steps"] / (mc["ms"] / 1e3),
+                "ms_per_round": mc["ms"] / mc["steps"], "steps": mc["steps"], "device_status": mc["status"],
+                "stages_us": {k: round(v["us"], 3) for k, v in st_c.items()},
+                "roof": {k: {kk: v[kk] for kk in ("bound", "frac", "hbm_frac", "tensor_frac_burst",
+                                                  "tensor_frac_sustained", "gbs", "tflops") if kk in v}
+                         for k, v in st_c.items()},
+                "accept_len_mean": mc["accept_len_mean"]}
+            del mc
+            torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        cpu = cpu_baseline(w, budget_s=12.0)
+        cpu = cpu_baseline(w, m["host0"], budget_s=15.0)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
-            "warmup": a.warmup, "ms_per_step": ms_max / a.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": workload_label(w),
-                       "config_id": w.cfg, "n_req": w.N, "parallelism": f"replicas x{world}",
-                       "l2": f"{R} rotating input sets of {per_set / 1e6:.1f} MB (> 2x L2)",
-                       "launch": "cuda graph per round" if use_graph else "eager"},
+            "warmup": a.warmup, "ms_per_step": m["ms"] / a.steps, "higher_is_better": True,
+            "scaling": "strong" if sharded else "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": workload_label(w), "config_id": w.cfg, "n_req": w.N,
+                       "parallelism": (f"requests sharded over {world} ranks (r mod {world})" if sharded
+                                       else f"replicas x{world}"),
+                       "l2": f"{m['R']} rotating input sets of {m['per_set'] / 1e6:.1f} MB (> 2x L2)",
+                       "launch": "cuda graph per round" if m["use_graph"] else "eager"},
             "stages_us": {k: round(v["us"], 3) for k, v in stages.items()},
             "stages": stages,
             "roofline": roof,
-            "gpu_launches": launches_per_round * a.steps,
+            "gpu_launches": m["launches"] * a.steps,
             "clocks": clocks.summary(),
             "e2e": e2e,
             "cpu_baseline": cpu,
-            "device_status": status,
-            "accept_len_mean": float(sets[0].acc.accept_len.float().mean().item()),
+            "per_config": per_config,
+            "device_status": m["status"],
+            "accept_len_mean": m["accept_len_mean"],
         }
         print(json.dumps(line))
     if torch.distributed.is_initialized():
@@ -479,91 +593,90 @@ def run_ours(a):
 
 # ---------------------------------------------------------------- the oracle (CPU baseline / reference arm)
 
-def oracle_round_sample(w, z, root, q, cache, prefix, tgt, frac_rows=1, node_limit=None, head_limit=None,
-                        layer_limit=None):
-    """Time the oracle on a sample of one round; return extrapolated seconds per round and a description."""
+def oracle_sample(w):
+    """The part of one round the oracle runs in a timed step, and the factor
+    that scales each stage's time to the full round.  The dense attention is
+    the slow part (8 ms per node and head at P = 8192): configs 1 and 2 run
+    in full, the larger ones on a stated subset."""
+    if w.cfg in (1, 2):
+        return dict(reqs=list(range(w.N)), layers=None, heads=None)
+    if w.cfg == 4:
+        return dict(reqs=[0, 1, 2, 3], layers=None, heads=[0, 16])
+    return dict(reqs=[0], layers=[0], heads=[0])
+
+
+def oracle_round(w, h, sample):
+    """The oracle on one round's real inputs (``h``: the host copy of an
+    input set): top-K of the sampled requests' rows, their heaps, dense
+    attention on the sampled layers and heads (every node), the target
+    argmax of every live node, the walk, and the compaction of every layer.
+    Returns (seconds scaled to the full round, per-stage seconds, description)."""
     import oracle
+    reqs = sample["reqs"]
+    n_r = len(reqs)
+    idx = torch.tensor(reqs, dtype=torch.long)
+    z = h["z"][idx].to(torch.float64).numpy()
     t = {}
-    rows = z.reshape(-1, w.V)
-    nrows = rows.shape[0]
-    take = max(1, min(nrows, frac_rows))
     t0 = time.perf_counter()
-    ids, lp32, _, _ = oracle.topk(rows[:take].to(torch.float64).numpy(), w.K)
-    t["topk"] = (time.perf_counter() - t0) * nrows / take
-    # the heap runs on the full table of request 0 (cheap); use the sampled rows' table tiled
-    full_ids = np.tile(ids, (math.ceil(w.L / take), 1))[:w.L]
-    full_lp = np.sort(np.tile(lp32, (math.ceil(w.L / take), 1))[:w.L], axis=1)[:, ::-1].copy()
+    ids, lp32, _, _ = oracle.topk(z, w.K)
+    t["topk"] = time.perf_counter() - t0
+    root = h["root"][idx].numpy()
     t0 = time.perf_counter()
-    tree = oracle.build_tree(full_ids, full_lp, int(root[0]), w.B)
-    t["build"] = (time.perf_counter() - t0) * w.N
-    st = oracle.stack_trees([tree])
-    nodes = list(range(tree.n_nodes))[:node_limit] if node_limit else None
-    heads = list(range(w.Hq))[:head_limit] if head_limit else None
-    layers = list(range(w.layers))[:layer_limit] if layer_limit else None
-    qq = q[:, :1].to(torch.float64).numpy()
-    kk = cache.k[:, :1].to(torch.float64).numpy() if cache.block_table is None else None
-    vv = cache.v[:, :1].to(torch.float64).numpy() if cache.block_table is None else None
-    if kk is None:
-        # paged pools: gather request 0's logical slots into a contiguous view
-        tb = cache.block_table[0]
-        S = int(prefix[0]) + w.n
-        nb = (S + 63) // 64
-        kk = cache.k[:, tb[:nb].long()].reshape(w.layers, 1, nb * 64, w.Hkv, w.D).to(torch.float64).numpy()
-        vv = cache.v[:, tb[:nb].long()].reshape(w.layers, 1, nb * 64, w.Hkv, w.D).to(torch.float64).numpy()
+    trees = oracle.build_trees(ids, lp32, root, w.B)
+    t["build"] = time.perf_counter() - t0
+    st = oracle.stack_trees(trees)
+    prefix = h["prefix"][idx].numpy()
+    cache = h["cache"]
+    layers = list(range(w.layers)) if sample["layers"] is None else sample["layers"]
+    t["attn"] = 0.0
+    for l in layers:
+        if cache.block_table is None:
+            kk = cache.k[l:l + 1, idx].to(torch.float64).numpy()
+            vv = cache.v[l:l + 1, idx].to(torch.float64).numpy()
+        else:       # the sampled requests' pages gathered into contiguous rows
+            S = int(prefix.max()) + w.n
+            nb = (S + 63) // 64
+            tb = cache.block_table[idx, :nb].clamp(min=0).long()
+            kk = cache.k[l][tb].reshape(1, n_r, nb * 64, w.Hkv, w.D).to(torch.float64).numpy()
+            vv = cache.v[l][tb].reshape(1, n_r, nb * 64, w.Hkv, w.D).to(torch.float64).numpy()
+        qq = h["q"][l:l + 1, idx].to(torch.float64).numpy()
+        t0 = time.perf_counter()
+        oracle.tree_attention(qq, kk, vv, prefix, st["anc"], st["n_nodes"], datagen.default_scale(w),
+                              heads=sample["heads"])
+        t["attn"] += time.perf_counter() - t0
+    tgt = h["tgt"][idx].to(torch.float32).numpy()
+    kb = cache.k.view(torch.int16).numpy() if w.dtype == "bf16" else cache.k.numpy()
+    vb = cache.v.view(torch.int16).numpy() if w.dtype == "bf16" else cache.v.numpy()
+    table = None if cache.block_table is None else cache.block_table.numpy()
     t0 = time.perf_counter()
-    oracle.tree_attention(qq, kk, vv, prefix[:1].numpy(), st["anc"], st["n_nodes"], datagen.default_scale(w),
-                          layers=layers, nodes=nodes, heads=heads)
-    frac = (len(layers) if layers else w.layers) * (len(nodes) if nodes else tree.n_nodes) * \
-        (len(heads) if heads else w.Hq) / (w.layers * tree.n_nodes * w.Hq)
-    t["attn"] = (time.perf_counter() - t0) / frac * w.N
-    # walk: target argmax on a sample of the node rows (scaled), then the walk
-    # and the compaction of the accepted path over every layer
-    arows = min(tree.n_nodes, frac_rows if w.cfg == 1 else 2)
-    t0 = time.perf_counter()
-    oracle.argmax_rows(tgt[0, :arows].to(torch.float32).numpy())
-    t_arg = (time.perf_counter() - t0) * tree.n_nodes / arows
-    tg = np.zeros((tree.n_nodes, 4))
-    for i in range(1, tree.n_nodes):      # a target that follows the deepest branch
-        tg[st["parent"][0][i], 0] = 0.0
-    t0 = time.perf_counter()
-    acc = oracle.accept(tg, st["node_token"][0], st["parent"][0], tree.n_nodes, w.L, int(prefix[0]))
-    oracle.compact(kk, vv, 0, acc)
-    t["accept"] = (t_arg + time.perf_counter() - t0) * w.N
-    desc = (f"request 0 of {w.N}; top-K on {take}/{nrows} rows; full heap; attention on "
-            f"{len(layers) if layers else w.layers}/{w.layers} layers x {len(nodes) if nodes else tree.n_nodes}/"
-            f"{tree.n_nodes} nodes x {len(heads) if heads else w.Hq}/{w.Hq} heads; target argmax on {arows}/"
-            f"{tree.n_nodes} rows; walk + compaction; "
-            f"each stage scaled to the full round")
-    return sum(t.values()), t, desc
+    for j, r in enumerate(reqs):
+        acc = oracle.accept(tgt[j], st["node_token"][j], st["parent"][j], int(st["n_nodes"][j]), w.L, int(prefix[j]))
+        oracle.compact(kb, vb, r, acc, block_table=table)
+    t["accept"] = time.perf_counter() - t0
+    heads = w.Hq if sample["heads"] is None else len(sample["heads"])
+    f_req = w.N / n_r
+    f_attn = f_req * (w.layers / len(layers)) * (w.Hq / heads)
+    full = (t["topk"] + t["build"] + t["accept"]) * f_req + t["attn"] * f_attn
+    desc = (f"real inputs of one round; requests {n_r}/{w.N}: top-K of all their rows, full heap, target argmax of "
+            f"every live node, walk, compaction of all {w.layers} layers; dense attention on "
+            f"{len(layers)}/{w.layers} layers x {heads}/{w.Hq} query heads x every node"
+            + ("" if f_attn == 1.0 else f"; attention time x{f_attn:g} and the rest x{f_req:g} to the full round"))
+    return full, t, desc
 
 
-def sample_limits(w):
-    """Sample sizes that keep one oracle step to tens of milliseconds."""
-    if w.cfg == 1:
-        return dict(frac_rows=w.N * w.L)
-    return dict(frac_rows=1, node_limit=2, head_limit=2, layer_limit=1)
-
-
-def cpu_baseline(w, budget_s=12.0):
+def cpu_baseline(w, h, budget_s=15.0):
     from threadpoolctl import threadpool_limits
-    z = datagen.drafter_logits(w)
-    prefix = datagen.prefix_lengths(w)
-    cache = datagen.kv_cache(w, prefix)
-    q = datagen.queries(w)
-    root = datagen.root_tokens(w)
-    tgt = datagen.target_logits(w, z, torch.zeros(w.N, w.n, dtype=torch.int32),
-                                torch.full((w.N,), w.n, dtype=torch.int32))
-    lim = sample_limits(w)
-    secs, n = [], 0
+    sample = oracle_sample(w)
+    secs, n, desc = [], 0, ""
     with threadpool_limits(limits=1):
         t_end = time.perf_counter() + budget_s
-        while n < 1 or (time.perf_counter() < t_end and n < 50):
-            s, _, desc = oracle_round_sample(w, z, root, q, cache, prefix, tgt, **lim)
+        while n < 1 or (time.perf_counter() < t_end and n < 20):
+            s, _, desc = oracle_round(w, h, sample)
             secs.append(s)
             n += 1
     per_round = statistics.median(secs)
     return {"value": 1.0 / per_round, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n} sampled rounds ({desc}); numpy/BLAS limited to 1 thread"}
+            "sample": f"{n} timed oracle rounds ({desc}); numpy/BLAS limited to 1 thread"}
 
 
 def run_reference(a):
@@ -577,23 +690,33 @@ def run_reference(a):
     cache = datagen.kv_cache(w, prefix)
     q = datagen.queries(w)
     root = datagen.root_tokens(w)
-    tgt = datagen.target_logits(w, z, torch.zeros(w.N, w.n, dtype=torch.int32),
-                                torch.full((w.N,), w.n, dtype=torch.int32))
-    lim = sample_limits(w)
+    # the target rows follow the oracle's own tree on this host (no GPU here)
+    import oracle
+    ids, lp32, _, _ = oracle.topk(z.to(torch.float64).numpy(), w.K)
+    st = oracle.stack_trees(oracle.build_trees(ids, lp32, root.numpy(), w.B))
+    tgt = datagen.target_logits(w, z, torch.from_numpy(st["depth"]), torch.from_numpy(st["n_nodes"]))
+    h = dict(z=z, prefix=prefix, cache=cache, q=q, root=root, tgt=tgt)
+    sample = oracle_sample(w)
+    desc = ""
     with threadpool_limits(limits=1):
         for _ in range(a.warmup):
-            oracle_round_sample(w, z, root, q, cache, prefix, tgt, **lim)
-        secs = []
-        desc = ""
+            oracle_round(w, h, sample)
+        step_s, full_s = [], []
         for _ in range(a.steps):
-            s, _, desc = oracle_round_sample(w, z, root, q, cache, prefix, tgt, **lim)
-            secs.append(s)
-    total = sum(secs)
+            t0 = time.perf_counter()
+            full, _, desc = oracle_round(w, h, sample)
+            step_s.append(time.perf_counter() - t0)
+            full_s.append(full)
+    total = sum(step_s)
     value = a.steps / total
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": total / a.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": workload_label(w), "config_id": w.cfg, "n_req": w.N},
+            "step": f"one oracle round on the stated sample: {desc}",
+            "extrapolated_full_round": {"rounds_per_s": a.steps / sum(full_s),
+                                        "ms_per_round": sum(full_s) / a.steps * 1e3,
+                                        "method": "each stage's sampled time scaled by its sample fraction"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": f"each step: {desc}; numpy/BLAS limited to 1 thread"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -610,15 +733,18 @@ def run_profile(a):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     w = workload_from_args(a)
-    rb = make_sets(w, 1, device)[0]
+    rb = to_round(w, host_inputs(w, 0, device), device)
     for _ in range(a.warmup + a.steps):
         dd.ddtree_round(rb, rb._args)
     torch.cuda.synchronize()
     print(json.dumps({"profile_run": w.name, "rounds": a.warmup + a.steps, "device_status": dd.device_status()}))
 
 
-def main():
-    a = parse()
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
+    a = parse(argv)
+    if a.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(subprocess.call(relaunch_cmd(argv, a.gpus, free_port())))
     if a.impl == "reference":
         run_reference(a)
     elif a.profile:

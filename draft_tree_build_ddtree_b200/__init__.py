@@ -87,6 +87,9 @@ _SIGS = {
     "ddtree_version": (_i, []),
     "ddtree_topk_static_ws": (_i, [_vp, _i, _i, _i, _ll, _i, _vp, _vp, _vp, _vp]),
     "ddtree_debug_attn_timeout": (_i, [ctypes.c_ulonglong, _i]),
+    "ddtree_round_host": (_i, [ctypes.POINTER(RoundArgs), _vp, _vp]),
+    "ddtree_round_host_bytes": (_i, [ctypes.POINTER(RoundArgs), _vp, ctypes.POINTER(ctypes.c_ulonglong),
+                                     ctypes.POINTER(ctypes.c_ulonglong)]),
 }
 
 

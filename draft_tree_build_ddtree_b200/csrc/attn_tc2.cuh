@@ -1,0 +1,591 @@
+// Stage 3, long key ranges: ancestor-only GQA tree attention with two M-tiles
+// per CTA sharing every K/V tile, and P kept in tensor memory.
+//
+// "DDTree Deep Dive" §4 (a tree node attends to the committed prefix, the
+// root, its ancestors and itself).  Same rows, mask and arithmetic as
+// tree_attn_tc_kernel; what differs is how the work meets the hardware.
+//
+// Why: at full tensor-core rate the single-M-tile kernel would move about
+// 250 bytes per clock through each SM's shared memory (the TMA writes of
+// every K/V tile per 128 rows, the Q operand re-read by every QK^T step, P
+// written by the softmax and read back by the PV product), against the
+// roughly 128 bytes per clock that shared memory serves.  Here:
+//   * two M-tiles (256 rows) per CTA share each 128-key K/V tile, halving
+//     the TMA traffic per flop;
+//   * QK^T runs at N = 128 keys (one A and one B operand of 4 KB per K=16
+//     step and 64 clocks of tensor work);
+//   * P is written by the softmax into tensor memory over its own S columns
+//     and read from there as the A operand of O += P V (tcgen05.mma with A in
+//     TMEM), so P never touches shared memory.
+// That is about 125 bytes per clock per SM at full rate.
+//
+// Tensor memory (512 columns): S0|P0 [0,128), S1|P1 [128,256), O0 [256,384),
+// O1 [384,512).  P(j) of M-tile t is stored as packed bf16 pairs in the first
+// 64 columns of S_t: column c of a lane holds keys 2c and 2c+1 of that row.
+//
+// Warps (320 threads): 0-3 softmax of M-tile 0, 4-7 softmax of M-tile 1 (a
+// thread owns one row = one TMEM lane), 8 the TMA producer, 9 TMEM
+// allocation and the single-thread MMA issuer.  The MMA issue order per key
+// tile j is PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): the tensor pipe computes one
+// M-tile's products while the other M-tile's softmax runs.  tcgen05
+// operations issued by one thread complete in issue order, so
+//   * S_t(j+1) overwriting P_t(j) runs after PV_t(j) has read it, and
+//   * when a softmax sees S_t(j) complete, PV_t(j-1) has completed too: the
+//     softmax may then rescale O_t in place (no product is writing it).
+// O is rescaled only when the running max grows by more than 2^8, as in the
+// single-tile kernel.  Every mbarrier wait is bounded; on timeout the kernel
+// flags DDTREE_STATUS_TIMEOUT, every role leaves its loop, waits (bounded)
+// for its copies and products in flight and frees the tensor memory.  No TMA
+// multicast is used.
+#pragma once
+
+#include "attn_tc.cuh"
+
+namespace ddt {
+
+constexpr int T2_THREADS = 320;
+constexpr int T2_BN = 128;                          // keys per tile
+constexpr int T2_KATOM = T2_BN * 64 * 2;            // [128 keys][64 dims] bf16: 16 KB
+constexpr int T2_KTILE = 2 * T2_KATOM;              // [128 keys][128 dims]: 32 KB
+constexpr int T2_STAGES = 2;
+constexpr uint32_t T2_TMEM_COLS = 512;
+
+struct T2Smem {
+  unsigned char q[2][TC_TILE];
+  unsigned char k[T2_STAGES][T2_KTILE];
+  unsigned char v[T2_STAGES][T2_KTILE];
+  uint64_t bar_q, bar_kf[T2_STAGES], bar_ke[T2_STAGES], bar_vf[T2_STAGES], bar_ve[T2_STAGES];
+  uint64_t bar_sfull[2], bar_pready[2], bar_odone;
+  uint32_t tmem_base;
+  int abort;
+  int lpt_r;
+};
+
+constexpr size_t t2_smem_bytes() { return sizeof(T2Smem); }
+
+// D[tmem] (+)= A[tmem] * B[smem]: kind::f16 with the A operand in tensor memory.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+struct T2Params {
+  AttnGeom g;
+  int G;               // query heads per KV head
+  int mtiles;          // M-tiles per (layer, request, KV head)
+  int mpairs;          // CTAs' M-tile groups per (layer, request, KV head): ceil(mtiles / nq)
+  int nq;              // M-tiles per CTA (1 or 2)
+  int splits;
+  int units;           // layers * n_req * Hkv * mpairs
+  const int32_t* block_table;
+  const int32_t* prefix_len;
+  const uint32_t* anc;
+  const int32_t* n_nodes;
+  __nv_bfloat16* out;
+  float* out_lse;
+  float* ws_o;         // partials per (M-tile unit, split), as for the combine kernel
+  float2* ws_ml;
+  int lpt;
+  uint64_t wait_ns;
+  int stop_tile;
+};
+
+__global__ void __maxnreg__(200)
+tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const T2Params p) {
+  extern __shared__ __align__(1024) unsigned char smem_dyn[];
+  T2Smem& sm = *reinterpret_cast<T2Smem*>(smem_dyn);
+  if ((smem_u32(smem_dyn) & 1023u) != 0u) {       // the 128B-swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) flag_status(DDTREE_STATUS_SETUP);
+    return;
+  }
+  const AttnGeom& g = p.g;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  // ---- which unit ----
+  const int split = blockIdx.x % p.splits;
+  int u = blockIdx.x / p.splits;
+  const int mp = u % p.mpairs; u /= p.mpairs;
+  const int kvh = u % g.Hkv; u /= g.Hkv;
+  int r = u % g.n_req; u /= g.n_req;
+  const int layer = u;
+  if (p.lpt) {     // ragged batch: longest key range first (see tree_attn_tc_kernel)
+    const int r_slot = r;
+    for (int i = tid; i < g.n_req; i += T2_THREADS) {
+      const int ki = p.prefix_len[i] + p.n_nodes[i];
+      int rank = 0;
+      for (int j = 0; j < g.n_req; ++j) {
+        const int kj = p.prefix_len[j] + p.n_nodes[j];
+        rank += (kj > ki) || (kj == ki && j < i);
+      }
+      if (rank == r_slot) sm.lpt_r = i;
+    }
+    __syncthreads();
+    r = sm.lpt_r;
+  }
+  const int nodes_per_tile = TC_BM / p.G;
+  const int mt0 = mp * p.nq;                          // first M-tile of this CTA
+  const int nn = p.n_nodes[r];
+  const int node_base = mt0 * nodes_per_tile;
+  if (node_base >= nn) return;                        // no live node in this CTA's M-tiles
+  // M-tiles of this CTA holding a live node (1 or 2)
+  const int ntl = (p.nq == 2 && node_base + nodes_per_tile < nn && mt0 + 1 < p.mtiles) ? 2 : 1;
+  const int P = p.prefix_len[r];
+  const long long cap = g.paged ? (long long)g.max_blocks * DDTREE_PAGE : (long long)g.s_max;
+  if (P < 0 || (long long)P + nn > cap) {
+    if (tid == 0 && mp == 0 && kvh == 0 && split == 0) flag_status(DDTREE_STATUS_CAPACITY);
+    return;
+  }
+  if (g.paged) {
+    const int nb = (P + nn + DDTREE_PAGE - 1) / DDTREE_PAGE;
+    int bad = 0;
+    for (int b = tid; b < nb; b += T2_THREADS) {
+      const int blk = p.block_table[(size_t)r * g.max_blocks + b];
+      bad |= (blk < 0 || blk >= g.num_blocks);
+    }
+    if (__syncthreads_or(bad)) {
+      if (tid == 0 && mp == 0 && kvh == 0 && split == 0) flag_status(DDTREE_STATUS_CAPACITY);
+      return;
+    }
+  }
+  const int T = P + nn;
+  const int ntiles = (T + T2_BN - 1) / T2_BN;
+  const int per = (ntiles + p.splits - 1) / p.splits;
+  const int t_begin = split * per;
+  const int t_end = min(ntiles, t_begin + per);
+  const int nt = max(0, t_end - t_begin);
+
+  if (tid == 0) {
+    mbar_init(&sm.bar_q, 1);
+    for (int s = 0; s < T2_STAGES; ++s) {
+      mbar_init(&sm.bar_kf[s], 1);
+      mbar_init(&sm.bar_ke[s], 1);
+      mbar_init(&sm.bar_vf[s], 1);
+      mbar_init(&sm.bar_ve[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&sm.bar_sfull[t], 1);
+      mbar_init(&sm.bar_pready[t], 128);
+    }
+    mbar_init(&sm.bar_odone, 1);
+    sm.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 9) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
+                 "r"(T2_TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+  const float sl2 = g.scale * 1.4426950408889634f;   // scale * log2(e)
+  const uint64_t wlim = p.wait_ns;
+
+  if (warp == 8) {
+    // =========================== TMA producer ===========================
+    if (lane == 0 && nt > 0) {
+      const int qb = layer * g.n_req + r;
+      mbar_expect_tx(&sm.bar_q, (uint32_t)(ntl * TC_TILE));
+      for (int t = 0; t < ntl; ++t) {
+        const int nd = node_base + t * nodes_per_tile;
+        tma_load_4d(smem_u32(sm.q[t]), &tm_q, &sm.bar_q, 0, kvh * p.G, nd, qb);
+        tma_load_4d(smem_u32(sm.q[t] + TC_ATOM), &tm_q, &sm.bar_q, 64, kvh * p.G, nd, qb);
+      }
+      int issued = 0;
+      for (int jj = 0; jj < nt; ++jj) {
+        if (jj == p.stop_tile) break;      // diagnostics: withhold the rest, a consumer wait runs out
+        const int j = t_begin + jj;
+        const int st = jj % T2_STAGES;
+        const int use = jj / T2_STAGES;
+        const int k0 = j * T2_BN;
+        int b0 = 0, b1 = 0;
+        if (g.paged) {     // the tile's two pages; a second page past the validated range reuses the first (masked)
+          const int pg = k0 / DDTREE_PAGE;
+          const int maxpg = (T + DDTREE_PAGE - 1) / DDTREE_PAGE;
+          b0 = p.block_table[(size_t)r * g.max_blocks + pg];
+          b1 = (pg + 1 < maxpg) ? p.block_table[(size_t)r * g.max_blocks + pg + 1] : b0;
+        }
+        auto load_tile = [&](const CUtensorMap* map, unsigned char* tile, uint64_t* bar) {
+          mbar_expect_tx(bar, T2_KTILE);
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t dst = smem_u32(tile + h * T2_KATOM);
+            if (!g.paged) {
+              tma_load_4d(dst, map, bar, 64 * h, kvh, k0, layer * g.n_req + r);
+            } else {
+              tma_load_4d(dst, map, bar, 64 * h, kvh, 0, layer * g.num_blocks + b0);
+              tma_load_4d(dst + T2_KATOM / 2, map, bar, 64 * h, kvh, 0, layer * g.num_blocks + b1);
+            }
+          }
+        };
+        if (use > 0 && !mbar_wait(&sm.bar_ke[st], (use - 1) & 1, abort, wlim)) break;
+        load_tile(&tm_k, sm.k[st], &sm.bar_kf[st]);
+        if (use > 0 && !mbar_wait(&sm.bar_ve[st], (use - 1) & 1, abort, wlim)) break;
+        load_tile(&tm_v, sm.v[st], &sm.bar_vf[st]);
+        issued = jj + 1;
+      }
+      if (*abort || issued < nt) {       // copies in flight must land before the CTA exits
+        int z = 0;
+        mbar_wait(&sm.bar_q, 0, (volatile int*)&z);
+        for (int jj = max(0, issued - T2_STAGES); jj < issued; ++jj) {
+          mbar_wait(&sm.bar_kf[jj % T2_STAGES], (jj / T2_STAGES) & 1, (volatile int*)&z);
+          mbar_wait(&sm.bar_vf[jj % T2_STAGES], (jj / T2_STAGES) & 1, (volatile int*)&z);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // =========================== MMA issuer ===========================
+    if (lane == 0 && nt > 0) {
+      constexpr uint32_t IDESC_QK = idesc_bf16_f32(TC_BM, T2_BN, false, false);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(TC_BM, TC_D, false, true);
+      bool ok = mbar_wait(&sm.bar_q, 0, abort, wlim);
+      bool any_commit = false;
+      auto issue_s = [&](int t, int st) {      // S_t = Q_t K^T over the 128 head dims
+        const uint32_t q_addr = smem_u32(sm.q[t]), k_addr = smem_u32(sm.k[st]);
+#pragma unroll
+        for (int kk = 0; kk < TC_D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * TC_ATOM + (kk & 3) * 32;
+          const uint32_t koff = (kk >> 2) * T2_KATOM + (kk & 3) * 32;
+          umma_f16(tmem + 128 * t, smem_desc_sw128(q_addr + off, 16, 1024),
+                   smem_desc_sw128(k_addr + koff, 16, 1024), IDESC_QK, kk > 0);
+        }
+        umma_commit(&sm.bar_sfull[t]);
+      };
+      auto issue_pv = [&](int t, int st, int jj) {   // O_t += P_t V over the 128 keys
+        const uint32_t v_addr = smem_u32(sm.v[st]);
+#pragma unroll
+        for (int kk = 0; kk < T2_BN / 16; ++kk)
+          umma_f16_ts(tmem + 256 + 128 * t, tmem + 128 * t + kk * 8,
+                      smem_desc_sw128(v_addr + kk * 16 * 128, T2_KATOM, 1024), IDESC_PV, (jj > 0 || kk > 0));
+      };
+      if (ok && mbar_wait(&sm.bar_kf[0], 0, abort, wlim)) {
+        tc_fence_after();
+        for (int t = 0; t < ntl; ++t) issue_s(t, 0);
+        umma_commit(&sm.bar_ke[0]);
+        any_commit = true;
+      } else {
+        ok = false;
+      }
+      for (int jj = 0; ok && jj < nt; ++jj) {
+        const int st = jj % T2_STAGES;
+        const int st1 = (jj + 1) % T2_STAGES;
+        const bool more = jj + 1 < nt;
+        if (!mbar_wait(&sm.bar_vf[st], (jj / T2_STAGES) & 1, abort, wlim)) break;
+        bool kready = false;
+        for (int t = 0; t < ntl; ++t) {
+          if (!mbar_wait(&sm.bar_pready[t], jj & 1, abort, wlim)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(t, st, jj);
+          if (more) {
+            if (!kready) {
+              if (!mbar_wait(&sm.bar_kf[st1], ((jj + 1) / T2_STAGES) & 1, abort, wlim)) { ok = false; break; }
+              tc_fence_after();
+              kready = true;
+            }
+            issue_s(t, st1);
+          }
+        }
+        if (!ok) break;
+        umma_commit(&sm.bar_ve[st]);
+        if (more) umma_commit(&sm.bar_ke[st1]);
+      }
+      if (ok) {
+        umma_commit(&sm.bar_odone);
+      } else if (any_commit) {
+        // products in flight must retire before the tensor memory is freed:
+        // a commit to a fresh phase of O-done tracks every earlier product
+        umma_commit(&sm.bar_odone);
+        int z = 0;
+        mbar_wait(&sm.bar_odone, 0, (volatile int*)&z);
+      }
+    }
+  } else {
+    // =========================== softmax warps ===========================
+    const int t = warp >> 2;                               // M-tile of this warpgroup
+    const int row = tid & 127;                             // TMEM lane == M row
+    const int node = node_base + t * nodes_per_tile + row / p.G;
+    const int hq = kvh * p.G + row % p.G;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tm_s = tmem + 128 * t + lane_off;
+    const uint32_t tm_o = tmem + 256 + 128 * t + lane_off;
+    const uint32_t* arow = p.anc + ((size_t)r * g.n + min(node, g.n - 1)) * g.W;
+    float m_used = -INFINITY;
+    float l = 0.f;
+    bool ok = t < ntl;
+    for (int jj = 0; ok && jj < nt; ++jj) {
+      const int k0 = (t_begin + jj) * T2_BN;
+      // tcgen05.ld/st are warp-collective: every exit and branch around them is warp-uniform
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull[t], jj & 1, abort, wlim))) { ok = false; break; }
+      tc_fence_after();
+      float s[T2_BN];
+#pragma unroll
+      for (int c = 0; c < T2_BN / 32; ++c) tmem_ld32(tm_s + c * 32, s + 32 * c);
+      tmem_wait_ld();
+      if (k0 + T2_BN > P) {     // keys >= P are tree slots (visible iff an ancestor); keys >= T absent
+#pragma unroll
+        for (int w = 0; w < T2_BN / 32; ++w) {
+          const int j0 = k0 + 32 * w - P;              // tree index of the word's first key
+          uint32_t word;
+          if (j0 <= -32) {
+            word = 0xffffffffu;
+          } else if (j0 < 0) {
+            word = (node < nn ? (arow[0] << (-j0)) : 0u) | ((1u << (-j0)) - 1u);
+          } else {
+            const int wi = j0 >> 5, sh = j0 & 31;
+            const uint32_t lo = (node < nn && wi < g.W) ? arow[wi] : 0u;
+            const uint32_t hi = (node < nn && wi + 1 < g.W) ? arow[wi + 1] : 0u;
+            word = __funnelshift_r(lo, hi, sh);
+          }
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (!((word >> c) & 1u)) s[32 * w + c] = -INFINITY;
+        }
+      }
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < T2_BN; c += 4) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mx4[e] = fmaxf(mx4[e], s[c + e]);
+      }
+      const float m_tile = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
+      bool rescale = false;
+      float m_new = m_used;
+      if (m_tile > m_used + TC_RESCALE_LOG2 || (m_used == -INFINITY && m_tile > -INFINITY)) {
+        m_new = m_tile;
+        rescale = true;
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+        const float corr = !rescale ? 1.f : ((m_used == -INFINITY) ? 0.f : ex2_approx(m_used - m_new));
+        l *= corr;
+        if (jj > 0) {        // PV_t(jj-1) has completed (it precedes S_t(jj)); O_t is ours to rescale
+#pragma unroll 1
+          for (int c = 0; c < TC_D / 32; ++c) {
+            float o[32];
+            tmem_ld32(tm_o + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= corr;
+            tmem_st32(tm_o + c * 32, o);
+          }
+          tmem_wait_st();
+        }
+        if (rescale) m_used = m_new;
+      }
+      const float mneg = (m_used == -INFINITY) ? 0.f : -m_used;
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {       // 64 keys -> 32 packed columns per store
+        float pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float e0 = ex2_approx(fmaf(s[64 * half + 2 * c], sl2, mneg));
+          const float e1 = ex2_approx(fmaf(s[64 * half + 2 * c + 1], sl2, mneg));
+          ls4[c & 3] += e0 + e1;
+          pk[c] = __uint_as_float(pack_bf16x2(e0, e1));
+        }
+        tmem_st32(tm_s + 32 * half, pk);
+      }
+      l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.bar_pready[t]);
+    }
+    // ---- epilogue ----
+    bool fin = ok && nt > 0;
+    if (fin) fin = mbar_wait(&sm.bar_odone, 0, abort, wlim);
+    const int mt = mt0 + t;
+    const size_t munit = (((size_t)layer * g.n_req + r) * g.Hkv + kvh) * p.mtiles + mt;
+    if (__all_sync(0xffffffffu, fin)) {
+      tc_fence_after();
+      const bool live = node < nn;
+      if (p.splits == 1) {
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        __nv_bfloat16* orow =
+            p.out + ((((size_t)layer * g.n_req + r) * g.n + min(node, g.n - 1)) * g.Hq + hq) * TC_D;
+#pragma unroll 1
+        for (int c = 0; c < TC_D / 32; ++c) {
+          float o[32];
+          tmem_ld32(tm_o + c * 32, o);
+          tmem_wait_ld();
+          if (live) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 q4;
+              q4.x = pack_bf16x2(o[e] * inv, o[e + 1] * inv);
+              q4.y = pack_bf16x2(o[e + 2] * inv, o[e + 3] * inv);
+              q4.z = pack_bf16x2(o[e + 4] * inv, o[e + 5] * inv);
+              q4.w = pack_bf16x2(o[e + 6] * inv, o[e + 7] * inv);
+              *reinterpret_cast<uint4*>(orow + c * 32 + e) = q4;
+            }
+          }
+        }
+        if (live && p.out_lse)
+          p.out_lse[(((size_t)layer * g.n_req + r) * g.n + node) * g.Hq + hq] =
+              (m_used + log2f(l)) * 0.6931471805599453f;
+      } else {
+        const size_t slot = munit * p.splits + split;
+        float4* wo = reinterpret_cast<float4*>(p.ws_o) + slot * (TC_D / 4) * TC_BM + row;
+#pragma unroll 1
+        for (int c = 0; c < TC_D / 32; ++c) {
+          float o[32];
+          tmem_ld32(tm_o + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            wo[(size_t)((c * 32 + e) / 4) * TC_BM] = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+        }
+        p.ws_ml[slot * TC_BM + row] = make_float2(m_used, l);
+      }
+    } else if (p.splits > 1 && t < ntl) {
+      const size_t slot = munit * p.splits + split;
+      p.ws_ml[slot * TC_BM + row] = make_float2(-INFINITY, 0.f);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(T2_TMEM_COLS));
+  }
+}
+
+// ---------------------------------------------------------------- host side
+// Which kernel runs: the two-M-tile kernel whenever each CTA keeps at least
+// T2_MIN_TILES key tiles after the split the GPU needs (long key ranges);
+// the single-M-tile kernel otherwise (short ranges, where set-up dominates).
+constexpr int T2_MIN_TILES = 8;
+
+struct AttnDispatch {
+  bool v2;
+  TcPlan v1;           // single-M-tile plan (v2 == false)
+  int splits, mtiles, mpairs, units2;   // two-M-tile plan
+};
+
+inline AttnDispatch attn_dispatch(const AttnGeom& g, int num_sms) {
+  AttnDispatch d;
+  d.v1 = tc_plan(g, num_sms);
+  const int G = g.Hq / g.Hkv;
+  d.mtiles = (g.n * G + TC_BM - 1) / TC_BM;
+  d.mpairs = (d.mtiles + 1) / 2;
+  d.units2 = g.layers * g.n_req * g.Hkv * d.mpairs;
+  const long long cap = g.paged ? (long long)g.max_blocks * DDTREE_PAGE : (long long)g.s_max;
+  const long long tiles = (cap + T2_BN - 1) / T2_BN;
+  int splits = 1;
+  if (d.units2 < num_sms) {
+    splits = num_sms / d.units2;
+    if (splits > TC_MAX_SPLITS) splits = TC_MAX_SPLITS;
+    if ((long long)splits * T2_MIN_TILES > tiles) splits = (int)(tiles / T2_MIN_TILES);
+    if (splits < 1) splits = 1;
+  }
+  d.splits = splits;
+  d.v2 = tiles / splits >= T2_MIN_TILES;
+  return d;
+}
+
+inline size_t attn_tc_ws_bytes(const AttnGeom& g, int num_sms) {
+  const AttnDispatch d = attn_dispatch(g, num_sms);
+  if (!d.v2) return tc_attn_ws_bytes(g, num_sms);
+  if (d.splits == 1) return 0;
+  const size_t slots = (size_t)g.layers * g.n_req * g.Hkv * d.mtiles * d.splits;
+  return align256(slots * TC_BM * TC_D * 4) + align256(slots * TC_BM * 8);
+}
+
+inline int attn_tc_launch(const void* q, const void* kc, const void* vc, const int32_t* block_table,
+                          const int32_t* prefix_len, const uint32_t* anc, const int32_t* n_nodes, const AttnGeom& g,
+                          void* out, float* out_lse, void* ws, int num_sms, cudaStream_t stream,
+                          uint64_t wait_ns = 0, int stop_tile = -1) {
+  const AttnDispatch d = attn_dispatch(g, num_sms);
+  if (!d.v2)
+    return tc_attn_launch(q, kc, vc, block_table, prefix_len, anc, n_nodes, g, out, out_lse, ws, num_sms, stream,
+                          wait_ns, stop_tile);
+  T2Params p;
+  p.g = g;
+  p.G = g.Hq / g.Hkv;
+  p.mtiles = d.mtiles;
+  p.mpairs = d.mpairs;
+  p.nq = 2;
+  p.splits = d.splits;
+  p.units = d.units2;
+  p.block_table = block_table;
+  p.prefix_len = prefix_len;
+  p.anc = anc;
+  p.n_nodes = n_nodes;
+  p.out = (__nv_bfloat16*)out;
+  p.out_lse = out_lse;
+  p.ws_o = nullptr;
+  p.ws_ml = nullptr;
+  p.lpt = (d.splits == 1 && g.n_req > 1 && g.n_req <= TC_LPT_MAX_REQ) ? 1 : 0;
+  p.wait_ns = wait_ns > 0 ? wait_ns : TC_WAIT_NS;
+  p.stop_tile = stop_tile;
+  const size_t slots = (size_t)g.layers * g.n_req * g.Hkv * d.mtiles * d.splits;
+  if (d.splits > 1) {
+    p.ws_o = (float*)ws;
+    p.ws_ml = (float2*)((char*)ws + align256(slots * TC_BM * TC_D * 4));
+  }
+  CUtensorMap mq, mk, mv;
+  if (!make_map_4d(&mq, q, (uint64_t)g.Hq, (uint64_t)g.n, (uint64_t)g.layers * g.n_req, (uint32_t)p.G,
+                   (uint32_t)(TC_BM / p.G)))
+    return DDTREE_ERR_CUDA;
+  if (!g.paged) {
+    if (!make_map_4d(&mk, kc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, T2_BN)) return DDTREE_ERR_CUDA;
+    if (!make_map_4d(&mv, vc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, T2_BN)) return DDTREE_ERR_CUDA;
+  } else {
+    if (!make_map_4d(&mk, kc, g.Hkv, DDTREE_PAGE, (uint64_t)g.layers * g.num_blocks, 1, DDTREE_PAGE))
+      return DDTREE_ERR_CUDA;
+    if (!make_map_4d(&mv, vc, g.Hkv, DDTREE_PAGE, (uint64_t)g.layers * g.num_blocks, 1, DDTREE_PAGE))
+      return DDTREE_ERR_CUDA;
+  }
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(tree_attn_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)t2_smem_bytes()) != cudaSuccess)
+      return DDTREE_ERR_CUDA;
+    attr_set = true;
+  }
+  const long long grid = (long long)d.units2 * d.splits;
+  if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
+  tree_attn_tc2_kernel<<<(unsigned)grid, T2_THREADS, t2_smem_bytes(), stream>>>(mq, mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return DDTREE_ERR_CUDA;
+  if (d.splits > 1) {
+    // the combine kernel walks M-tile units
+    TcParams c;
+    c.g = g;
+    c.G = p.G;
+    c.mtiles = d.mtiles;
+    c.splits = d.splits;
+    c.units = g.layers * g.n_req * g.Hkv * d.mtiles;
+    c.block_table = block_table;
+    c.prefix_len = prefix_len;
+    c.anc = anc;
+    c.n_nodes = n_nodes;
+    c.out = p.out;
+    c.out_lse = out_lse;
+    c.ws_o = p.ws_o;
+    c.ws_ml = p.ws_ml;
+    c.lpt = 0;
+    c.wait_ns = p.wait_ns;
+    c.stop_tile = -1;
+    if (d.splits <= 8)
+      tree_attn_combine_kernel<8><<<c.units * (TC_D / 8), TC_BM, 0, stream>>>(c);
+    else
+      tree_attn_combine_kernel<TC_MAX_SPLITS><<<c.units * (TC_D / 8), TC_BM, 0, stream>>>(c);
+    if (cudaGetLastError() != cudaSuccess) return DDTREE_ERR_CUDA;
+  }
+  return DDTREE_OK;
+}
+
+}  // namespace ddt

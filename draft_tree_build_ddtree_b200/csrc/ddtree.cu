@@ -15,6 +15,7 @@
 #include "accept.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
+#include "attn_tc2.cuh"
 
 using namespace ddt;
 
@@ -223,7 +224,7 @@ bool use_tc_attn(int dtype, const ddtree_kv_desc* kv) {
 
 size_t attn_ws(const ddtree_kv_desc* kv, int B, int dtype) {
   if (!use_tc_attn(dtype, kv)) return 0;
-  return tc_attn_ws_bytes(geom_of(kv, B), num_sms());
+  return attn_tc_ws_bytes(geom_of(kv, B), num_sms());
 }
 
 int attn_launch(const void* q, const void* k_cache, const void* v_cache, int dtype, const ddtree_kv_desc* kv,
@@ -239,9 +240,9 @@ int attn_launch(const void* q, const void* k_cache, const void* v_cache, int dty
     return DDTREE_ERR_INVALID_ARG;
   AttnGeom g = geom_of(kv, B);
   if (use_tc_attn(dtype, kv)) {
-    const size_t need = tc_attn_ws_bytes(g, num_sms());
+    const size_t need = attn_tc_ws_bytes(g, num_sms());
     if (need && (!ws || !aligned16(ws) || ws_bytes < need)) return DDTREE_ERR_INVALID_ARG;
-    return tc_attn_launch(q, k_cache, v_cache, block_table, prefix_len, anc, n_nodes, g, out, out_lse, ws,
+    return attn_tc_launch(q, k_cache, v_cache, block_table, prefix_len, anc, n_nodes, g, out, out_lse, ws,
                           num_sms(), s, g_attn_wait_ns, g_attn_stop_tile);
   }
   const long long grid =
@@ -444,7 +445,7 @@ int ddtree_round_launch_count(const ddtree_round_args* a) {
   if (!a || a->n_req < 1 || a->L < 1 || a->V < 1 || a->K < 1 || a->B < 0 || kv_check(&a->kv)) return -1;
   int n = 2;                                                             // top-K, build
   n += 1;                                                                // attention
-  if (use_tc_attn(a->dtype, &a->kv) && tc_attn_ws_bytes(geom_of(&a->kv, a->B), num_sms()) > 0) n += 1;   // combine
+  if (use_tc_attn(a->dtype, &a->kv) && attn_tc_ws_bytes(geom_of(&a->kv, a->B), num_sms()) > 0) n += 1;   // combine
   n += 1;                                                                // argmax (+ walk)
   if (a->kv.layers > WALK_FUSE_MAX_LAYERS) n += 1;                       // walk and compaction
   return n;
@@ -478,6 +479,82 @@ int ddtree_debug_attn_timeout(unsigned long long wait_ns, int withhold_tile) {
   g_attn_wait_ns = wait_ns;
   g_attn_stop_tile = withhold_tile;
   return DDTREE_OK;
+}
+
+// ---------------------------------------------------------------- host-buffer round
+static int round_host_plan(const ddtree_round_args* a, const ddtree_round_host_io* h, unsigned long long* h2d,
+                           unsigned long long* d2h, cudaStream_t s, bool run) {
+  if (!a || !h) return DDTREE_ERR_INVALID_ARG;
+  if (kv_check(&a->kv) || a->kv.n_req != a->n_req || !dtype_ok(a->dtype)) return DDTREE_ERR_INVALID_ARG;
+  const size_t es = (size_t)esize_of(a->dtype);
+  const size_t N = (size_t)a->n_req, n = (size_t)a->B + 1, layers = (size_t)a->kv.layers;
+  const size_t row = (size_t)a->kv.Hkv * a->kv.D * es;                 // one cache slot
+  const size_t qbytes = layers * N * n * a->kv.Hq * a->kv.D * es;
+  unsigned long long in = 0, out = 0;
+  auto h2d_copy = [&](void* dst, const void* src, size_t bytes) -> int {
+    if (!src) return DDTREE_OK;
+    if (!dst) return DDTREE_ERR_INVALID_ARG;
+    in += bytes;
+    if (run && cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return DDTREE_ERR_CUDA;
+    return DDTREE_OK;
+  };
+  auto d2h_copy = [&](void* dst, const void* src, size_t bytes) -> int {
+    if (!dst) return DDTREE_OK;
+    if (!src) return DDTREE_ERR_INVALID_ARG;
+    out += bytes;
+    if (run && cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return DDTREE_ERR_CUDA;
+    return DDTREE_OK;
+  };
+  int st;
+  if ((st = h2d_copy((void*)a->drafter_logits, h->drafter_logits, N * a->L * (size_t)a->drafter_stride * es))) return st;
+  if ((st = h2d_copy((void*)a->root_token, h->root_token, N * 4))) return st;
+  if ((st = h2d_copy((void*)a->q, h->q, qbytes))) return st;
+  if ((st = h2d_copy((void*)a->target_logits, h->target_logits, N * n * (size_t)a->target_stride * es))) return st;
+  if ((st = h2d_copy((void*)a->prefix_len, h->prefix_len, N * 4))) return st;
+  if ((h->tree_k != nullptr) != (h->tree_v != nullptr)) return DDTREE_ERR_INVALID_ARG;
+  if (h->tree_k) {
+    if (!h->prefix_len || !a->k_cache || !a->v_cache) return DDTREE_ERR_INVALID_ARG;
+    if (a->kv.paged && !a->block_table) return DDTREE_ERR_INVALID_ARG;
+    // a paged cache's block table is device memory: the host cannot address its tree slots
+    if (a->kv.paged) return DDTREE_ERR_UNSUPPORTED;
+    const size_t cap = (size_t)a->kv.s_max;
+    for (size_t r = 0; r < N; ++r) {
+      const int P = h->prefix_len[r];
+      if (P < 0 || (size_t)P + n > cap) return DDTREE_ERR_INVALID_ARG;
+      for (int c = 0; c < 2; ++c) {
+        const unsigned char* src = (const unsigned char*)(c ? h->tree_v : h->tree_k) + r * n * row;
+        unsigned char* dst = (unsigned char*)(c ? a->v_cache : a->k_cache) + (r * cap + (size_t)P) * row;
+        // one 2-D copy over the layers: rows of n * row bytes
+        in += layers * n * row;
+        if (run && cudaMemcpy2DAsync(dst, N * cap * row, src, N * n * row, n * row, layers, cudaMemcpyHostToDevice,
+                                     s) != cudaSuccess)
+          return DDTREE_ERR_CUDA;
+      }
+    }
+  }
+  if (run && (st = ddtree_round(a, s))) return st;
+  if ((st = d2h_copy(h->attn_out, a->attn_out, qbytes))) return st;
+  if ((st = d2h_copy(h->node_token, a->node_token, N * n * 4))) return st;
+  if ((st = d2h_copy(h->parent, a->parent, N * n * 4))) return st;
+  if ((st = d2h_copy(h->n_nodes, a->n_nodes, N * 4))) return st;
+  if ((st = d2h_copy(h->path, a->path, N * (a->L + 1) * 4))) return st;
+  if ((st = d2h_copy(h->accept_len, a->accept_len, N * 4))) return st;
+  if ((st = d2h_copy(h->next_bonus, a->next_bonus, N * 4))) return st;
+  if ((st = d2h_copy(h->new_prefix_len, a->new_prefix_len, N * 4))) return st;
+  if (h2d) *h2d = in;
+  if (d2h) *d2h = out;
+  return DDTREE_OK;
+}
+
+int ddtree_round_host(const ddtree_round_args* dev, const ddtree_round_host_io* host, cudaStream_t stream) {
+  int st = round_host_plan(dev, host, nullptr, nullptr, stream, false);   // validate before any copy
+  if (st) return st;
+  return round_host_plan(dev, host, nullptr, nullptr, stream, true);
+}
+
+int ddtree_round_host_bytes(const ddtree_round_args* dev, const ddtree_round_host_io* host, unsigned long long* h2d,
+                            unsigned long long* d2h) {
+  return round_host_plan(dev, host, h2d, d2h, nullptr, false) ? -1 : 0;
 }
 
 const char* ddtree_status_string(int status) {

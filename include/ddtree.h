@@ -306,6 +306,52 @@ int ddtree_round(const ddtree_round_args* a, cudaStream_t stream);
  * -1 for an invalid geometry.  Host only: no device work. */
 int ddtree_round_launch_count(const ddtree_round_args* a);
 
+/*
+ * The round from host memory: the call a user makes whose drafter and
+ * target produce their logits and tree-node Q/K/V on the host.  All copies
+ * are cudaMemcpyAsync on `stream` (one per buffer, or one 2-D copy per
+ * request for the tree K/V rows); use pinned host memory for them to
+ * overlap.  In order on the stream:
+ *   1. host -> device: drafter_logits, root_token, q, target_logits and
+ *      prefix_len into the buffers of `dev` (same layouts); when tree_k and
+ *      tree_v are given, the K and V rows of the B+1 tree nodes of every
+ *      layer and request ([layers][n_req][B+1][Hkv][D] on the host) into
+ *      cache slots P_r .. P_r + B (Deep Dive §5: tree K/V sit in the cache
+ *      tail), P_r read from the host prefix_len;
+ *   2. ddtree_round(dev);
+ *   3. device -> host: every non-NULL output of `host` from the matching
+ *      buffer of `dev`.
+ * The call returns once everything is enqueued; synchronise `stream` before
+ * reading the host outputs.  Host pointers left NULL are not copied (an
+ * input then keeps whatever the device buffer holds).
+ */
+typedef struct {
+  /* inputs (host) */
+  const void* drafter_logits;      /* [n_req*L][drafter_stride] */
+  const int32_t* root_token;       /* [n_req] */
+  const void* q;                   /* [layers][n_req][B+1][Hq][D] */
+  const void* target_logits;       /* [n_req][B+1][target_stride] */
+  const int32_t* prefix_len;       /* [n_req] */
+  const void* tree_k;              /* [layers][n_req][B+1][Hkv][D]; contiguous caches only */
+  const void* tree_v;              /* (paged: DDTREE_ERR_UNSUPPORTED) */
+  /* outputs (host) */
+  void* attn_out;                  /* [layers][n_req][B+1][Hq][D] */
+  int32_t* node_token;             /* [n_req][B+1] */
+  int32_t* parent;                 /* [n_req][B+1] */
+  int32_t* n_nodes;                /* [n_req] */
+  int32_t* path;                   /* [n_req][L+1] */
+  int32_t* accept_len;             /* [n_req] */
+  int32_t* next_bonus;             /* [n_req] */
+  int32_t* new_prefix_len;         /* [n_req] */
+} ddtree_round_host_io;
+
+int ddtree_round_host(const ddtree_round_args* dev, const ddtree_round_host_io* host, cudaStream_t stream);
+
+/* Bytes ddtree_round_host copies host -> device (*h2d) and device -> host
+ * (*d2h) with these arguments; -1 for invalid arguments.  Host only. */
+int ddtree_round_host_bytes(const ddtree_round_args* dev, const ddtree_round_host_io* host,
+                            unsigned long long* h2d, unsigned long long* d2h);
+
 /* ---------------------------------------------------------------------- */
 /* Top-K without a caller workspace (no counterpart in the paper: an      */
 /* interface convenience of this library).                                */

@@ -465,8 +465,9 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 
 // ---------------------------------------------------------------- host side
 // Which kernel runs: the two-M-tile kernel whenever each CTA keeps at least
-// T2_MIN_TILES key tiles after the split the GPU needs (long key ranges);
-// the single-M-tile kernel otherwise (short ranges, where set-up dominates).
+// T2_MIN_TILES key tiles after the split the GPU needs (long key ranges) and
+// its CTAs still cover half the SMs; the single-M-tile kernel otherwise
+// (short ranges, where set-up and latency dominate).
 constexpr int T2_MIN_TILES = 8;
 
 struct AttnDispatch {
@@ -492,7 +493,8 @@ inline AttnDispatch attn_dispatch(const AttnGeom& g, int num_sms) {
     if (splits < 1) splits = 1;
   }
   d.splits = splits;
-  d.v2 = tiles / splits >= T2_MIN_TILES;
+  // long enough per CTA, and enough CTAs to keep at least half the SMs busy
+  d.v2 = tiles / splits >= T2_MIN_TILES && (long long)d.units2 * splits * 2 >= num_sms;
   return d;
 }
 

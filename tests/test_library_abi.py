@@ -121,7 +121,8 @@ def test_launch_plans_from_sizes(lib):
     sizes: b64_p2k top-K cuts each of its 16 bf16 rows into 9 chunks (one
     wave of 144 CTAs) with K + K candidate slots each; the b64_p2k attention splits
     its 20 units (4 KV heads x 5 M-tiles) 7 ways over 128-key tiles; the
-    48-layer and 32-request workloads fill the GPU unsplit."""
+    32k-prefix sweep splits its M-tile pairs; the 48-layer and 32-request
+    workloads fill the GPU unsplit."""
     rows, V, K = 16, 151936, 64
     cap = 2 * K
 
@@ -135,6 +136,12 @@ def test_launch_plans_from_sizes(lib):
     kv2 = dd.kv_desc(1, 1, 32, 4, 128, s_max=2176)
     slots = 20 * 7
     assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv2), 64) == \
+        _align256(slots * 128 * 128 * 4) + _align256(slots * 128 * 8)
+    # sweep_p32k at B = 64: the two-M-tile kernel, 4 KV heads x 3 M-tile pairs
+    # split 12 ways; partials per (M-tile, split): 4 x 5 x 12
+    kv5 = dd.kv_desc(1, 1, 32, 4, 128, s_max=32896)
+    slots = 4 * 5 * 12
+    assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv5), 64) == \
         _align256(slots * 128 * 128 * 4) + _align256(slots * 128 * 8)
     kv3 = dd.kv_desc(48, 1, 32, 4, 128, s_max=8512)
     assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv3), 256) == 0

@@ -25,7 +25,7 @@ import torch
 
 __all__ = [
     "DDTreeError", "KVDesc", "lib", "ddtree_topk", "ddtree_build", "ddtree_tree_attn",
-    "ddtree_accept", "ddtree_round", "device_status", "RoundBuffers", "Workspace",
+    "ddtree_accept", "ddtree_round", "device_status", "RoundBuffers", "Workspace", "Sampling",
     "BF16", "F32",
 ]
 
@@ -50,6 +50,10 @@ class KVDesc(ctypes.Structure):
                 ("num_blocks", _i), ("max_blocks", _i)]
 
 
+class Sampling(ctypes.Structure):
+    _fields_ = [("temperature", ctypes.c_double), ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_ulonglong)]
+
+
 class RoundArgs(ctypes.Structure):
     _fields_ = [("n_req", _i), ("L", _i), ("V", _i), ("K", _i), ("B", _i), ("dtype", _i),
                 ("kv", KVDesc),
@@ -64,7 +68,7 @@ class RoundArgs(ctypes.Structure):
                 ("next_bonus", _vp), ("src_slot", _vp), ("dst_slot", _vp),
                 ("new_prefix_len", _vp),
                 ("ws", _vp), ("ws_bytes", _sz),
-                ("gain_floor", _vp)]
+                ("gain_floor", _vp), ("sampling", ctypes.POINTER(Sampling))]
 
 
 _SIGS = {
@@ -79,6 +83,9 @@ _SIGS = {
     "ddtree_accept_workspace_bytes": (_sz, [_i, _i, _i]),
     "ddtree_accept": (_i, [_vp, _i, _i, _ll, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp,
                            ctypes.POINTER(KVDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "ddtree_accept_ex": (_i, [_vp, _i, _i, _ll, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp,
+                              ctypes.POINTER(KVDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                              ctypes.POINTER(Sampling), _vp, _sz, _vp]),
     "ddtree_round_workspace_bytes": (_sz, [ctypes.POINTER(RoundArgs)]),
     "ddtree_round": (_i, [ctypes.POINTER(RoundArgs), _vp]),
     "ddtree_round_launch_count": (_i, [ctypes.POINTER(RoundArgs)]),
@@ -307,8 +314,13 @@ def alloc_accept(n_req: int, L: int, B: int, device) -> Accept:
 
 def ddtree_accept(target_logits, node_token, parent, n_nodes, L, prefix_len,
                   k_cache=None, v_cache=None, kv: Optional[KVDesc] = None, block_table=None,
-                  out: Optional[Accept] = None, ws=None) -> Accept:
-    """Greedy walk over [n_req, B+1, V] target logits; compacts the KV in place."""
+                  out: Optional[Accept] = None, ws=None, temperature: float = 0.0, seed: int = 0,
+                  offset: int = 0) -> Accept:
+    """Verifier walk over [n_req, B+1, V] target logits; compacts the KV in place.
+
+    temperature <= 0: greedy (argmax); > 0: one draw per node from
+    softmax(z / temperature), keyed by (seed, offset) (ddtree_accept_ex).
+    """
     _dev(target_logits, "target_logits")
     if target_logits.dim() != 3 or target_logits.stride(2) != 1:
         raise DDTreeError("target_logits must be [n_req, B+1, V] with a contiguous last dim")
@@ -319,15 +331,16 @@ def ddtree_accept(target_logits, node_token, parent, n_nodes, L, prefix_len,
     a = alloc_accept(n_req, L, B, target_logits.device) if out is None else out
     need = lib().ddtree_accept_workspace_bytes(n_req, B, V)
     w = _ws["accept"].get(need, target_logits.device) if ws is None else ws
-    _check(lib().ddtree_accept(_ptr(target_logits), _dtype_code(target_logits), V,
-                               target_logits.stride(1), _ptr(node_token), _ptr(parent), _ptr(n_nodes),
-                               n_req, L, B, _ptr(prefix_len), _ptr(a.new_prefix_len),
-                               _ptr(k_cache), _ptr(v_cache),
-                               ctypes.byref(kv) if kv is not None else None, _ptr(block_table),
-                               _ptr(a.target_argmax), _ptr(a.path), _ptr(a.accept_len),
-                               _ptr(a.next_bonus), _ptr(a.src_slot), _ptr(a.dst_slot),
-                               _ptr(w), w.numel(), _stream()),
-           "ddtree_accept")
+    samp = Sampling(float(temperature), int(seed) & (2 ** 64 - 1), int(offset) & (2 ** 64 - 1))
+    _check(lib().ddtree_accept_ex(_ptr(target_logits), _dtype_code(target_logits), V,
+                                  target_logits.stride(1), _ptr(node_token), _ptr(parent), _ptr(n_nodes),
+                                  n_req, L, B, _ptr(prefix_len), _ptr(a.new_prefix_len),
+                                  _ptr(k_cache), _ptr(v_cache),
+                                  ctypes.byref(kv) if kv is not None else None, _ptr(block_table),
+                                  _ptr(a.target_argmax), _ptr(a.path), _ptr(a.accept_len),
+                                  _ptr(a.next_bonus), _ptr(a.src_slot), _ptr(a.dst_slot),
+                                  ctypes.byref(samp), _ptr(w), w.numel(), _stream()),
+           "ddtree_accept_ex")
     return a
 
 
@@ -359,6 +372,7 @@ class RoundBuffers:
     acc: Accept = None
     ws: torch.Tensor = None
     gain_floor: Optional[torch.Tensor] = None   # float32 [n_req]: adaptive-budget floor of the build
+    sampling: Optional[Sampling] = None         # temperature > 0 verification (None: greedy)
     _args: RoundArgs = None
 
     def allocate_outputs(self):
@@ -397,6 +411,8 @@ class RoundBuffers:
         a.next_bonus, a.src_slot, a.dst_slot = _ptr(c.next_bonus), _ptr(c.src_slot), _ptr(c.dst_slot)
         a.new_prefix_len = _ptr(c.new_prefix_len)
         a.gain_floor = _ptr(self.gain_floor)
+        if self.sampling is not None:
+            a.sampling = ctypes.pointer(self.sampling)
         need = lib().ddtree_round_workspace_bytes(ctypes.byref(a))
         if need == 0:
             raise DDTreeError("invalid round geometry")

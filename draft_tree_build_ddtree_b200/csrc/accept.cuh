@@ -206,14 +206,64 @@ __device__ void walk_request(const WalkArgs& a, int r, int nn, int P, int lk0, i
   }
 }
 
+// ---------------------------------------------------------------------------
+// Temperature > 0: one draw per tree node from softmax(z / T) by the
+// Gumbel-max identity, argmax_v (z_v / T - log(-log u_v)), with u_v from
+// Philox4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
+// easy as 1, 2, 3", SC 2011): output word v % 4 at counter
+// (v / 4, node, request, 0) and key (seed, offset).  The perturbed score is
+// formed in fp64 with explicitly rounded operations and rounded once to fp32;
+// the argmax then runs exactly as at temperature 0 (lowest id on ties).
+// ---------------------------------------------------------------------------
+struct SampleArgs {
+  double inv_t;                    // 1 / T in fp64
+  unsigned long long seed, offset;
+};
+
+__device__ __forceinline__ void philox4x64_10(unsigned long long c[4], unsigned long long k0, unsigned long long k1) {
+  constexpr unsigned long long M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+  constexpr unsigned long long W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const unsigned long long hi0 = __umul64hi(M0, c[0]), lo0 = M0 * c[0];
+    const unsigned long long hi1 = __umul64hi(M1, c[2]), lo1 = M1 * c[2];
+    const unsigned long long n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+    c[0] = n0;
+    c[1] = lo1;
+    c[2] = n2;
+    c[3] = lo0;
+    k0 += W0;
+    k1 += W1;
+  }
+}
+
+// The four Philox words of counter (block, node, req, 0).
+__device__ __forceinline__ void philox_block(unsigned long long w[4], unsigned long long block, int node, int req,
+                                             const SampleArgs& sa) {
+  w[0] = block;
+  w[1] = (unsigned long long)node;
+  w[2] = (unsigned long long)req;
+  w[3] = 0ull;
+  philox4x64_10(w, sa.seed, sa.offset);
+}
+
+// fp32 rounding of z / T + Gumbel(u(word)); u = ((word >> 12) + 1/2) 2^-52 is exact.
+__device__ __forceinline__ float gumbel_score(float z, unsigned long long word, double inv_t) {
+  const double u = __dmul_rn(__dadd_rn((double)(word >> 12), 0.5), 0x1p-52);
+  const double g = -log(-log(u));
+  return __double2float_rn(__dadd_rn(__dmul_rn((double)z, inv_t), g));
+}
+
 // The argmax of one chunk of a row: per-thread running best over batches of
 // 16-byte loads (elements visited in increasing index order, so the first
 // maximum -- the lowest index -- is kept; NaN never compares greater and is
-// flagged), then a block-wide maximum of 64-bit composites.
-template <int DT>
-__global__ void __launch_bounds__(ARGMAX_THREADS, ARGMAX_CTAS_PER_SM)
+// flagged), then a block-wide maximum of 64-bit composites.  SAMPLE: the
+// argmax of the Gumbel-perturbed scores (a draw at temperature T > 0).
+template <int DT, bool SAMPLE>
+__global__ void __launch_bounds__(ARGMAX_THREADS, SAMPLE ? 2 : ARGMAX_CTAS_PER_SM)
 argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_stride,
-              const int32_t* __restrict__ n_nodes, int cpr, int chunk, ArgmaxWs ws, WalkArgs wa, int fuse_walk) {
+              const int32_t* __restrict__ n_nodes, int cpr, int chunk, ArgmaxWs ws, WalkArgs wa, int fuse_walk,
+              SampleArgs sa) {
   constexpr int EPV = (DT == DDTREE_BF16) ? 8 : 4;
   __shared__ unsigned long long red[ARGMAX_THREADS / 32];
   __shared__ int s_last;
@@ -241,28 +291,53 @@ argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_strid
   auto visit = [&](float f, uint32_t idx) {
     if (f > bv || (bi == 0xFFFFFFFFu && f == bv)) { bv = f; bi = idx; }
   };
-  for (int vb = 0; vb < nvec_full; vb += ARGMAX_THREADS * ARGMAX_VPT) {
-    uint4 vec[ARGMAX_VPT];
+  constexpr int VPT = SAMPLE ? 2 : ARGMAX_VPT;     // sampling is compute-bound: fewer loads in flight
+  for (int vb = 0; vb < nvec_full; vb += ARGMAX_THREADS * VPT) {
+    uint4 vec[VPT];
 #pragma unroll
-    for (int v = 0; v < ARGMAX_VPT; ++v) {
+    for (int v = 0; v < VPT; ++v) {
       const int vi = vb + v * ARGMAX_THREADS + tid;
       vec[v] = vi < nvec_full ? ldg_stream_v4(base + (size_t)vi * 16) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int v = 0; v < ARGMAX_VPT; ++v) {
+    for (int v = 0; v < VPT; ++v) {
       const int vi = vb + v * ARGMAX_THREADS + tid;
       if (vi < nvec_full) {
+        if (!SAMPLE) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t w = u32_at(vec[v], q);
-          if (DT == DDTREE_BF16) {
-            mag = max(mag, max(w & 0x7FFFu, (w >> 16) & 0x7FFFu));
-            visit(__uint_as_float(w << 16), (uint32_t)(vi * EPV + 2 * q));
-            visit(__uint_as_float(w & 0xFFFF0000u), (uint32_t)(vi * EPV + 2 * q + 1));
-          } else {
-            const float f = __uint_as_float(w);
-            mag |= (f != f) ? 0xFFFFu : 0u;
-            visit(f, (uint32_t)(vi * EPV + q));
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t w = u32_at(vec[v], q);
+            if (DT == DDTREE_BF16) {
+              mag = max(mag, max(w & 0x7FFFu, (w >> 16) & 0x7FFFu));
+              visit(__uint_as_float(w << 16), (uint32_t)(vi * EPV + 2 * q));
+              visit(__uint_as_float(w & 0xFFFF0000u), (uint32_t)(vi * EPV + 2 * q + 1));
+            } else {
+              const float f = __uint_as_float(w);
+              mag |= (f != f) ? 0xFFFFu : 0u;
+              visit(f, (uint32_t)(vi * EPV + q));
+            }
+          }
+        } else {
+          // the vector's elements start at a multiple of 4 of the row (chunks are multiples of 8)
+          const long long e0 = c0 + (long long)vi * EPV;
+#pragma unroll
+          for (int b = 0; b < EPV / 4; ++b) {
+            unsigned long long rw[4];
+            philox_block(rw, (unsigned long long)(e0 / 4 + b), node, req, sa);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int e = 4 * b + j;
+              float f;
+              if (DT == DDTREE_BF16) {
+                const uint32_t bits = (u32_at(vec[v], e >> 1) >> (16 * (e & 1))) & 0xFFFFu;
+                mag = max(mag, bits & 0x7FFFu);
+                f = bf16_bits_to_f32((uint16_t)bits);
+              } else {
+                f = __uint_as_float(u32_at(vec[v], e));
+                mag |= (f != f) ? 0xFFFFu : 0u;
+              }
+              visit(gumbel_score(f, rw[j], sa.inv_t), (uint32_t)(vi * EPV + e));
+            }
           }
         }
       }
@@ -279,6 +354,12 @@ argmax_kernel(const void* __restrict__ logits, int n, int V, long long row_strid
       } else {
         f = ((const float*)base)[e];
         mag |= (f != f) ? 0xFFFFu : 0u;
+      }
+      if (SAMPLE) {
+        unsigned long long rw[4];
+        const long long g = c0 + e;
+        philox_block(rw, (unsigned long long)(g / 4), node, req, sa);
+        f = gumbel_score(f, rw[g & 3], sa.inv_t);
       }
       visit(f, (uint32_t)e);
     }

@@ -298,9 +298,16 @@ int accept_launch(const void* target_logits, int dtype, int V, long long row_str
                   const int32_t* prefix_len, int32_t* new_prefix_len, void* k_cache, void* v_cache,
                   const ddtree_kv_desc* kv, const int32_t* block_table, int32_t* target_argmax, int32_t* path,
                   int32_t* accept_len, int32_t* next_bonus, int32_t* src_slot, int32_t* dst_slot, void* ws,
-                  size_t ws_bytes, cudaStream_t s) {
+                  size_t ws_bytes, cudaStream_t s, const ddtree_sampling* sampling = nullptr) {
   if (!target_logits || !node_token || !parent || !n_nodes || !prefix_len || !new_prefix_len)
     return DDTREE_ERR_INVALID_ARG;
+  const bool sample = sampling != nullptr && sampling->temperature > 0.0;
+  if (sampling != nullptr && !(sampling->temperature <= 0.0 || sampling->temperature < INFINITY))
+    return DDTREE_ERR_INVALID_ARG;   // NaN or +inf temperature
+  SampleArgs sa;
+  sa.inv_t = sample ? 1.0 / sampling->temperature : 0.0;
+  sa.seed = sample ? sampling->seed : 0ull;
+  sa.offset = sample ? sampling->offset : 0ull;
   if (new_prefix_len == prefix_len) return DDTREE_ERR_INVALID_ARG;
   if (!dtype_ok(dtype) || V < 1 || V > MAX_V || n_req < 1 || n_req > MAX_REQ || L < 1 || L > MAX_L || B < 0 ||
       B > MAX_B)
@@ -350,12 +357,15 @@ int accept_launch(const void* target_logits, int dtype, int V, long long row_str
   a.row_bytes = row_bytes;
   // few layers: the CTA that publishes a request's last argmax walks and compacts it
   const int fuse = (!k_cache || kv->layers <= WALK_FUSE_MAX_LAYERS) ? 1 : 0;
-  if (dtype == DDTREE_BF16)
-    argmax_kernel<DDTREE_BF16><<<(unsigned)grid, ARGMAX_THREADS, 0, s>>>(target_logits, n, V, row_stride, n_nodes,
-                                                                        p.cpr, p.chunk, w, a, fuse);
-  else
-    argmax_kernel<DDTREE_F32><<<(unsigned)grid, ARGMAX_THREADS, 0, s>>>(target_logits, n, V, row_stride, n_nodes,
-                                                                       p.cpr, p.chunk, w, a, fuse);
+#define DDT_ARGMAX(DT, SM)                                                                               \
+  argmax_kernel<DT, SM><<<(unsigned)grid, ARGMAX_THREADS, 0, s>>>(target_logits, n, V, row_stride, n_nodes, \
+                                                                  p.cpr, p.chunk, w, a, fuse, sa)
+  if (dtype == DDTREE_BF16) {
+    if (sample) DDT_ARGMAX(DDTREE_BF16, true); else DDT_ARGMAX(DDTREE_BF16, false);
+  } else {
+    if (sample) DDT_ARGMAX(DDTREE_F32, true); else DDT_ARGMAX(DDTREE_F32, false);
+  }
+#undef DDT_ARGMAX
   int st = launch_status();
   if (st || fuse) return st;
   const size_t smem = (size_t)n * 16;   // next, argmax, parent, token
@@ -408,6 +418,17 @@ int ddtree_tree_attn(const void* q, const void* k_cache, const void* v_cache, in
                      cudaStream_t stream) {
   return attn_launch(q, k_cache, v_cache, dtype, kv, block_table, prefix_len, anc, n_nodes, B, out, out_lse,
                      ws, ws_bytes, stream);
+}
+
+int ddtree_accept_ex(const void* target_logits, int dtype, int V, long long row_stride, const int32_t* node_token,
+                     const int32_t* parent, const int32_t* n_nodes, int n_req, int L, int B,
+                     const int32_t* prefix_len, int32_t* new_prefix_len, void* k_cache, void* v_cache,
+                     const ddtree_kv_desc* kv, const int32_t* block_table, int32_t* target_argmax, int32_t* path,
+                     int32_t* accept_len, int32_t* next_bonus, int32_t* src_slot, int32_t* dst_slot,
+                     const ddtree_sampling* sampling, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return accept_launch(target_logits, dtype, V, row_stride, node_token, parent, n_nodes, n_req, L, B, prefix_len,
+                       new_prefix_len, k_cache, v_cache, kv, block_table, target_argmax, path, accept_len,
+                       next_bonus, src_slot, dst_slot, ws, ws_bytes, stream, sampling);
 }
 
 size_t ddtree_accept_workspace_bytes(int n_req, int B, int V) {
@@ -471,7 +492,7 @@ int ddtree_round(const ddtree_round_args* a, cudaStream_t stream) {
   return accept_launch(a->target_logits, a->dtype, a->V, a->target_stride, a->node_token, a->parent, a->n_nodes,
                        a->n_req, a->L, a->B, a->prefix_len, a->new_prefix_len, a->k_cache, a->v_cache, &a->kv,
                        a->block_table, a->target_argmax, a->path, a->accept_len, a->next_bonus, a->src_slot,
-                       a->dst_slot, ws + off_acc, need - off_acc, stream);
+                       a->dst_slot, ws + off_acc, need - off_acc, stream, a->sampling);
 }
 
 int ddtree_debug_attn_timeout(unsigned long long wait_ns, int withhold_tile) {

@@ -254,6 +254,42 @@ int ddtree_accept(const void* target_logits, int dtype, int V, long long row_str
                   int32_t* next_bonus, int32_t* src_slot, int32_t* dst_slot,
                   void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/*
+ * ddtree_accept_ex: ddtree_accept at temperature > 0 ("DDTree Deep Dive" §6
+ * and §9: tree verification that keeps the target distribution; the pages
+ * give no rule, this is the plainest one that does).  With sampling NULL or
+ * temperature <= 0 it is ddtree_accept.  Otherwise the target's token at
+ * every live node is one draw from softmax(z / temperature) instead of the
+ * argmax, and the walk is unchanged: each committed token is then a draw
+ * from the target at its context.  The draw is the Gumbel-max identity,
+ * argmax_v (z_v / T - log(-log u_v)), with
+ *   u_v = ((w >> 12) + 1/2) * 2^-52,  w = word v % 4 of Philox4x64-10
+ *         (Salmon et al., SC 2011) at counter (v / 4, node, request, 0)
+ *         and key (seed, offset),
+ * the score formed in fp64 (z times the fp64 value of 1/T, plus the
+ * Gumbel term, each operation rounded) and rounded once to fp32; the
+ * argmax takes the lowest id among equal fp32 scores.  target_argmax then
+ * holds the drawn tokens.  Reuse (seed, offset) only to reproduce a round:
+ * e.g. offset = the round index.  NaN or +inf temperature:
+ * DDTREE_ERR_INVALID_ARG.
+ */
+typedef struct {
+  double temperature;          /* > 0: draw; <= 0: greedy argmax */
+  unsigned long long seed;     /* Philox key, first word */
+  unsigned long long offset;   /* Philox key, second word */
+} ddtree_sampling;
+
+int ddtree_accept_ex(const void* target_logits, int dtype, int V, long long row_stride,
+                     const int32_t* node_token, const int32_t* parent, const int32_t* n_nodes,
+                     int n_req, int L, int B,
+                     const int32_t* prefix_len, int32_t* new_prefix_len,
+                     void* k_cache, void* v_cache, const ddtree_kv_desc* kv,
+                     const int32_t* block_table,
+                     int32_t* target_argmax, int32_t* path, int32_t* accept_len,
+                     int32_t* next_bonus, int32_t* src_slot, int32_t* dst_slot,
+                     const ddtree_sampling* sampling,
+                     void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* ---------------------------------------------------------------------- */
 /* The whole round (Deep Dive §3 stage pipeline: draft -> tree_build ->   */
 /* tree_compile -> verify -> commit; the draft and the target forward are */
@@ -289,6 +325,9 @@ typedef struct {
   /* optional (NULL: none): per-request adaptive-budget floor of the build,
    * device float [n_req], as gain_floor of ddtree_build_ex */
   const float* gain_floor;
+  /* optional (NULL: greedy): verification at temperature > 0, as for
+   * ddtree_accept_ex */
+  const ddtree_sampling* sampling;
 } ddtree_round_args;
 
 /* Bytes of a->ws the round needs (0 for an invalid geometry).  The

@@ -46,6 +46,12 @@ R7  Greedy verification (temperature 0): the target's argmax takes the
 R9  Adaptive budget: a node is worth adding while its gain q(u) exceeds the
     cost c of verifying one more node (in accepted tokens); the build keeps
     the pops whose score is strictly above log c.
+R10 Temperature T > 0: the verifier draws the target's token at every tree
+    node from softmax(z / T) and walks as at temperature 0; each committed
+    token is then a draw from the target at its context, so the output
+    follows the target distribution (Deep Dive §6 and §9 assert this property
+    and give no rule).  The draws use Philox4x64-10 uniforms and the
+    Gumbel-max identity (sample_rows).
 """
 from __future__ import annotations
 
@@ -412,15 +418,17 @@ class Acceptance:
 
 
 def accept(target: np.ndarray, node_token: np.ndarray, parent: np.ndarray,
-           n_nodes: int, L: int, prefix_len: int) -> Acceptance:
-    """The verifier walk of Deep Dive §6 for one request, temperature 0.
+           n_nodes: int, L: int, prefix_len: int, tokens: Optional[np.ndarray] = None) -> Acceptance:
+    """The verifier walk of Deep Dive §6 for one request.
 
     Start at the root; while the root-side node has a child whose token is
-    the target's argmax at that node, descend into it.  The first unmatched
-    argmax is the next bonus token (Block Diffusion Drafters, Core Mechanism:
-    the longest matching prefix is accepted).
+    the target's token at that node, descend into it.  The first unmatched
+    token is the next bonus token (Block Diffusion Drafters, Core Mechanism:
+    the longest matching prefix is accepted).  The target's token at a node
+    is its argmax at temperature 0 (reading R7), or ``tokens`` when given
+    (a draw per node at temperature > 0, reading R10: ``sample_rows``).
     """
-    t = argmax_rows(target[:n_nodes])
+    t = argmax_rows(target[:n_nodes]) if tokens is None else np.asarray(tokens[:n_nodes], dtype=np.int64)
     cur = 0
     path = [0]
     while True:
@@ -441,6 +449,76 @@ def accept(target: np.ndarray, node_token: np.ndarray, parent: np.ndarray,
     src[:k + 1] = prefix_len + np.array(path)
     dst[:k + 1] = prefix_len + np.arange(k + 1)
     return Acceptance(p, k + 1, int(t[cur]), src, dst, prefix_len + k + 1, t)
+
+
+# --------------------------------------------------------------------------
+# Temperature > 0: one draw of the target's token per tree node
+# --------------------------------------------------------------------------
+
+_PHILOX_M = (0xD2E7470EE14C6C93, 0xCA5A826395121157)
+_PHILOX_W = (0x9E3779B97F4A7C15, 0xBB67AE8584CAA73B)
+_LO32 = np.uint64(0xFFFFFFFF)
+
+
+def _mulhilo64(a: np.ndarray, b: int):
+    """(high, low) 64-bit halves of the 128-bit products a * b (uint64)."""
+    b = np.uint64(b)
+    a_lo, a_hi = a & _LO32, a >> np.uint64(32)
+    b_lo, b_hi = b & _LO32, b >> np.uint64(32)
+    ll, lh, hl, hh = a_lo * b_lo, a_lo * b_hi, a_hi * b_lo, a_hi * b_hi
+    mid = (ll >> np.uint64(32)) + (lh & _LO32) + (hl & _LO32)
+    hi = hh + (lh >> np.uint64(32)) + (hl >> np.uint64(32)) + (mid >> np.uint64(32))
+    return hi, a * b
+
+
+def philox4x64(counter, key) -> np.ndarray:
+    """Philox4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers:
+    as easy as 1, 2, 3", SC 2011): ten rounds of two 64x64 -> 128-bit
+    multiplications by the published multipliers, a Weyl-sequence key bump
+    between rounds.  ``counter`` is four uint64 arrays (broadcast), ``key``
+    two uint64; returns [4, ...] uint64 outputs."""
+    c = [np.asarray(x, dtype=np.uint64) for x in np.broadcast_arrays(*counter)]
+    k0, k1 = int(key[0]) & (2 ** 64 - 1), int(key[1]) & (2 ** 64 - 1)
+    with np.errstate(over="ignore"):
+        for _ in range(10):
+            hi0, lo0 = _mulhilo64(c[0], _PHILOX_M[0])
+            hi1, lo1 = _mulhilo64(c[2], _PHILOX_M[1])
+            c = [hi1 ^ c[1] ^ np.uint64(k0), lo1, hi0 ^ c[3] ^ np.uint64(k1), lo0]
+            k0 = (k0 + _PHILOX_W[0]) & (2 ** 64 - 1)
+            k1 = (k1 + _PHILOX_W[1]) & (2 ** 64 - 1)
+    return np.stack(c)
+
+
+def uniforms(V: int, node: int, req: int, seed: int, offset: int) -> np.ndarray:
+    """u_v in (0, 1), float64, for v < V: output word v % 4 of Philox4x64-10
+    at counter (v // 4, node, req, 0) with key (seed, offset); the top 52
+    bits plus one half, times 2^-52 (every step exact in float64)."""
+    blocks = (V + 3) // 4
+    out = philox4x64((np.arange(blocks, dtype=np.uint64), node, req, 0), (seed, offset))
+    words = out.T.reshape(-1)[:V]
+    return ((words >> np.uint64(12)).astype(np.float64) + 0.5) * 2.0 ** -52
+
+
+def sample_rows(target: np.ndarray, temperature: float, seed: int, offset: int, req: int) -> np.ndarray:
+    """One draw from softmax(z / temperature) per row (reading R10).
+
+    Gumbel-max: token = argmax_v (z_v / T + g_v), g_v = -log(-log u_v),
+    which is a draw from softmax(z / T) (the Gumbel-max identity).  The
+    perturbed score is formed in float64 (z times the float64 value of 1/T)
+    and rounded once to float32; the argmax takes the lowest token id among
+    equal maxima, like the temperature-0 argmax.  NaN logits are rejected.
+    """
+    x = np.asarray(target, dtype=np.float64)
+    if np.isnan(x).any():
+        raise ValueError("NaN target logits")
+    inv_t = 1.0 / float(temperature)
+    out = np.empty(x.shape[0], dtype=np.int32)
+    for i in range(x.shape[0]):
+        u = uniforms(x.shape[1], i, req, seed, offset)
+        g = -np.log(-np.log(u))
+        s32 = (x[i] * inv_t + g).astype(np.float32)
+        out[i] = int(np.argmax(s32))
+    return out
 
 
 def compact(k_cache: np.ndarray, v_cache: np.ndarray, req: int, acc: Acceptance,

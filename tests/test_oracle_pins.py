@@ -595,3 +595,86 @@ def test_pins_catch_a_wrong_scale_in_attention():
     out, _ = oracle.tree_attention(q, k, v, P, st["anc"], st["n_nodes"], scale * 1.01)
     ref = _sdpa_reference(q, k, v, P, st["parent"], st["n_nodes"], scale, 0, 0)
     assert np.max(np.abs(out[(0, 0, 1, 0)] - ref[1, 0])) > 1e-6
+
+
+# ---------------------------------------------------------------- temperature > 0 (reading R10)
+
+@pytest.mark.parametrize("ctr,key", [((1, 0, 0, 0), (5, 7)), ((0, 6, 0, 0), (2 ** 64 - 1, 3)),
+                                     ((17, 2, 9, 4), (123456789, 987654321))])
+def test_philox4x64_matches_numpy_bit_generator(ctr, key):
+    """The oracle's Philox4x64-10 against numpy's Philox bit generator (a
+    library implementation of the same published generator), which first
+    advances its 256-bit counter by one and then emits the four words."""
+    c0, c1, c2, c3 = ctr
+    start = (c0 - 1) % 2 ** 64, c1 - (1 if c0 == 0 else 0), c2, c3
+    bg = np.random.Philox(key=np.array(key, dtype=np.uint64), counter=np.array(start, dtype=np.uint64))
+    raw = bg.random_raw(8)
+    ours = oracle.philox4x64((np.array([c0, (c0 + 1) % 2 ** 64], dtype=np.uint64),
+                              np.array([c1, c1 + (1 if c0 == 2 ** 64 - 1 else 0)], dtype=np.uint64), c2, c3), key)
+    assert np.array_equal(ours.T.reshape(-1), raw)
+
+
+def test_uniforms_are_open_unit_interval_and_distinct_per_counter():
+    u = oracle.uniforms(1001, 3, 2, seed=11, offset=5)
+    assert u.shape == (1001,) and np.all(u > 0.0) and np.all(u < 1.0)
+    assert not np.array_equal(u, oracle.uniforms(1001, 4, 2, seed=11, offset=5))     # another node
+    assert not np.array_equal(u, oracle.uniforms(1001, 3, 2, seed=11, offset=6))     # another round
+    # a Kolmogorov-Smirnov distance consistent with uniform draws
+    d = np.max(np.abs(np.sort(u) - (np.arange(1, 1002) - 0.5) / 1001))
+    assert d < 1.63 / math.sqrt(1001) + 0.5 / 1001
+
+
+def _chi2(counts, probs):
+    n = counts.sum()
+    e = probs * n
+    return float(((counts - e) ** 2 / e).sum())
+
+
+def test_sampling_follows_tempered_softmax():
+    """Gumbel-max draws over many seeds follow softmax(z / T): chi-square
+    with 4 degrees of freedom below its 1e-4 tail (23.5)."""
+    z = np.array([1.0, 0.2, -0.5, 2.0, 0.0])
+    T = 0.8
+    p = np.exp(z / T - np.max(z / T))
+    p /= p.sum()
+    counts = np.zeros(5)
+    for seed in range(20000):
+        counts[oracle.sample_rows(z[None], T, seed, 0, 0)[0]] += 1
+    assert _chi2(counts, p) < 23.5
+
+
+def test_sampling_cold_limit_is_argmax():
+    g = np.random.default_rng(4)
+    x = np.round(g.normal(size=(6, 300)) * 100) / 100 + np.arange(300) * 1e-5   # distinct values
+    assert np.array_equal(oracle.sample_rows(x, 1e-6, 9, 1, 0), oracle.argmax_rows(x))
+
+
+def test_tree_walk_at_temperature_keeps_the_target_distribution():
+    """Reading R10 on a two-level tree: the first committed token follows the
+    root's tempered target distribution, and, when it is a tree child, the
+    second one follows that child's (chi-square, 1e-4 tails)."""
+    T = 1.3
+    V = 4
+    target = np.array([[0.5, 1.5, -1.0, 0.0],     # root
+                       [1.0, -0.5, 0.3, 0.2],     # node 1 (token 1)
+                       [0.0, 0.0, 2.0, -2.0],     # node 2 (token 0)
+                       [0.4, 0.1, 0.1, 0.3]])     # node 3 (token 2, child of node 1)
+    node_token = np.array([7, 1, 0, 2], np.int32)
+    parent = np.array([-1, 0, 0, 1], np.int32)
+
+    def pr(row):
+        e = np.exp(target[row] / T - np.max(target[row] / T))
+        return e / e.sum()
+    first = np.zeros(V)
+    second = {1: np.zeros(V), 2: np.zeros(V)}
+    for seed in range(12000):
+        t = oracle.sample_rows(target, T, seed, 0, 0)
+        a = oracle.accept(target, node_token, parent, 4, 2, 0, tokens=t)
+        toks = [int(node_token[n]) for n in a.path[1:a.accept_len]] + [a.next_bonus]
+        first[toks[0]] += 1
+        if a.accept_len >= 2:
+            node = int(a.path[1])
+            second[node][toks[1]] += 1
+    assert _chi2(first, pr(0)) < 21.1            # 3 degrees of freedom
+    assert _chi2(second[1], pr(1)) < 21.1
+    assert _chi2(second[2], pr(2)) < 21.1

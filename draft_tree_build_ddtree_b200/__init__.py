@@ -26,6 +26,7 @@ import torch
 __all__ = [
     "DDTreeError", "KVDesc", "lib", "ddtree_topk", "ddtree_build", "ddtree_tree_attn",
     "ddtree_accept", "ddtree_round", "device_status", "RoundBuffers", "Workspace", "Sampling",
+    "ddtree_tree_kv_write",
     "BF16", "F32",
 ]
 
@@ -68,7 +69,8 @@ class RoundArgs(ctypes.Structure):
                 ("next_bonus", _vp), ("src_slot", _vp), ("dst_slot", _vp),
                 ("new_prefix_len", _vp),
                 ("ws", _vp), ("ws_bytes", _sz),
-                ("gain_floor", _vp), ("sampling", ctypes.POINTER(Sampling))]
+                ("gain_floor", _vp), ("sampling", ctypes.POINTER(Sampling)),
+                ("tree_q_in", _vp), ("tree_k_in", _vp), ("tree_v_in", _vp), ("rope_theta", ctypes.c_double)]
 
 
 _SIGS = {
@@ -77,6 +79,8 @@ _SIGS = {
     "ddtree_build": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "ddtree_build_ex": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i,
                              _vp, _vp]),
+    "ddtree_tree_kv_write": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, ctypes.POINTER(KVDesc), _vp, _i,
+                                  ctypes.c_double, _vp, _vp, _vp]),
     "ddtree_attn_workspace_bytes": (_sz, [ctypes.POINTER(KVDesc), _i]),
     "ddtree_tree_attn": (_i, [_vp, _vp, _vp, _i, ctypes.POINTER(KVDesc), _vp, _vp, _vp, _vp, _i,
                               _vp, _vp, _vp, _sz, _vp]),
@@ -291,6 +295,23 @@ def ddtree_tree_attn(q, k_cache, v_cache, kv: KVDesc, prefix_len, anc, n_nodes, 
     return out, out_lse
 
 
+def ddtree_tree_kv_write(k_in, v_in, depth, n_nodes, prefix_len, kv: KVDesc, k_cache, v_cache, B,
+                         rope_theta: float = 1e6, q_in=None, q_out=None, block_table=None):
+    """Rotate the tree nodes' Q/K to position P + depth and write K/V into the
+    cache tail (ddtree_tree_kv_write); q_out defaults to q_in (in place)."""
+    for t, nm in ((k_in, "k_in"), (v_in, "v_in"), (depth, "depth"), (n_nodes, "n_nodes"),
+                  (prefix_len, "prefix_len"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _contig(t, nm)
+    if q_in is not None and q_out is None:
+        q_out = q_in
+    _check(lib().ddtree_tree_kv_write(_ptr(q_in), _ptr(q_out), _ptr(k_in), _ptr(v_in), _dtype_code(k_in),
+                                      _ptr(depth), _ptr(n_nodes), _ptr(prefix_len), ctypes.byref(kv),
+                                      _ptr(block_table), B, float(rope_theta), _ptr(k_cache), _ptr(v_cache),
+                                      _stream()),
+           "ddtree_tree_kv_write")
+    return q_out
+
+
 # ------------------------------------------------------------------ stage 4
 
 @dataclasses.dataclass
@@ -373,6 +394,10 @@ class RoundBuffers:
     ws: torch.Tensor = None
     gain_floor: Optional[torch.Tensor] = None   # float32 [n_req]: adaptive-budget floor of the build
     sampling: Optional[Sampling] = None         # temperature > 0 verification (None: greedy)
+    tree_q_in: Optional[torch.Tensor] = None    # un-rotated tree Q/K/V: the round rotates and writes them
+    tree_k_in: Optional[torch.Tensor] = None
+    tree_v_in: Optional[torch.Tensor] = None
+    rope_theta: float = 1e6
     _args: RoundArgs = None
 
     def allocate_outputs(self):
@@ -413,6 +438,8 @@ class RoundBuffers:
         a.gain_floor = _ptr(self.gain_floor)
         if self.sampling is not None:
             a.sampling = ctypes.pointer(self.sampling)
+        a.tree_q_in, a.tree_k_in, a.tree_v_in = _ptr(self.tree_q_in), _ptr(self.tree_k_in), _ptr(self.tree_v_in)
+        a.rope_theta = float(self.rope_theta)
         need = lib().ddtree_round_workspace_bytes(ctypes.byref(a))
         if need == 0:
             raise DDTreeError("invalid round geometry")

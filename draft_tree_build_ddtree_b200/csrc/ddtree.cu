@@ -16,6 +16,7 @@
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "attn_tc2.cuh"
+#include "rope.cuh"
 
 using namespace ddt;
 
@@ -273,6 +274,51 @@ int attn_launch(const void* q, const void* k_cache, const void* v_cache, int dty
   return launch_status();
 }
 
+// ------------------------------------------------------------------ tree K/V write with rotary positions
+int rope_launch(const void* q_in, void* q_out, const void* k_in, const void* v_in, int dtype, const int32_t* depth,
+                const int32_t* n_nodes, const int32_t* prefix_len, const ddtree_kv_desc* kv,
+                const int32_t* block_table, int B, double theta, void* k_cache, void* v_cache, cudaStream_t s) {
+  int st = kv_check(kv);
+  if (st) return st;
+  if (!dtype_ok(dtype) || B < 0 || B > MAX_B) return DDTREE_ERR_INVALID_ARG;
+  if (!k_in || !v_in || !depth || !n_nodes || !prefix_len || !k_cache || !v_cache) return DDTREE_ERR_INVALID_ARG;
+  if ((q_in == nullptr) != (q_out == nullptr)) return DDTREE_ERR_INVALID_ARG;
+  if (kv->paged && !block_table) return DDTREE_ERR_INVALID_ARG;
+  if (theta != theta) return DDTREE_ERR_INVALID_ARG;
+  for (const void* p : {(const void*)q_in, (const void*)q_out, k_in, v_in, (const void*)k_cache, (const void*)v_cache})
+    if (p && !aligned16(p)) return DDTREE_ERR_INVALID_ARG;
+  RopeArgs a;
+  a.q_in = (const unsigned char*)q_in;
+  a.q_out = (unsigned char*)q_out;
+  a.k_in = (const unsigned char*)k_in;
+  a.v_in = (const unsigned char*)v_in;
+  a.depth = depth;
+  a.n_nodes = n_nodes;
+  a.prefix_len = prefix_len;
+  a.block_table = block_table;
+  a.k_cache = (unsigned char*)k_cache;
+  a.v_cache = (unsigned char*)v_cache;
+  a.layers = kv->layers;
+  a.n_req = kv->n_req;
+  a.n = B + 1;
+  a.Hq = kv->Hq;
+  a.Hkv = kv->Hkv;
+  a.D = kv->D;
+  a.paged = kv->paged;
+  a.s_max = kv->s_max;
+  a.num_blocks = kv->num_blocks;
+  a.max_blocks = kv->max_blocks;
+  a.theta = theta;
+  const long long grid = (long long)a.layers * a.n_req * a.n;
+  if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
+  const size_t smem = (size_t)(kv->D / 2) * sizeof(float2);
+  if (dtype == DDTREE_BF16)
+    tree_rope_kernel<__nv_bfloat16><<<(unsigned)grid, ROPE_THREADS, smem, s>>>(a);
+  else
+    tree_rope_kernel<float><<<(unsigned)grid, ROPE_THREADS, smem, s>>>(a);
+  return launch_status();
+}
+
 // ------------------------------------------------------------------ accept
 struct AcceptPlan {
   int cpr, chunk;
@@ -407,6 +453,14 @@ int ddtree_build_ex(const int32_t* ids, const float* lp, const int32_t* root_tok
                       n_nodes, stream, flags, gain_floor, build_path);
 }
 
+int ddtree_tree_kv_write(const void* q_in, void* q_out, const void* k_in, const void* v_in, int dtype,
+                         const int32_t* depth, const int32_t* n_nodes, const int32_t* prefix_len,
+                         const ddtree_kv_desc* kv, const int32_t* block_table, int B, double rope_theta,
+                         void* k_cache, void* v_cache, cudaStream_t stream) {
+  return rope_launch(q_in, q_out, k_in, v_in, dtype, depth, n_nodes, prefix_len, kv, block_table, B, rope_theta,
+                     k_cache, v_cache, stream);
+}
+
 size_t ddtree_attn_workspace_bytes(const ddtree_kv_desc* kv, int B) {
   if (kv_check(kv) || B < 0 || B > MAX_B) return 0;
   return attn_ws(kv, B, DDTREE_BF16);
@@ -467,6 +521,7 @@ int ddtree_round_launch_count(const ddtree_round_args* a) {
   int n = 2;                                                             // top-K, build
   n += 1;                                                                // attention
   if (use_tc_attn(a->dtype, &a->kv) && attn_tc_ws_bytes(geom_of(&a->kv, a->B), num_sms()) > 0) n += 1;   // combine
+  if (a->tree_k_in != nullptr) n += 1;                                   // tree K/V write
   n += 1;                                                                // argmax (+ walk)
   if (a->kv.layers > WALK_FUSE_MAX_LAYERS) n += 1;                       // walk and compaction
   return n;
@@ -486,6 +541,12 @@ int ddtree_round(const ddtree_round_args* a, cudaStream_t stream) {
   st = build_launch(a->ids, a->lp, a->root_token, a->n_req, a->L, a->K, a->B, a->node_token, a->parent, a->depth,
                     a->node_rank, a->score, a->anc, a->n_nodes, stream, 0, a->gain_floor, nullptr);
   if (st) return st;
+  if (a->tree_k_in != nullptr) {   // the tree's positions are known now: rotate and write its K/V
+    st = rope_launch(a->tree_q_in, a->tree_q_in ? (void*)a->q : nullptr, a->tree_k_in, a->tree_v_in, a->dtype,
+                     a->depth, a->n_nodes, a->prefix_len, &a->kv, a->block_table, a->B, a->rope_theta, a->k_cache,
+                     a->v_cache, stream);
+    if (st) return st;
+  }
   st = attn_launch(a->q, a->k_cache, a->v_cache, a->dtype, &a->kv, a->block_table, a->prefix_len, a->anc,
                    a->n_nodes, a->B, a->attn_out, a->attn_lse, ws + off_attn, off_acc - off_attn, stream);
   if (st) return st;

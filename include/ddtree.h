@@ -187,6 +187,31 @@ int ddtree_build_ex(const int32_t* ids, const float* lp, const int32_t* root_tok
 /* Stage 3: ancestor-only tree attention (Deep Dive §4).                  */
 /* ---------------------------------------------------------------------- */
 
+/*
+ * ddtree_tree_kv_write: the verify layer's neighbour before tree attention
+ * ("DDTree Deep Dive" §3, tree_compile: a node's position id is P + depth,
+ * siblings share it; §5: node i's K/V sit at cache slot P + i).  For every
+ * layer, request r and live node i < n_nodes[r]:
+ *   q_out[l][r][i] = rope(q_in[l][r][i], P_r + depth[r][i])   (if q_in)
+ *   K cache slot P_r + i = rope(k_in[l][r][i], P_r + depth[r][i])
+ *   V cache slot P_r + i = v_in[l][r][i]
+ * rope: the rotary position embedding (Su et al., "RoFormer", §3.4) with the
+ * half-split pairing: for i < D/2 the pair (x_i, x_{i+D/2}) turns by the
+ * angle pos * rope_theta^(-2i/D) (the Qwen3 family uses rope_theta = 1e6);
+ * rope_theta <= 0 writes K unrotated.  The angles are computed in fp64, the
+ * rotation in fp32, the result rounded to the dtype.
+ * q_in, q_out  device [layers][n_req][B+1][Hq][D] or both NULL; q_out may
+ *              alias q_in.
+ * k_in, v_in   device [layers][n_req][B+1][Hkv][D].
+ * depth, n_nodes  device, from ddtree_build.  prefix_len device [n_req].
+ * A request whose tree does not fit its cache (or whose block-table entry is
+ * out of range) is skipped and flags DDTREE_STATUS_CAPACITY.
+ */
+int ddtree_tree_kv_write(const void* q_in, void* q_out, const void* k_in, const void* v_in, int dtype,
+                         const int32_t* depth, const int32_t* n_nodes, const int32_t* prefix_len,
+                         const ddtree_kv_desc* kv, const int32_t* block_table, int B, double rope_theta,
+                         void* k_cache, void* v_cache, cudaStream_t stream);
+
 size_t ddtree_attn_workspace_bytes(const ddtree_kv_desc* kv, int B);
 
 /*
@@ -328,6 +353,15 @@ typedef struct {
   /* optional (NULL: greedy): verification at temperature > 0, as for
    * ddtree_accept_ex */
   const ddtree_sampling* sampling;
+  /* optional (tree_k_in NULL: none): the tree nodes' un-rotated Q, K, V
+   * ([layers][n_req][B+1][H][D]); after the build the round runs
+   * ddtree_tree_kv_write with them, writing the rotated Q into `q` (which
+   * must then be writable; tree_q_in NULL leaves q as given) and K/V into the
+   * cache tail, before the attention. */
+  const void* tree_q_in;
+  const void* tree_k_in;
+  const void* tree_v_in;
+  double rope_theta;
 } ddtree_round_args;
 
 /* Bytes of a->ws the round needs (0 for an invalid geometry).  The

@@ -46,6 +46,9 @@ R7  Greedy verification (temperature 0): the target's argmax takes the
 R9  Adaptive budget: a node is worth adding while its gain q(u) exceeds the
     cost c of verifying one more node (in accepted tokens); the build keeps
     the pops whose score is strictly above log c.
+R11 Rotary positions: the verify layer turns the tree nodes' Q and K at
+    position P + depth with the half-split RoPE pairing and base theta
+    (1e6 for the Qwen3 family the pages use; a parameter).
 R10 Temperature T > 0: the verifier draws the target's token at every tree
     node from softmax(z / T) and walks as at temperature 0; each committed
     token is then a draw from the target at its context, so the output
@@ -449,6 +452,58 @@ def accept(target: np.ndarray, node_token: np.ndarray, parent: np.ndarray,
     src[:k + 1] = prefix_len + np.array(path)
     dst[:k + 1] = prefix_len + np.arange(k + 1)
     return Acceptance(p, k + 1, int(t[cur]), src, dst, prefix_len + k + 1, t)
+
+
+# --------------------------------------------------------------------------
+# Tree K/V into the cache with rotary positions (the verify layer's neighbour)
+# --------------------------------------------------------------------------
+
+def tree_positions(depth: np.ndarray, prefix_len: int, n_nodes: int) -> np.ndarray:
+    """Sequence position of every live node: P + depth (Deep Dive §3,
+    tree_compile: a node's position id is its depth past the committed
+    prefix)."""
+    return prefix_len + np.asarray(depth[:n_nodes], dtype=np.int64)
+
+
+def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
+    """Rotary position embedding (Su et al., "RoFormer", §3.4), half-split
+    pairing (reading R11): for i < D/2, the pair (x_i, x_{i+D/2}) turns by the
+    angle pos * theta^(-2i/D).  ``x`` is [..., D] with the position axis
+    leading (``pos`` broadcasts over the middle axes); float64."""
+    x = np.asarray(x, dtype=np.float64)
+    D = x.shape[-1]
+    h = D // 2
+    inv = theta ** (-(2.0 * np.arange(h)) / D)
+    ang = np.asarray(pos, dtype=np.float64).reshape((-1,) + (1,) * (x.ndim - 1)) * inv
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = x[..., :h], x[..., h:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
+def write_tree_kv(k_cache: np.ndarray, v_cache: np.ndarray, k_in: np.ndarray, v_in: np.ndarray,
+                  depth: np.ndarray, prefix_len: np.ndarray, n_nodes: np.ndarray, theta: float,
+                  block_table: Optional[np.ndarray] = None) -> None:
+    """The tree nodes' K and V into their cache slots (Deep Dive §5: tree
+    K/V sit in the cache tail, node i at slot P + i): K rotated at position
+    P + depth[i], V as is.  k_in / v_in are [layers, N, n, Hkv, D]; the caches
+    are contiguous [layers, N, S, Hkv, D] or paged pools with ``block_table``;
+    writes float64 values into them (the caller rounds)."""
+    layers, N = k_in.shape[0], k_in.shape[1]
+    for r in range(N):
+        nn = int(n_nodes[r])
+        P = int(prefix_len[r])
+        pos = tree_positions(depth[r], P, nn)
+        slots = P + np.arange(nn)
+        for l in range(layers):
+            kr = rope(k_in[l, r, :nn], pos, theta) if theta > 0 else np.asarray(k_in[l, r, :nn], np.float64)
+            vr = np.asarray(v_in[l, r, :nn], np.float64)
+            if block_table is None:
+                k_cache[l, r, slots] = kr
+                v_cache[l, r, slots] = vr
+            else:
+                blk = block_table[r, slots // PAGE]
+                k_cache[l, blk, slots % PAGE] = kr
+                v_cache[l, blk, slots % PAGE] = vr
 
 
 # --------------------------------------------------------------------------

@@ -678,3 +678,47 @@ def test_tree_walk_at_temperature_keeps_the_target_distribution():
     assert _chi2(first, pr(0)) < 21.1            # 3 degrees of freedom
     assert _chi2(second[1], pr(1)) < 21.1
     assert _chi2(second[2], pr(2)) < 21.1
+
+
+# ---------------------------------------------------------------- rotary positions (reading R11)
+
+def test_rope_is_complex_rotation():
+    """Half-split RoPE equals multiplying z_i = x_i + i x_{i+D/2} by
+    exp(i pos theta^(-2i/D)) (numpy complex arithmetic)."""
+    g = np.random.default_rng(2)
+    x = g.normal(size=(5, 3, 16))
+    pos = np.array([0, 1, 7, 300, 32768])
+    theta = 1e6
+    z = x[..., :8] + 1j * x[..., 8:]
+    w = z * np.exp(1j * pos[:, None, None] * theta ** (-np.arange(8) * 2.0 / 16))
+    ref = np.concatenate([w.real, w.imag], axis=-1)
+    assert np.allclose(oracle.rope(x, pos, theta), ref, rtol=0, atol=1e-12)
+
+
+def test_rope_properties():
+    g = np.random.default_rng(3)
+    q, k = g.normal(size=(1, 128)), g.normal(size=(1, 128))
+    assert np.allclose(oracle.rope(q, [0], 1e6), q, atol=0)              # position 0: identity
+    r = oracle.rope(q, [12345], 1e6)
+    assert np.allclose(r[0, :64] ** 2 + r[0, 64:] ** 2, q[0, :64] ** 2 + q[0, 64:] ** 2, atol=1e-12)
+    # the score depends on the relative position only
+    for m, n, sft in ((5, 2, 100), (40000, 3, 777)):
+        a = oracle.rope(q, [m], 1e6) @ oracle.rope(k, [n], 1e6).T
+        b = oracle.rope(q, [m + sft], 1e6) @ oracle.rope(k, [n + sft], 1e6).T
+        assert abs(float((a - b)[0, 0])) < 1e-9
+
+
+def test_write_tree_kv_places_rotated_rows():
+    g = np.random.default_rng(4)
+    L_, N, n, H, D = 2, 2, 5, 1, 8
+    k_in, v_in = g.normal(size=(L_, N, n, H, D)), g.normal(size=(L_, N, n, H, D))
+    depth = np.array([[0, 1, 1, 2, -1], [0, 1, 2, 3, 4]])
+    nn = np.array([4, 5])
+    P = np.array([3, 0])
+    kc, vc = np.zeros((L_, N, 12, H, D)), np.zeros((L_, N, 12, H, D))
+    oracle.write_tree_kv(kc, vc, k_in, v_in, depth, P, nn, 1e4)
+    for r in range(N):
+        for i in range(nn[r]):
+            assert np.allclose(kc[:, r, P[r] + i], oracle.rope(k_in[:, r, i], [P[r] + depth[r, i]] * L_, 1e4))
+            assert np.array_equal(vc[:, r, P[r] + i], v_in[:, r, i])
+    assert np.all(kc[:, 0, :3] == 0) and np.all(kc[:, 0, 7:] == 0)      # nothing outside the tree slots

@@ -96,6 +96,7 @@ _SIGS = {
     "ddtree_status_string": (ctypes.c_char_p, [_i]),
     "ddtree_device_status": (_i, [_vp, ctypes.POINTER(ctypes.c_uint)]),
     "ddtree_version": (_i, []),
+    "ddtree_last_error": (ctypes.c_char_p, []),
     "ddtree_topk_static_ws": (_i, [_vp, _i, _i, _i, _ll, _i, _vp, _vp, _vp, _vp]),
     "ddtree_debug_attn_timeout": (_i, [ctypes.c_ulonglong, _i]),
     "ddtree_round_host": (_i, [ctypes.POINTER(RoundArgs), _vp, _vp]),
@@ -127,6 +128,8 @@ def exported_symbols():
 def _check(status: int, what: str):
     if status != 0:
         msg = lib().ddtree_status_string(status).decode()
+        if status == 3:
+            msg += f" [{lib().ddtree_last_error().decode()}]"
         raise DDTreeError(f"{what}: {msg} ({status})")
 
 

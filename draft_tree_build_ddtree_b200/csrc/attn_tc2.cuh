@@ -541,27 +541,30 @@ inline int attn_tc_launch(const void* q, const void* kc, const void* vc, const i
   CUtensorMap mq, mk, mv;
   if (!make_map_4d(&mq, q, (uint64_t)g.Hq, (uint64_t)g.n, (uint64_t)g.layers * g.n_req, (uint32_t)p.G,
                    (uint32_t)(TC_BM / p.G)))
-    return DDTREE_ERR_CUDA;
+    return cuda_fail_msg("tree attention: tensor map of q");
   if (!g.paged) {
-    if (!make_map_4d(&mk, kc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, T2_BN)) return DDTREE_ERR_CUDA;
-    if (!make_map_4d(&mv, vc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, T2_BN)) return DDTREE_ERR_CUDA;
+    if (!make_map_4d(&mk, kc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, T2_BN) ||
+        !make_map_4d(&mv, vc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, T2_BN))
+      return cuda_fail_msg("tree attention: tensor map of the cache");
   } else {
-    if (!make_map_4d(&mk, kc, g.Hkv, DDTREE_PAGE, (uint64_t)g.layers * g.num_blocks, 1, DDTREE_PAGE))
-      return DDTREE_ERR_CUDA;
-    if (!make_map_4d(&mv, vc, g.Hkv, DDTREE_PAGE, (uint64_t)g.layers * g.num_blocks, 1, DDTREE_PAGE))
-      return DDTREE_ERR_CUDA;
+    if (!make_map_4d(&mk, kc, g.Hkv, DDTREE_PAGE, (uint64_t)g.layers * g.num_blocks, 1, DDTREE_PAGE) ||
+        !make_map_4d(&mv, vc, g.Hkv, DDTREE_PAGE, (uint64_t)g.layers * g.num_blocks, 1, DDTREE_PAGE))
+      return cuda_fail_msg("tree attention: tensor map of the paged cache");
   }
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(tree_attn_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)t2_smem_bytes()) != cudaSuccess)
-      return DDTREE_ERR_CUDA;
+    cudaError_t e = cudaFuncSetAttribute(tree_attn_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)t2_smem_bytes());
+    if (e != cudaSuccess) return cuda_fail(e, "tree attention (two M-tiles): shared-memory attribute");
     attr_set = true;
   }
   const long long grid = (long long)d.units2 * d.splits;
   if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
   tree_attn_tc2_kernel<<<(unsigned)grid, T2_THREADS, t2_smem_bytes(), stream>>>(mq, mk, mv, p);
-  if (cudaGetLastError() != cudaSuccess) return DDTREE_ERR_CUDA;
+  {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "tree attention (two M-tiles): launch");
+  }
   if (d.splits > 1) {
     // the combine kernel walks M-tile units
     TcParams c;
@@ -585,7 +588,8 @@ inline int attn_tc_launch(const void* q, const void* kc, const void* vc, const i
       tree_attn_combine_kernel<8><<<c.units * (TC_D / 8), TC_BM, 0, stream>>>(c);
     else
       tree_attn_combine_kernel<TC_MAX_SPLITS><<<c.units * (TC_D / 8), TC_BM, 0, stream>>>(c);
-    if (cudaGetLastError() != cudaSuccess) return DDTREE_ERR_CUDA;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "tree attention: combine launch");
   }
   return DDTREE_OK;
 }

@@ -4,10 +4,26 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdio.h>
 
 #include "ddtree.h"
 
 namespace ddt {
+
+// The last host-side CUDA failure behind a DDTREE_ERR_CUDA return: the
+// call that failed and the runtime's message (ddtree_last_error()).
+inline char* last_error_buf() {
+  static char buf[256] = "";
+  return buf;
+}
+inline int cuda_fail(cudaError_t e, const char* where) {
+  snprintf(last_error_buf(), 256, "%s: %s", where, cudaGetErrorString(e));
+  return DDTREE_ERR_CUDA;
+}
+inline int cuda_fail_msg(const char* where) {
+  snprintf(last_error_buf(), 256, "%s", where);
+  return DDTREE_ERR_CUDA;
+}
 
 // Device status word read by ddtree_device_status(); bits DDTREE_STATUS_*.
 __device__ unsigned int g_status;

@@ -49,7 +49,7 @@ bool dtype_ok(int dtype) { return dtype == DDTREE_BF16 || dtype == DDTREE_F32; }
 
 int launch_status() {
   cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? DDTREE_OK : DDTREE_ERR_CUDA;
+  return e == cudaSuccess ? DDTREE_OK : cuda_fail(e, "kernel launch");
 }
 
 // Opt a kernel in to `bytes` of dynamic shared memory when its static plus
@@ -663,7 +663,9 @@ int ddtree_device_status(cudaStream_t stream, unsigned int* bits) {
   return DDTREE_OK;
 }
 
-int ddtree_version(void) { return 100; }
+int ddtree_version(void) { return 200; }
+
+const char* ddtree_last_error(void) { return last_error_buf(); }
 
 }  // extern "C"
 

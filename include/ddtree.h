@@ -493,6 +493,10 @@ int ddtree_device_status(cudaStream_t stream, unsigned int* bits);
  */
 int ddtree_debug_attn_timeout(unsigned long long wait_ns, int withhold_tile);
 
+/* The call and the CUDA runtime's message behind the last DDTREE_ERR_CUDA
+ * return of a host-side launch or set-up step (empty before any). */
+const char* ddtree_last_error(void);
+
 /* Library version, major*10000 + minor*100 + patch. */
 int ddtree_version(void);
 

@@ -26,7 +26,7 @@ import torch
 __all__ = [
     "DDTreeError", "KVDesc", "lib", "ddtree_topk", "ddtree_build", "ddtree_tree_attn",
     "ddtree_accept", "ddtree_round", "device_status", "RoundBuffers", "Workspace", "Sampling",
-    "ddtree_tree_kv_write",
+    "ddtree_tree_kv_write", "ddtree_lmhead_argmax", "ddtree_walk",
     "BF16", "F32",
 ]
 
@@ -70,7 +70,8 @@ class RoundArgs(ctypes.Structure):
                 ("new_prefix_len", _vp),
                 ("ws", _vp), ("ws_bytes", _sz),
                 ("gain_floor", _vp), ("sampling", ctypes.POINTER(Sampling)),
-                ("tree_q_in", _vp), ("tree_k_in", _vp), ("tree_v_in", _vp), ("rope_theta", ctypes.c_double)]
+                ("tree_q_in", _vp), ("tree_k_in", _vp), ("tree_v_in", _vp), ("rope_theta", ctypes.c_double),
+                ("target_hidden", _vp), ("lm_head", _vp), ("d_model", _i)]
 
 
 _SIGS = {
@@ -81,6 +82,10 @@ _SIGS = {
                              _vp, _vp]),
     "ddtree_tree_kv_write": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, ctypes.POINTER(KVDesc), _vp, _i,
                                   ctypes.c_double, _vp, _vp, _vp]),
+    "ddtree_lmhead_workspace_bytes": (_sz, [_i]),
+    "ddtree_lmhead_argmax": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
+    "ddtree_walk": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, ctypes.POINTER(KVDesc), _vp, _i,
+                         _vp, _vp, _vp, _vp, _vp, _vp]),
     "ddtree_attn_workspace_bytes": (_sz, [ctypes.POINTER(KVDesc), _i]),
     "ddtree_tree_attn": (_i, [_vp, _vp, _vp, _i, ctypes.POINTER(KVDesc), _vp, _vp, _vp, _vp, _i,
                               _vp, _vp, _vp, _sz, _vp]),
@@ -315,6 +320,38 @@ def ddtree_tree_kv_write(k_in, v_in, depth, n_nodes, prefix_len, kv: KVDesc, k_c
     return q_out
 
 
+_ws["lmhead"] = Workspace()
+
+
+def ddtree_lmhead_argmax(hidden: torch.Tensor, weight: torch.Tensor, out=None, out_max=None, ws=None):
+    """Per-row argmax of hidden [rows, d] @ weight[V, d]^T without writing the logits."""
+    _contig(hidden, "hidden")
+    _contig(weight, "weight")
+    if hidden.dtype != torch.bfloat16 or weight.dtype != torch.bfloat16:
+        raise DDTreeError("hidden and weight must be bf16")
+    rows, d = hidden.shape
+    V = weight.shape[0]
+    out = torch.empty((rows,), dtype=torch.int32, device=hidden.device) if out is None else out
+    w = _ws["lmhead"].get(lib().ddtree_lmhead_workspace_bytes(rows), hidden.device) if ws is None else ws
+    _check(lib().ddtree_lmhead_argmax(_ptr(hidden), _ptr(weight), rows, V, d, _ptr(out), _ptr(out_max), _ptr(w),
+                                      w.numel(), _stream()), "ddtree_lmhead_argmax")
+    return out
+
+
+def ddtree_walk(target_token, node_token, parent, n_nodes, L, prefix_len, k_cache=None, v_cache=None,
+                kv: Optional[KVDesc] = None, block_table=None, out: Optional["Accept"] = None, dtype=BF16):
+    """The verifier walk + compaction from per-node target tokens [n_req, B+1]."""
+    _contig(target_token, "target_token")
+    n_req, n = target_token.shape
+    a = alloc_accept(n_req, L, n - 1, target_token.device) if out is None else out
+    _check(lib().ddtree_walk(_ptr(target_token), _ptr(node_token), _ptr(parent), _ptr(n_nodes), n_req, L, n - 1,
+                             _ptr(prefix_len), _ptr(a.new_prefix_len), _ptr(k_cache), _ptr(v_cache),
+                             ctypes.byref(kv) if kv is not None else None, _ptr(block_table), int(dtype),
+                             _ptr(a.path), _ptr(a.accept_len), _ptr(a.next_bonus), _ptr(a.src_slot),
+                             _ptr(a.dst_slot), _stream()), "ddtree_walk")
+    return a
+
+
 # ------------------------------------------------------------------ stage 4
 
 @dataclasses.dataclass
@@ -401,6 +438,8 @@ class RoundBuffers:
     tree_k_in: Optional[torch.Tensor] = None
     tree_v_in: Optional[torch.Tensor] = None
     rope_theta: float = 1e6
+    target_hidden: Optional[torch.Tensor] = None   # [n_req*(B+1), d] bf16: argmax from the LM head instead
+    lm_head: Optional[torch.Tensor] = None         # [V, d] bf16
     _args: RoundArgs = None
 
     def allocate_outputs(self):
@@ -443,6 +482,8 @@ class RoundBuffers:
             a.sampling = ctypes.pointer(self.sampling)
         a.tree_q_in, a.tree_k_in, a.tree_v_in = _ptr(self.tree_q_in), _ptr(self.tree_k_in), _ptr(self.tree_v_in)
         a.rope_theta = float(self.rope_theta)
+        a.target_hidden, a.lm_head = _ptr(self.target_hidden), _ptr(self.lm_head)
+        a.d_model = 0 if self.target_hidden is None else int(self.target_hidden.shape[-1])
         need = lib().ddtree_round_workspace_bytes(ctypes.byref(a))
         if need == 0:
             raise DDTreeError("invalid round geometry")

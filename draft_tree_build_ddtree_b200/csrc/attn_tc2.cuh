@@ -72,6 +72,23 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
+// 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -99,7 +116,7 @@ struct T2Params {
   int stop_tile;
 };
 
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(T2_THREADS, 1)
 tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const T2Params p) {
   extern __shared__ __align__(1024) unsigned char smem_dyn[];
@@ -371,13 +388,13 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         l *= corr;
         if (jj > 0) {        // PV_t(jj-1) has completed (it precedes S_t(jj)); O_t is ours to rescale
 #pragma unroll 1
-          for (int c = 0; c < TC_D / 32; ++c) {
-            float o[32];
-            tmem_ld32(tm_o + c * 32, o);
+          for (int c = 0; c < TC_D / 16; ++c) {     // 16 columns at a time: S stays in registers
+            uint32_t o[16];
+            tmem_ld16(tm_o + c * 16, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= corr;
-            tmem_st32(tm_o + c * 32, o);
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+            tmem_st16(tm_o + c * 16, o);
           }
           tmem_wait_st();
         }
@@ -386,16 +403,16 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const float mneg = (m_used == -INFINITY) ? 0.f : -m_used;
       float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {       // 64 keys -> 32 packed columns per store
-        float pk[32];
+      for (int q4 = 0; q4 < 4; ++q4) {             // 32 keys -> 16 packed columns per store
+        uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float e0 = ex2_approx(fmaf(s[64 * half + 2 * c], sl2, mneg));
-          const float e1 = ex2_approx(fmaf(s[64 * half + 2 * c + 1], sl2, mneg));
+        for (int c = 0; c < 16; ++c) {
+          const float e0 = ex2_approx(fmaf(s[32 * q4 + 2 * c], sl2, mneg));
+          const float e1 = ex2_approx(fmaf(s[32 * q4 + 2 * c + 1], sl2, mneg));
           ls4[c & 3] += e0 + e1;
-          pk[c] = __uint_as_float(pack_bf16x2(e0, e1));
+          pk[c] = pack_bf16x2(e0, e1);
         }
-        tmem_st32(tm_s + 32 * half, pk);
+        tmem_st16(tm_s + 16 * q4, pk);
       }
       l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
       tmem_wait_st();

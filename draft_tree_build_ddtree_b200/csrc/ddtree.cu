@@ -17,6 +17,7 @@
 #include "attn_tc.cuh"
 #include "attn_tc2.cuh"
 #include "rope.cuh"
+#include "lmhead.cuh"
 
 using namespace ddt;
 
@@ -420,6 +421,66 @@ int accept_launch(const void* target_logits, int dtype, int V, long long row_str
   return launch_status();
 }
 
+// ------------------------------------------------------------------ LM head + walk
+int lmhead_check(const void* hidden, const void* weight, int rows, int V, int d, const void* out) {
+  if (!hidden || !weight || !out) return DDTREE_ERR_INVALID_ARG;
+  if (rows < 1 || rows > MAX_REQ * (MAX_B + 1) || V < 1 || V > MAX_V || d < 64 || d % 64 != 0 || d > 65536)
+    return DDTREE_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(weight)) return DDTREE_ERR_INVALID_ARG;
+  return DDTREE_OK;
+}
+
+// The walk and compaction from given per-node target tokens (target_token
+// [n_req][B+1]): one CTA per (request, layer, K/V).
+int walk_launch(const int32_t* target_token, const int32_t* node_token, const int32_t* parent,
+                const int32_t* n_nodes, int n_req, int L, int B, const int32_t* prefix_len, int32_t* new_prefix_len,
+                void* k_cache, void* v_cache, const ddtree_kv_desc* kv, const int32_t* block_table, int dtype,
+                int32_t* path, int32_t* accept_len, int32_t* next_bonus, int32_t* src_slot, int32_t* dst_slot,
+                cudaStream_t s) {
+  if (!target_token || !node_token || !parent || !n_nodes || !prefix_len || !new_prefix_len)
+    return DDTREE_ERR_INVALID_ARG;
+  if (new_prefix_len == prefix_len || !dtype_ok(dtype)) return DDTREE_ERR_INVALID_ARG;
+  if (n_req < 1 || n_req > MAX_REQ || L < 1 || L > MAX_L || B < 0 || B > MAX_B) return DDTREE_ERR_INVALID_ARG;
+  int row_bytes = 0;
+  if (k_cache) {
+    int st = kv_check(kv);
+    if (st) return st;
+    if (!v_cache || kv->n_req != n_req || (kv->paged && !block_table)) return DDTREE_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache)) return DDTREE_ERR_INVALID_ARG;
+    row_bytes = kv->Hkv * kv->D * esize_of(dtype);
+    if (row_bytes % 16 != 0) return DDTREE_ERR_UNSUPPORTED;
+  }
+  WalkArgs a;
+  a.node_token = node_token;
+  a.parent = parent;
+  a.n_nodes = n_nodes;
+  a.prefix_len = prefix_len;
+  a.argmax_ws = target_token;
+  a.n = B + 1;
+  a.L = L;
+  a.new_prefix_len = new_prefix_len;
+  a.target_argmax = nullptr;
+  a.path = path;
+  a.accept_len = accept_len;
+  a.next_bonus = next_bonus;
+  a.src_slot = src_slot;
+  a.dst_slot = dst_slot;
+  a.k_cache = (unsigned char*)k_cache;
+  a.v_cache = (unsigned char*)v_cache;
+  a.block_table = block_table;
+  a.layers = k_cache ? kv->layers : 1;
+  a.n_req = n_req;
+  a.paged = k_cache ? kv->paged : 0;
+  a.s_max = k_cache ? kv->s_max : 0;
+  a.num_blocks = k_cache ? kv->num_blocks : 0;
+  a.max_blocks = k_cache ? kv->max_blocks : 0;
+  a.row_bytes = row_bytes;
+  const size_t smem = (size_t)(B + 1) * 16;
+  dim3 grid2(n_req, a.layers * 2);
+  walk_compact_kernel<<<grid2, WALK_THREADS, smem, s>>>(a);
+  return launch_status();
+}
+
 }  // namespace
 
 // ======================================================================
@@ -485,6 +546,24 @@ int ddtree_accept_ex(const void* target_logits, int dtype, int V, long long row_
                        next_bonus, src_slot, dst_slot, ws, ws_bytes, stream, sampling);
 }
 
+size_t ddtree_lmhead_workspace_bytes(int rows) { return rows < 1 ? 0 : lm_ws_bytes(rows); }
+
+int ddtree_lmhead_argmax(const void* hidden, const void* weight, int rows, int V, int d, int32_t* out_argmax,
+                         float* out_max, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int st = lmhead_check(hidden, weight, rows, V, d, out_argmax);
+  if (st) return st;
+  if (!ws || !aligned16(ws) || ws_bytes < lm_ws_bytes(rows)) return DDTREE_ERR_INVALID_ARG;
+  return lmhead_launch(hidden, weight, rows, V, d, out_argmax, out_max, ws, num_sms(), stream, g_attn_wait_ns);
+}
+
+int ddtree_walk(const int32_t* target_token, const int32_t* node_token, const int32_t* parent, const int32_t* n_nodes,
+                int n_req, int L, int B, const int32_t* prefix_len, int32_t* new_prefix_len, void* k_cache,
+                void* v_cache, const ddtree_kv_desc* kv, const int32_t* block_table, int dtype, int32_t* path,
+                int32_t* accept_len, int32_t* next_bonus, int32_t* src_slot, int32_t* dst_slot, cudaStream_t stream) {
+  return walk_launch(target_token, node_token, parent, n_nodes, n_req, L, B, prefix_len, new_prefix_len, k_cache,
+                     v_cache, kv, block_table, dtype, path, accept_len, next_bonus, src_slot, dst_slot, stream);
+}
+
 size_t ddtree_accept_workspace_bytes(int n_req, int B, int V) {
   (void)V;
   if (n_req < 1 || B < 0) return 0;
@@ -505,7 +584,8 @@ int ddtree_accept(const void* target_logits, int dtype, int V, long long row_str
 static size_t round_parts(const ddtree_round_args* a, size_t* off_attn, size_t* off_acc) {
   const size_t t = align256(topk_ws(a->n_req * a->L, a->V, a->K, a->dtype));
   const size_t at = align256(attn_ws(&a->kv, a->B, a->dtype));
-  const size_t ac = align256(accept_ws(a->n_req, a->B));
+  const size_t ac = a->target_hidden ? align256(lm_ws_bytes(a->n_req * (a->B + 1)) + (size_t)a->n_req * (a->B + 1) * 4)
+                                     : align256(accept_ws(a->n_req, a->B));
   if (off_attn) *off_attn = t;
   if (off_acc) *off_acc = t + at;
   return t + at + ac;
@@ -522,6 +602,7 @@ int ddtree_round_launch_count(const ddtree_round_args* a) {
   n += 1;                                                                // attention
   if (use_tc_attn(a->dtype, &a->kv) && attn_tc_ws_bytes(geom_of(&a->kv, a->B), num_sms()) > 0) n += 1;   // combine
   if (a->tree_k_in != nullptr) n += 1;                                   // tree K/V write
+  if (a->target_hidden != nullptr) return n + 2;                         // LM-head argmax, walk
   n += 1;                                                                // argmax (+ walk)
   if (a->kv.layers > WALK_FUSE_MAX_LAYERS) n += 1;                       // walk and compaction
   return n;
@@ -550,6 +631,21 @@ int ddtree_round(const ddtree_round_args* a, cudaStream_t stream) {
   st = attn_launch(a->q, a->k_cache, a->v_cache, a->dtype, &a->kv, a->block_table, a->prefix_len, a->anc,
                    a->n_nodes, a->B, a->attn_out, a->attn_lse, ws + off_attn, off_acc - off_attn, stream);
   if (st) return st;
+  if (a->target_hidden != nullptr) {   // the target's argmax from its LM head, logits never written
+    if (a->dtype != DDTREE_BF16 || (a->sampling && a->sampling->temperature > 0.0)) return DDTREE_ERR_UNSUPPORTED;
+    const int rows = a->n_req * (a->B + 1);
+    if ((st = lmhead_check(a->target_hidden, a->lm_head, rows, a->V, a->d_model, a->target_argmax ? a->target_argmax
+                                                                                                   : (int32_t*)ws)))
+      return st;
+    int32_t* tok = a->target_argmax ? a->target_argmax
+                                    : (int32_t*)(ws + off_acc + align256(lm_ws_bytes(rows)));
+    if ((st = lmhead_launch(a->target_hidden, a->lm_head, rows, a->V, a->d_model, tok, nullptr, ws + off_acc,
+                            num_sms(), stream, g_attn_wait_ns)))
+      return st;
+    return walk_launch(tok, a->node_token, a->parent, a->n_nodes, a->n_req, a->L, a->B, a->prefix_len,
+                       a->new_prefix_len, a->k_cache, a->v_cache, &a->kv, a->block_table, a->dtype, a->path,
+                       a->accept_len, a->next_bonus, a->src_slot, a->dst_slot, stream);
+  }
   return accept_launch(a->target_logits, a->dtype, a->V, a->target_stride, a->node_token, a->parent, a->n_nodes,
                        a->n_req, a->L, a->B, a->prefix_len, a->new_prefix_len, a->k_cache, a->v_cache, &a->kv,
                        a->block_table, a->target_argmax, a->path, a->accept_len, a->next_bonus, a->src_slot,

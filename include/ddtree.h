@@ -315,6 +315,39 @@ int ddtree_accept_ex(const void* target_logits, int dtype, int V, long long row_
                      const ddtree_sampling* sampling,
                      void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/*
+ * The target's LM head with its argmax fused into the product ("DDTree Deep
+ * Dive" §6: the verifier needs only the target's token at each node), so
+ * the [rows][V] logits are never written:
+ *   out_argmax[r] = lowest v maximising sum_k hidden[r][k] * weight[v][k]
+ * with bf16 operands and fp32 accumulation on the tensor cores (the order of
+ * that accumulation is the hardware's: two logits within its rounding of
+ * each other may resolve either way).
+ * hidden     device bf16 [rows][d] (e.g. the tree nodes' final hidden states,
+ *            rows = n_req * (B+1)); weight device bf16 [V][d]; d % 64 == 0.
+ * out_argmax device int32 [rows]; out_max device float [rows] (may be NULL):
+ *            the maximum logit.
+ * ws         device scratch of ddtree_lmhead_workspace_bytes(rows) bytes,
+ *            zero-filled before first use; every call leaves it at zero.
+ */
+size_t ddtree_lmhead_workspace_bytes(int rows);
+int ddtree_lmhead_argmax(const void* hidden, const void* weight, int rows, int V, int d,
+                         int32_t* out_argmax, float* out_max, void* ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/*
+ * The verifier walk and KV compaction of ddtree_accept from given per-node
+ * target tokens (target_token device int32 [n_req][B+1]: e.g. the output of
+ * ddtree_lmhead_argmax, or drawn tokens).  Outputs, compaction and dtype
+ * (of the caches) as for ddtree_accept.
+ */
+int ddtree_walk(const int32_t* target_token, const int32_t* node_token, const int32_t* parent,
+                const int32_t* n_nodes, int n_req, int L, int B,
+                const int32_t* prefix_len, int32_t* new_prefix_len,
+                void* k_cache, void* v_cache, const ddtree_kv_desc* kv, const int32_t* block_table,
+                int dtype, int32_t* path, int32_t* accept_len, int32_t* next_bonus,
+                int32_t* src_slot, int32_t* dst_slot, cudaStream_t stream);
+
 /* ---------------------------------------------------------------------- */
 /* The whole round (Deep Dive §3 stage pipeline: draft -> tree_build ->   */
 /* tree_compile -> verify -> commit; the draft and the target forward are */
@@ -362,6 +395,13 @@ typedef struct {
   const void* tree_k_in;
   const void* tree_v_in;
   double rope_theta;
+  /* optional (target_hidden NULL: none): the target's final hidden states of
+   * the tree nodes, bf16 [n_req*(B+1)][d_model], and its LM head, bf16
+   * [V][d_model]; the accept stage then takes each node's token from
+   * ddtree_lmhead_argmax instead of target_logits (greedy only). */
+  const void* target_hidden;
+  const void* lm_head;
+  int d_model;
 } ddtree_round_args;
 
 /* Bytes of a->ws the round needs (0 for an invalid geometry).  The

@@ -506,6 +506,15 @@ def write_tree_kv(k_cache: np.ndarray, v_cache: np.ndarray, k_in: np.ndarray, v_
                 v_cache[l, blk, slots % PAGE] = vr
 
 
+def lm_head_argmax(hidden: np.ndarray, weight: np.ndarray):
+    """The target's token at each node from its LM head (Deep Dive §6, the
+    verifier's argmax): logits = hidden . weight^T in float64, then the
+    lowest index among the maxima of each row (reading R7).  Returns (argmax
+    int32 [rows], max float64 [rows])."""
+    logits = np.asarray(hidden, dtype=np.float64) @ np.asarray(weight, dtype=np.float64).T
+    return argmax_rows(logits), logits.max(axis=-1)
+
+
 # --------------------------------------------------------------------------
 # Temperature > 0: one draw of the target's token per tree node
 # --------------------------------------------------------------------------

@@ -722,3 +722,29 @@ def test_write_tree_kv_places_rotated_rows():
             assert np.allclose(kc[:, r, P[r] + i], oracle.rope(k_in[:, r, i], [P[r] + depth[r, i]] * L_, 1e4))
             assert np.array_equal(vc[:, r, P[r] + i], v_in[:, r, i])
     assert np.all(kc[:, 0, :3] == 0) and np.all(kc[:, 0, 7:] == 0)      # nothing outside the tree slots
+
+
+# ---------------------------------------------------------------- LM-head argmax
+
+def _hadamard(n):
+    h = np.array([[1.0]])
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def test_lm_head_argmax_orthogonal_rows():
+    """Orthogonal (Hadamard) weight rows: hidden = a * row v gives logit a*d
+    at v and 0 elsewhere, so the argmax is v (a > 0), and a row scaled by 2
+    beats its own copy (lowest index only decides exact ties)."""
+    d = 64
+    W = _hadamard(d)
+    hidden = np.stack([0.5 * W[7], 3.0 * W[0], 1.0 * W[63]])
+    am, mx = oracle.lm_head_argmax(hidden, W)
+    assert am.tolist() == [7, 0, 63]
+    assert np.allclose(mx, [0.5 * d, 3.0 * d, 1.0 * d])
+    W2 = np.concatenate([W, 2 * W[5:6], W[5:6]])          # rows 64 (2x row 5) and 65 (= row 5)
+    am2, _ = oracle.lm_head_argmax(W[5:6], W2)
+    assert am2.tolist() == [64]
+    am3, _ = oracle.lm_head_argmax(W[9:10], np.concatenate([W, W[9:10]]))
+    assert am3.tolist() == [9]                            # exact tie with row 64: the lower index

@@ -61,6 +61,8 @@ def parse(argv=None):
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG)
     ap.add_argument("--budget", type=int, default=None, help="config 5: B")
     ap.add_argument("--sigma", type=float, default=None, help="config 5: drafter logit std-dev")
+    ap.add_argument("--layers", type=int, default=None, help="override the workload's attention layers "
+                    "(profiling runs on a smaller case)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true", help="launch rounds eagerly instead of CUDA graphs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -229,6 +231,8 @@ def workload_from_args(a):
     over = {}
     if a.config == 5:
         over = {"B": a.budget or 64, "sigma": a.sigma or 4.0}
+    if a.layers:
+        over["layers"] = a.layers
     return workload_of(a.config, over)
 
 

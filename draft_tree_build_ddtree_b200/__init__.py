@@ -71,7 +71,8 @@ class RoundArgs(ctypes.Structure):
                 ("ws", _vp), ("ws_bytes", _sz),
                 ("gain_floor", _vp), ("sampling", ctypes.POINTER(Sampling)),
                 ("tree_q_in", _vp), ("tree_k_in", _vp), ("tree_v_in", _vp), ("rope_theta", ctypes.c_double),
-                ("target_hidden", _vp), ("lm_head", _vp), ("d_model", _i)]
+                ("target_hidden", _vp), ("lm_head", _vp), ("d_model", _i),
+                ("stage_events", ctypes.POINTER(_vp))]
 
 
 _SIGS = {
@@ -499,6 +500,24 @@ def ddtree_round(rb: RoundBuffers, args: Optional[RoundArgs] = None):
     a = rb.args() if args is None else args
     _check(lib().ddtree_round(ctypes.byref(a), _stream()), "ddtree_round")
     return rb
+
+
+STAGES = ("topk", "build", "tree_kv_write", "attn", "accept")
+
+
+def ddtree_round_timed(rb: RoundBuffers) -> dict:
+    """One round with stage events: {stage: ms} from the events the round
+    records at its stage boundaries (synchronises the current stream)."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
+    for e in evs:
+        e.record()                          # creates the event
+    arr = (ctypes.c_void_p * len(evs))(*[e.cuda_event for e in evs])
+    a = rb.args()
+    a.stage_events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+    _check(lib().ddtree_round(ctypes.byref(a), _stream()), "ddtree_round")
+    evs[-1].synchronize()
+    a.stage_events = None
+    return {name: evs[i].elapsed_time(evs[i + 1]) for i, name in enumerate(STAGES)}
 
 
 def ddtree_round_launch_count(rb: RoundBuffers, args: Optional[RoundArgs] = None) -> int:

@@ -8,6 +8,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "ddtree.h"
 #include "common.cuh"
 #include "topk.cuh"
@@ -608,29 +610,54 @@ int ddtree_round_launch_count(const ddtree_round_args* a) {
   return n;
 }
 
-int ddtree_round(const ddtree_round_args* a, cudaStream_t stream) {
-  if (!a) return DDTREE_ERR_INVALID_ARG;
-  if (kv_check(&a->kv)) return DDTREE_ERR_INVALID_ARG;
-  if (a->kv.n_req != a->n_req) return DDTREE_ERR_INVALID_ARG;
-  size_t off_attn = 0, off_acc = 0;
-  const size_t need = round_parts(a, &off_attn, &off_acc);
-  if (!a->ws || a->ws_bytes < need) return DDTREE_ERR_INVALID_ARG;
-  char* ws = (char*)a->ws;
-  int st = topk_launch(a->drafter_logits, a->dtype, a->n_req * a->L, a->V, a->drafter_stride, a->K, a->ids, a->lp,
-                       a->lse, ws, off_attn, stream);
+// Stage boundaries of a round: an NVTX range per stage on the host timeline
+// and, when the caller passes events, one event recorded on the stream at
+// each boundary (before top-K, build, tree K/V write, attention, accept, and
+// after accept).
+struct StageMarks {
+  cudaEvent_t* ev;
+  cudaStream_t s;
+  int i = 0;
+  bool open = false;
+  int next(const char* name) {
+    if (open) nvtxRangePop();
+    open = name != nullptr;
+    if (open) nvtxRangePushA(name);
+    if (ev != nullptr) {
+      cudaError_t e = cudaEventRecord(ev[i], s);
+      if (e != cudaSuccess) return cuda_fail(e, "ddtree_round: stage event");
+    }
+    ++i;
+    return DDTREE_OK;
+  }
+  ~StageMarks() {
+    if (open) nvtxRangePop();
+  }
+};
+
+static int round_stages(const ddtree_round_args* a, cudaStream_t stream, char* ws, size_t off_attn, size_t off_acc,
+                        size_t need, StageMarks& mk) {
+  int st;
+  if ((st = mk.next("ddtree_topk"))) return st;
+  st = topk_launch(a->drafter_logits, a->dtype, a->n_req * a->L, a->V, a->drafter_stride, a->K, a->ids, a->lp,
+                   a->lse, ws, off_attn, stream);
   if (st) return st;
+  if ((st = mk.next("ddtree_build"))) return st;
   st = build_launch(a->ids, a->lp, a->root_token, a->n_req, a->L, a->K, a->B, a->node_token, a->parent, a->depth,
                     a->node_rank, a->score, a->anc, a->n_nodes, stream, 0, a->gain_floor, nullptr);
   if (st) return st;
+  if ((st = mk.next("ddtree_tree_kv_write"))) return st;
   if (a->tree_k_in != nullptr) {   // the tree's positions are known now: rotate and write its K/V
     st = rope_launch(a->tree_q_in, a->tree_q_in ? (void*)a->q : nullptr, a->tree_k_in, a->tree_v_in, a->dtype,
                      a->depth, a->n_nodes, a->prefix_len, &a->kv, a->block_table, a->B, a->rope_theta, a->k_cache,
                      a->v_cache, stream);
     if (st) return st;
   }
+  if ((st = mk.next("ddtree_tree_attn"))) return st;
   st = attn_launch(a->q, a->k_cache, a->v_cache, a->dtype, &a->kv, a->block_table, a->prefix_len, a->anc,
                    a->n_nodes, a->B, a->attn_out, a->attn_lse, ws + off_attn, off_acc - off_attn, stream);
   if (st) return st;
+  if ((st = mk.next("ddtree_accept"))) return st;
   if (a->target_hidden != nullptr) {   // the target's argmax from its LM head, logits never written
     if (a->dtype != DDTREE_BF16 || (a->sampling && a->sampling->temperature > 0.0)) return DDTREE_ERR_UNSUPPORTED;
     const int rows = a->n_req * (a->B + 1);
@@ -642,14 +669,28 @@ int ddtree_round(const ddtree_round_args* a, cudaStream_t stream) {
     if ((st = lmhead_launch(a->target_hidden, a->lm_head, rows, a->V, a->d_model, tok, nullptr, ws + off_acc,
                             num_sms(), stream, g_attn_wait_ns)))
       return st;
-    return walk_launch(tok, a->node_token, a->parent, a->n_nodes, a->n_req, a->L, a->B, a->prefix_len,
-                       a->new_prefix_len, a->k_cache, a->v_cache, &a->kv, a->block_table, a->dtype, a->path,
-                       a->accept_len, a->next_bonus, a->src_slot, a->dst_slot, stream);
-  }
-  return accept_launch(a->target_logits, a->dtype, a->V, a->target_stride, a->node_token, a->parent, a->n_nodes,
+    st = walk_launch(tok, a->node_token, a->parent, a->n_nodes, a->n_req, a->L, a->B, a->prefix_len,
+                     a->new_prefix_len, a->k_cache, a->v_cache, &a->kv, a->block_table, a->dtype, a->path,
+                     a->accept_len, a->next_bonus, a->src_slot, a->dst_slot, stream);
+  } else {
+    st = accept_launch(a->target_logits, a->dtype, a->V, a->target_stride, a->node_token, a->parent, a->n_nodes,
                        a->n_req, a->L, a->B, a->prefix_len, a->new_prefix_len, a->k_cache, a->v_cache, &a->kv,
                        a->block_table, a->target_argmax, a->path, a->accept_len, a->next_bonus, a->src_slot,
                        a->dst_slot, ws + off_acc, need - off_acc, stream, a->sampling);
+  }
+  if (st) return st;
+  return mk.next(nullptr);
+}
+
+int ddtree_round(const ddtree_round_args* a, cudaStream_t stream) {
+  if (!a) return DDTREE_ERR_INVALID_ARG;
+  if (kv_check(&a->kv)) return DDTREE_ERR_INVALID_ARG;
+  if (a->kv.n_req != a->n_req) return DDTREE_ERR_INVALID_ARG;
+  size_t off_attn = 0, off_acc = 0;
+  const size_t need = round_parts(a, &off_attn, &off_acc);
+  if (!a->ws || a->ws_bytes < need) return DDTREE_ERR_INVALID_ARG;
+  StageMarks mk{a->stage_events, stream};
+  return round_stages(a, stream, (char*)a->ws, off_attn, off_acc, need, mk);
 }
 
 int ddtree_debug_attn_timeout(unsigned long long wait_ns, int withhold_tile) {

@@ -402,6 +402,11 @@ typedef struct {
   const void* target_hidden;
   const void* lm_head;
   int d_model;
+  /* optional (NULL: none): 6 events the round records on `stream` at its
+   * stage boundaries (before top-K, build, tree K/V write, attention and
+   * accept, and after accept), for per-stage cudaEventElapsedTime; the round
+   * also marks each stage with an NVTX range on the host. */
+  cudaEvent_t* stage_events;
 } ddtree_round_args;
 
 /* Bytes of a->ws the round needs (0 for an invalid geometry).  The

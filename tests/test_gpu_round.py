@@ -190,3 +190,16 @@ def test_round_repeats_are_identical():
     torch.cuda.synchronize()
     for a, b in zip(first, (rb.ids, rb.lp, rb.tree.anc, rb.attn_out, rb.acc.path)):
         assert torch.equal(a, b)
+
+
+def test_round_stage_events():
+    """The round's stage events bracket its stages: five non-negative times
+    whose sum is the round, with the attention the largest at 48 layers."""
+    w = datagen.workload(3, layers=4)
+    rb, h = make_round(w)
+    dd.ddtree_round(rb)
+    t = dd.ddtree_round_timed(rb)
+    assert set(t) == set(dd.STAGES)
+    assert all(v >= 0.0 for v in t.values())
+    assert t["tree_kv_write"] < 0.05           # no tree K/V given: an empty stage
+    assert t["attn"] == max(t.values())

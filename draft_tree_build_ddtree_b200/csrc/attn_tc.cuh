@@ -628,11 +628,11 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 constexpr int TC_MAX_SPLITS = 16;
 constexpr int TC_LPT_MAX_REQ = 128;   // longest-first request order up to this batch (each CTA ranks them all)
 
-template <int S>   // capacity for the number of splits (>= p.splits)
+template <int S, int D = TC_D>   // capacity for the number of splits (>= p.splits); head dim
 __global__ void __launch_bounds__(128)
 tree_attn_combine_kernel(const TcParams p) {
   const AttnGeom& g = p.g;
-  const int groups = TC_D / 8;
+  const int groups = D / 8;
   int u = blockIdx.x / groups;
   const int rg = blockIdx.x - u * groups;
   const int unit = u;
@@ -660,7 +660,7 @@ tree_attn_combine_kernel(const TcParams p) {
       const size_t slot = (size_t)unit * p.splits + s;
       ml[s] = p.ws_ml[slot * TC_BM + row];
       // partial O layout: [slot][D/4][128 rows] float4, so consecutive rows are consecutive
-      const float4* wo = reinterpret_cast<const float4*>(p.ws_o) + (slot * (TC_D / 4) + d0 / 4) * TC_BM + row;
+      const float4* wo = reinterpret_cast<const float4*>(p.ws_o) + (slot * (D / 4) + d0 / 4) * TC_BM + row;
       pa[s] = wo[0];
       pb[s] = wo[TC_BM];
     }
@@ -683,7 +683,7 @@ tree_attn_combine_kernel(const TcParams p) {
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  __nv_bfloat16* orow = p.out + ((((size_t)layer * g.n_req + r) * g.n + node) * g.Hq + hq) * TC_D + d0;
+  __nv_bfloat16* orow = p.out + ((((size_t)layer * g.n_req + r) * g.n + node) * g.Hq + hq) * D + d0;
   uint4 pk;
   pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
@@ -758,11 +758,11 @@ inline EncodeTiledFn encode_fn() {
 
 // 4-D bf16 map over (D, dim1, dim2, dim3) with a (64, b1, b2, 1) box and 128B swizzle.
 inline bool make_map_4d(CUtensorMap* m, const void* base, uint64_t d1, uint64_t d2, uint64_t d3, uint32_t b1,
-                        uint32_t b2) {
+                        uint32_t b2, uint64_t D = TC_D) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[4] = {TC_D, d1, d2, d3};
-  cuuint64_t strides[3] = {TC_D * 2, TC_D * 2 * d1, TC_D * 2 * d1 * d2};
+  cuuint64_t dims[4] = {D, d1, d2, d3};
+  cuuint64_t strides[3] = {D * 2, D * 2 * d1, D * 2 * d1 * d2};
   cuuint32_t box[4] = {64, b1, b2, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult res = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,

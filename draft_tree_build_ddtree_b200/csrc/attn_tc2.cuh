@@ -46,14 +46,18 @@ namespace ddt {
 constexpr int T2_THREADS = 320;
 constexpr int T2_BN = 128;                          // keys per tile
 constexpr int T2_KATOM = T2_BN * 64 * 2;            // [128 keys][64 dims] bf16: 16 KB
-constexpr int T2_KTILE = 2 * T2_KATOM;              // [128 keys][128 dims]: 32 KB
 constexpr int T2_STAGES = 2;
 constexpr uint32_t T2_TMEM_COLS = 512;
 
+// Head dim D in {64, 128}: a Q tile is D/64 swizzle atoms of [128 rows][64
+// dims] (16 KB each), a K or V tile D/64 atoms of [128 keys][64 dims].
+template <int D>
 struct T2Smem {
-  unsigned char q[2][TC_TILE];
-  unsigned char k[T2_STAGES][T2_KTILE];
-  unsigned char v[T2_STAGES][T2_KTILE];
+  static constexpr int QTILE = (D / 64) * TC_ATOM;
+  static constexpr int KTILE = (D / 64) * T2_KATOM;
+  unsigned char q[2][QTILE];
+  unsigned char k[T2_STAGES][KTILE];
+  unsigned char v[T2_STAGES][KTILE];
   uint64_t bar_q, bar_kf[T2_STAGES], bar_ke[T2_STAGES], bar_vf[T2_STAGES], bar_ve[T2_STAGES];
   uint64_t bar_sfull[2], bar_pready[2], bar_odone;
   uint32_t tmem_base;
@@ -61,7 +65,8 @@ struct T2Smem {
   int lpt_r;
 };
 
-constexpr size_t t2_smem_bytes() { return sizeof(T2Smem); }
+template <int D>
+constexpr size_t t2_smem_bytes() { return sizeof(T2Smem<D>); }
 
 // D[tmem] (+)= A[tmem] * B[smem]: kind::f16 with the A operand in tensor memory.
 __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
@@ -116,11 +121,14 @@ struct T2Params {
   int stop_tile;
 };
 
+template <int D>
 __global__ void __launch_bounds__(T2_THREADS, 1)
 tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const T2Params p) {
   extern __shared__ __align__(1024) unsigned char smem_dyn[];
-  T2Smem& sm = *reinterpret_cast<T2Smem*>(smem_dyn);
+  typedef T2Smem<D> Smem;
+  Smem& sm = *reinterpret_cast<Smem*>(smem_dyn);
+  constexpr int HA = D / 64;                          // 64-dim atoms per row
   if ((smem_u32(smem_dyn) & 1023u) != 0u) {       // the 128B-swizzled tiles need 1024-byte alignment
     if (threadIdx.x == 0) flag_status(DDTREE_STATUS_SETUP);
     return;
@@ -215,11 +223,11 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // =========================== TMA producer ===========================
     if (lane == 0 && nt > 0) {
       const int qb = layer * g.n_req + r;
-      mbar_expect_tx(&sm.bar_q, (uint32_t)(ntl * TC_TILE));
+      mbar_expect_tx(&sm.bar_q, (uint32_t)(ntl * Smem::QTILE));
       for (int t = 0; t < ntl; ++t) {
         const int nd = node_base + t * nodes_per_tile;
-        tma_load_4d(smem_u32(sm.q[t]), &tm_q, &sm.bar_q, 0, kvh * p.G, nd, qb);
-        tma_load_4d(smem_u32(sm.q[t] + TC_ATOM), &tm_q, &sm.bar_q, 64, kvh * p.G, nd, qb);
+        for (int h = 0; h < HA; ++h)
+          tma_load_4d(smem_u32(sm.q[t] + h * TC_ATOM), &tm_q, &sm.bar_q, 64 * h, kvh * p.G, nd, qb);
       }
       int issued = 0;
       for (int jj = 0; jj < nt; ++jj) {
@@ -236,8 +244,8 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           b1 = (pg + 1 < maxpg) ? p.block_table[(size_t)r * g.max_blocks + pg + 1] : b0;
         }
         auto load_tile = [&](const CUtensorMap* map, unsigned char* tile, uint64_t* bar) {
-          mbar_expect_tx(bar, T2_KTILE);
-          for (int h = 0; h < 2; ++h) {
+          mbar_expect_tx(bar, Smem::KTILE);
+          for (int h = 0; h < HA; ++h) {
             const uint32_t dst = smem_u32(tile + h * T2_KATOM);
             if (!g.paged) {
               tma_load_4d(dst, map, bar, 64 * h, kvh, k0, layer * g.n_req + r);
@@ -266,13 +274,13 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // =========================== MMA issuer ===========================
     if (lane == 0 && nt > 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(TC_BM, T2_BN, false, false);
-      constexpr uint32_t IDESC_PV = idesc_bf16_f32(TC_BM, TC_D, false, true);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(TC_BM, D, false, true);
       bool ok = mbar_wait(&sm.bar_q, 0, abort, wlim);
       bool any_commit = false;
       auto issue_s = [&](int t, int st) {      // S_t = Q_t K^T over the 128 head dims
         const uint32_t q_addr = smem_u32(sm.q[t]), k_addr = smem_u32(sm.k[st]);
 #pragma unroll
-        for (int kk = 0; kk < TC_D / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * TC_ATOM + (kk & 3) * 32;
           const uint32_t koff = (kk >> 2) * T2_KATOM + (kk & 3) * 32;
           umma_f16(tmem + 128 * t, smem_desc_sw128(q_addr + off, 16, 1024),
@@ -388,7 +396,7 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         l *= corr;
         if (jj > 0) {        // PV_t(jj-1) has completed (it precedes S_t(jj)); O_t is ours to rescale
 #pragma unroll 1
-          for (int c = 0; c < TC_D / 16; ++c) {     // 16 columns at a time: S stays in registers
+          for (int c = 0; c < D / 16; ++c) {        // 16 columns at a time: S stays in registers
             uint32_t o[16];
             tmem_ld16(tm_o + c * 16, o);
             tmem_wait_ld();
@@ -430,9 +438,9 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (p.splits == 1) {
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
         __nv_bfloat16* orow =
-            p.out + ((((size_t)layer * g.n_req + r) * g.n + min(node, g.n - 1)) * g.Hq + hq) * TC_D;
+            p.out + ((((size_t)layer * g.n_req + r) * g.n + min(node, g.n - 1)) * g.Hq + hq) * D;
 #pragma unroll 1
-        for (int c = 0; c < TC_D / 32; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           float o[32];
           tmem_ld32(tm_o + c * 32, o);
           tmem_wait_ld();
@@ -453,9 +461,9 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
               (m_used + log2f(l)) * 0.6931471805599453f;
       } else {
         const size_t slot = munit * p.splits + split;
-        float4* wo = reinterpret_cast<float4*>(p.ws_o) + slot * (TC_D / 4) * TC_BM + row;
+        float4* wo = reinterpret_cast<float4*>(p.ws_o) + slot * (D / 4) * TC_BM + row;
 #pragma unroll 1
-        for (int c = 0; c < TC_D / 32; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           float o[32];
           tmem_ld32(tm_o + c * 32, o);
           tmem_wait_ld();
@@ -493,7 +501,7 @@ struct AttnDispatch {
   int splits, mtiles, mpairs, units2;   // two-M-tile plan
 };
 
-inline AttnDispatch attn_dispatch(const AttnGeom& g, int num_sms) {
+inline AttnDispatch attn_dispatch(const AttnGeom& g, int num_sms) {   // D = 64: always the two-M-tile kernel
   AttnDispatch d;
   d.v1 = tc_plan(g, num_sms);
   const int G = g.Hq / g.Hkv;
@@ -510,8 +518,9 @@ inline AttnDispatch attn_dispatch(const AttnGeom& g, int num_sms) {
     if (splits < 1) splits = 1;
   }
   d.splits = splits;
-  // long enough per CTA, and enough CTAs to keep at least half the SMs busy
-  d.v2 = tiles / splits >= T2_MIN_TILES && (long long)d.units2 * splits * 2 >= num_sms;
+  // long enough per CTA, and enough CTAs to keep at least half the SMs busy;
+  // the single-M-tile kernel is built for D = 128 only
+  d.v2 = g.D == 64 || (tiles / splits >= T2_MIN_TILES && (long long)d.units2 * splits * 2 >= num_sms);
   return d;
 }
 
@@ -520,7 +529,7 @@ inline size_t attn_tc_ws_bytes(const AttnGeom& g, int num_sms) {
   if (!d.v2) return tc_attn_ws_bytes(g, num_sms);
   if (d.splits == 1) return 0;
   const size_t slots = (size_t)g.layers * g.n_req * g.Hkv * d.mtiles * d.splits;
-  return align256(slots * TC_BM * TC_D * 4) + align256(slots * TC_BM * 8);
+  return align256(slots * TC_BM * g.D * 4) + align256(slots * TC_BM * 8);
 }
 
 inline int attn_tc_launch(const void* q, const void* kc, const void* vc, const int32_t* block_table,
@@ -553,31 +562,38 @@ inline int attn_tc_launch(const void* q, const void* kc, const void* vc, const i
   const size_t slots = (size_t)g.layers * g.n_req * g.Hkv * d.mtiles * d.splits;
   if (d.splits > 1) {
     p.ws_o = (float*)ws;
-    p.ws_ml = (float2*)((char*)ws + align256(slots * TC_BM * TC_D * 4));
+    p.ws_ml = (float2*)((char*)ws + align256(slots * TC_BM * g.D * 4));
   }
   CUtensorMap mq, mk, mv;
+  const uint64_t D = (uint64_t)g.D;
   if (!make_map_4d(&mq, q, (uint64_t)g.Hq, (uint64_t)g.n, (uint64_t)g.layers * g.n_req, (uint32_t)p.G,
-                   (uint32_t)(TC_BM / p.G)))
+                   (uint32_t)(TC_BM / p.G), D))
     return cuda_fail_msg("tree attention: tensor map of q");
   if (!g.paged) {
-    if (!make_map_4d(&mk, kc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, T2_BN) ||
-        !make_map_4d(&mv, vc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, T2_BN))
+    if (!make_map_4d(&mk, kc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, T2_BN, D) ||
+        !make_map_4d(&mv, vc, g.Hkv, g.s_max, (uint64_t)g.layers * g.n_req, 1, T2_BN, D))
       return cuda_fail_msg("tree attention: tensor map of the cache");
   } else {
-    if (!make_map_4d(&mk, kc, g.Hkv, DDTREE_PAGE, (uint64_t)g.layers * g.num_blocks, 1, DDTREE_PAGE) ||
-        !make_map_4d(&mv, vc, g.Hkv, DDTREE_PAGE, (uint64_t)g.layers * g.num_blocks, 1, DDTREE_PAGE))
+    if (!make_map_4d(&mk, kc, g.Hkv, DDTREE_PAGE, (uint64_t)g.layers * g.num_blocks, 1, DDTREE_PAGE, D) ||
+        !make_map_4d(&mv, vc, g.Hkv, DDTREE_PAGE, (uint64_t)g.layers * g.num_blocks, 1, DDTREE_PAGE, D))
       return cuda_fail_msg("tree attention: tensor map of the paged cache");
   }
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tree_attn_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)t2_smem_bytes());
+    cudaError_t e = cudaFuncSetAttribute(tree_attn_tc2_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)t2_smem_bytes<128>());
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tree_attn_tc2_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)t2_smem_bytes<64>());
     if (e != cudaSuccess) return cuda_fail(e, "tree attention (two M-tiles): shared-memory attribute");
     attr_set = true;
   }
   const long long grid = (long long)d.units2 * d.splits;
   if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
-  tree_attn_tc2_kernel<<<(unsigned)grid, T2_THREADS, t2_smem_bytes(), stream>>>(mq, mk, mv, p);
+  if (g.D == 64)
+    tree_attn_tc2_kernel<64><<<(unsigned)grid, T2_THREADS, t2_smem_bytes<64>(), stream>>>(mq, mk, mv, p);
+  else
+    tree_attn_tc2_kernel<128><<<(unsigned)grid, T2_THREADS, t2_smem_bytes<128>(), stream>>>(mq, mk, mv, p);
   {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "tree attention (two M-tiles): launch");
@@ -601,10 +617,14 @@ inline int attn_tc_launch(const void* q, const void* kc, const void* vc, const i
     c.lpt = 0;
     c.wait_ns = p.wait_ns;
     c.stop_tile = -1;
-    if (d.splits <= 8)
-      tree_attn_combine_kernel<8><<<c.units * (TC_D / 8), TC_BM, 0, stream>>>(c);
-    else
-      tree_attn_combine_kernel<TC_MAX_SPLITS><<<c.units * (TC_D / 8), TC_BM, 0, stream>>>(c);
+    const unsigned cgrid = (unsigned)(c.units * (g.D / 8));
+    if (g.D == 64) {
+      if (d.splits <= 8) tree_attn_combine_kernel<8, 64><<<cgrid, TC_BM, 0, stream>>>(c);
+      else tree_attn_combine_kernel<TC_MAX_SPLITS, 64><<<cgrid, TC_BM, 0, stream>>>(c);
+    } else {
+      if (d.splits <= 8) tree_attn_combine_kernel<8><<<cgrid, TC_BM, 0, stream>>>(c);
+      else tree_attn_combine_kernel<TC_MAX_SPLITS><<<cgrid, TC_BM, 0, stream>>>(c);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "tree attention: combine launch");
   }

@@ -223,7 +223,7 @@ unsigned long long g_attn_wait_ns = 0;   // 0: the default limit
 int g_attn_stop_tile = -1;
 
 bool use_tc_attn(int dtype, const ddtree_kv_desc* kv) {
-  return dtype == DDTREE_BF16 && kv->D == 128 && tc_attn_supported(kv->Hq / kv->Hkv);
+  return dtype == DDTREE_BF16 && (kv->D == 128 || kv->D == 64) && tc_attn_supported(kv->Hq / kv->Hkv);
 }
 
 size_t attn_ws(const ddtree_kv_desc* kv, int B, int dtype) {

@@ -232,8 +232,8 @@ size_t ddtree_attn_workspace_bytes(const ddtree_kv_desc* kv, int B);
  *            (16-byte aligned; NULL when that is 0).  It must be zero-filled
  *            before its first use; every call leaves its counters at zero.
  *            Calls that share a workspace must not overlap.
- * bf16: tcgen05 tensor-core path for D = 128 (fp32 accumulation, P rounded
- * to bf16 for the PV product); fp32 and D = 64: CUDA-core fp32 path.
+ * bf16 (D = 64 or 128): tcgen05 tensor-core kernels (fp32 accumulation, P
+ * rounded to bf16 for the PV product); fp32: the CUDA-core fp32 kernel.
  */
 int ddtree_tree_attn(const void* q, const void* k_cache, const void* v_cache, int dtype,
                      const ddtree_kv_desc* kv, const int32_t* block_table,

@@ -290,3 +290,17 @@ def test_attention_wait_timeout_reports_and_recovers():
     assert lib.ddtree_debug_attn_timeout(0, -2) != 0
     out, lse = _gpu_attn(w, st, prefix, cache, q)
     _check_attn(w, st, prefix, cache, q, out, lse)
+
+
+@pytest.mark.parametrize("cfg,over", [(2, dict(D=64)), (4, dict(N=3, D=64)), (3, dict(layers=2, D=64)),
+                                      (5, dict(B=256, K=256, D=64))])
+def test_attention_bf16_d64_tensor_cores(cfg, over):
+    """bf16 with head dim 64 runs on the tensor cores (two-M-tile kernel,
+    split or not, contiguous or paged) and matches the oracle."""
+    w = datagen.workload(cfg, **over)
+    st, prefix, cache, q = _attn_case(w)
+    out, lse = _gpu_attn(w, st, prefix, cache, q)
+    sample = {} if cfg == 2 else dict(nodes=[0, 1, w.B // 2, w.B], heads=[0, 9, w.Hq - 1])
+    if cfg == 4:
+        sample["reqs"] = [0, w.N - 1]
+    _check_attn(w, st, prefix, cache, q, out, lse, **sample)

@@ -143,6 +143,12 @@ def test_launch_plans_from_sizes(lib):
     slots = 4 * 5 * 12
     assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv5), 64) == \
         _align256(slots * 128 * 128 * 4) + _align256(slots * 128 * 8)
+    # bf16 with D = 64 always takes the two-M-tile kernel: b64_p2k's shape
+    # with D = 64 splits its 12 M-tile pairs twice (8 key tiles each at least)
+    kv64 = dd.kv_desc(1, 1, 32, 4, 64, s_max=2176)
+    slots = 4 * 5 * 2
+    assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv64), 64) == \
+        _align256(slots * 128 * 64 * 4) + _align256(slots * 128 * 8)
     kv3 = dd.kv_desc(48, 1, 32, 4, 128, s_max=8512)
     assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv3), 256) == 0
     kv4 = dd.kv_desc(1, 32, 32, 4, 128, paged=True, num_blocks=4096, max_blocks=258)

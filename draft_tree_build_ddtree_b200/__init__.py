@@ -31,8 +31,10 @@ __all__ = [
 ]
 
 BF16, F32 = 0, 1
-STATUS_NONFINITE, STATUS_TIMEOUT, STATUS_CAPACITY, STATUS_SETUP = 1, 2, 4, 8
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libddtree.so")
+STATUS_NONFINITE, STATUS_TIMEOUT, STATUS_CAPACITY, STATUS_SETUP, STATUS_BOUNDS = 1, 2, 4, 8, 16
+# DDTREE_LIBRARY=debug selects the bounds-checked build libddtree_debug.so
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                         "libddtree_debug.so" if os.environ.get("DDTREE_LIBRARY") == "debug" else "libddtree.so")
 _lib = None
 
 _vp = ctypes.c_void_p

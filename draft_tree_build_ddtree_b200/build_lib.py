@@ -14,6 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libddtree.so")
+LIB_DEBUG = os.path.join(PKG, "libddtree_debug.so")   # -DDDTREE_DEBUG: internal bounds checks into the status word
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -35,26 +36,29 @@ def sources():
                   [os.path.join(INCLUDE, "ddtree.h")])
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I" + INCLUDE, os.path.join(CSRC, "ddtree.cu"), "-o", LIB + ".tmp"]
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Build libddtree.so (or, with debug, libddtree_debug.so with -DDDTREE_DEBUG)."""
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not stale(lib):
+        return lib
+    extra = ["-DDDTREE_DEBUG"] if debug else []
+    cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I" + INCLUDE, os.path.join(CSRC, "ddtree.cu"), "-o", lib + ".tmp"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed building libddtree.so")
+        raise RuntimeError(f"nvcc failed building {os.path.basename(lib)}")
     if verbose:
         sys.stderr.write(res.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

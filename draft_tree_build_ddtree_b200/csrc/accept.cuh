@@ -126,6 +126,7 @@ __device__ void walk_request(const WalkArgs& a, int r, int nn, int P, int lk0, i
     int cur = 0, k = 0;
     ws.path[0] = 0;
     while (k < a.L && ws.nxt[cur] >= 0) {
+      if (!DDT_IN_RANGE(ws.nxt[cur], cur + 1, nn)) break;
       cur = ws.nxt[cur];
       ws.path[++k] = cur;
     }
@@ -189,7 +190,7 @@ __device__ void walk_request(const WalkArgs& a, int r, int nn, int P, int lk0, i
         const int e = b0 + t * nth + tid;
         if (e < total) {
           const int j = 1 + e / vec_per_row, c = e % vec_per_row;
-          buf[t] = *((const uint4*)row_ptr(P + ws.path[j]) + c);
+          if (DDT_IN_RANGE(ws.path[j], j, nn)) buf[t] = *((const uint4*)row_ptr(P + ws.path[j]) + c);
         }
       }
       __syncthreads();   // every source of this batch is read before any write
@@ -198,7 +199,7 @@ __device__ void walk_request(const WalkArgs& a, int r, int nn, int P, int lk0, i
         const int e = b0 + t * nth + tid;
         if (e < total) {
           const int j = 1 + e / vec_per_row, c = e % vec_per_row;
-          if (ws.path[j] != j) *((uint4*)row_ptr(P + j) + c) = buf[t];
+          if (ws.path[j] != j && DDT_IN_RANGE(ws.path[j], j, nn)) *((uint4*)row_ptr(P + j) + c) = buf[t];
         }
       }
       __syncthreads();

@@ -39,7 +39,10 @@
 // multicast is used.
 #pragma once
 
+#include <type_traits>
+
 #include "attn_tc.cuh"
+#include "exp2_poly.h"
 
 namespace ddt {
 
@@ -48,6 +51,9 @@ constexpr int T2_BN = 128;                          // keys per tile
 constexpr int T2_KATOM = T2_BN * 64 * 2;            // [128 keys][64 dims] bf16: 16 KB
 constexpr int T2_STAGES = 2;
 constexpr uint32_t T2_TMEM_COLS = 512;
+#ifndef T2_POLY
+#define T2_POLY 0   // exponentials per eight on the FMA pipe (unmasked tiles)
+#endif
 
 // Head dim D in {64, 128}: a Q tile is D/64 swizzle atoms of [128 rows][64
 // dims] (16 KB each), a K or V tile D/64 atoms of [128 keys][64 dims].
@@ -92,6 +98,50 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: two independent lanes, each
+// rounded as the scalar operation would be).
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(unsigned long long v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// max of three (sm_100 three-input max)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x on the FMA pipe, for x <= 2^8 with no -inf (unmasked keys): x is split
+// into the nearest integer j (the 1.5*2^23 shifter, whose low bits then hold
+// j) and f in [-1/2, 1/2]; 2^f is a degree-3 least-squares polynomial
+// (coefficients from gen_exp2_poly.py; relative error 1.4e-4, below bf16's
+// 2^-9 rounding of P) and j is added to the exponent field.  Inputs below
+// -126 are clamped there (2^-126: a P that rounds to nothing against the row).
+__device__ __forceinline__ float ex2_fma(float x) {
+  x = fmaxf(x, -126.0f);
+  const float r = __fadd_rn(x, 12582912.0f);
+  const float f = __fsub_rn(x, __fsub_rn(r, 12582912.0f));
+  float p = fmaf(EX2_POLY_C3, f, EX2_POLY_C2);
+  p = fmaf(p, f, EX2_POLY_C1);
+  p = fmaf(p, f, EX2_POLY_C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(r) << 23));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -378,25 +428,61 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (!((word >> c) & 1u)) s[32 * w + c] = -INFINITY;
         }
       }
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // The running max m_used only moves when a tile's max exceeds it by more
+      // than 2^8 (then every P <= 256), so the exponentials need not wait for
+      // this tile's max: P = 2^(s*sl2 - m_used) is computed and stored while the
+      // tile's max is taken in the same pass; a tile that does exceed it (rare
+      // after the first) rescales O and recomputes its P from the registers.  A
+      // row without a finite max yet takes its max first.
+      auto tile_max = [&]() {
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < T2_BN; c += 4) {
+        for (int c = 0; c < T2_BN; c += 8) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) mx4[e] = fmaxf(mx4[e], s[c + e]);
-      }
-      const float m_tile = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
-      bool rescale = false;
-      float m_new = m_used;
-      if (m_tile > m_used + TC_RESCALE_LOG2 || (m_used == -INFINITY && m_tile > -INFINITY)) {
-        m_new = m_tile;
-        rescale = true;
-      }
-      if (__any_sync(0xffffffffu, rescale)) {
-        const float corr = !rescale ? 1.f : ((m_used == -INFINITY) ? 0.f : ex2_approx(m_used - m_new));
+          for (int e = 0; e < 4; ++e) mx4[e] = max3f(mx4[e], s[c + 2 * e], s[c + 2 * e + 1]);
+        }
+        return max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2;
+      };
+      // P of this tile with the current m_used into S's first 64 columns, two
+      // keys per packed f32x2 instruction for the scaling and the sums; on
+      // tiles without masked keys NPOLY of every eight exponentials run as a
+      // polynomial on the FMA pipe (ex2_fma) beside the ex2 unit.  Returns the
+      // row sum; *tmax receives the tile's max (log2 units).
+      auto exp_pass = [&](auto npoly, float* tmax) {
+        constexpr int NPOLY = decltype(npoly)::value;
+        const float mneg = (m_used == -INFINITY) ? 0.f : -m_used;
+        const unsigned long long sl2x2 = f2_pack(sl2, sl2), m2 = f2_pack(mneg, mneg);
+        unsigned long long acc[2] = {0ull, 0ull};
+        float mx2[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {           // 32 keys -> 16 packed columns per store
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float s0 = s[32 * q4 + 2 * c], s1 = s[32 * q4 + 2 * c + 1];
+            mx2[c & 1] = max3f(mx2[c & 1], s0, s1);
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(s0, s1), sl2x2, m2), x0, x1);
+            const bool p0 = NPOLY >= 1 && (c & 3) == 3, p1 = NPOLY >= 2 && (c & 3) == 3;
+            const float e0 = p0 ? ex2_fma(x0) : ex2_approx(x0);
+            const float e1 = p1 ? ex2_fma(x1) : ex2_approx(x1);
+            acc[c & 1] = f2_add(acc[c & 1], f2_pack(e0, e1));
+            pk[c] = pack_bf16x2(e0, e1);
+          }
+          tmem_st16(tm_s + 16 * q4, pk);
+        }
+        *tmax = fmaxf(mx2[0], mx2[1]) * sl2;
+        float lo, hi;
+        f2_unpack(f2_add(acc[0], acc[1]), lo, hi);
+        return lo + hi;
+      };
+      // O *= corr (per row) and l *= corr; PV_t(jj-1) has completed (it precedes
+      // S_t(jj)), so O_t is ours to rescale
+      auto rescale_o = [&](float corr) {
         l *= corr;
-        if (jj > 0) {        // PV_t(jj-1) has completed (it precedes S_t(jj)); O_t is ours to rescale
+        if (jj > 0) {
 #pragma unroll 1
-          for (int c = 0; c < D / 16; ++c) {        // 16 columns at a time: S stays in registers
+          for (int c = 0; c < D / 16; ++c) {          // 16 columns at a time: S stays in registers
             uint32_t o[16];
             tmem_ld16(tm_o + c * 16, o);
             tmem_wait_ld();
@@ -406,23 +492,24 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           }
           tmem_wait_st();
         }
-        if (rescale) m_used = m_new;
+      };
+      if (__any_sync(0xffffffffu, m_used == -INFINITY)) {   // rows without a max yet: take it first
+        const float m_tile = tile_max();
+        const bool set = m_used == -INFINITY && m_tile > -INFINITY;
+        if (set) m_used = m_tile;                     // O and l are still zero for such rows
       }
-      const float mneg = (m_used == -INFINITY) ? 0.f : -m_used;
-      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {             // 32 keys -> 16 packed columns per store
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float e0 = ex2_approx(fmaf(s[32 * q4 + 2 * c], sl2, mneg));
-          const float e1 = ex2_approx(fmaf(s[32 * q4 + 2 * c + 1], sl2, mneg));
-          ls4[c & 3] += e0 + e1;
-          pk[c] = pack_bf16x2(e0, e1);
-        }
-        tmem_st16(tm_s + 16 * q4, pk);
+      float m_tile;
+      float lt = (k0 + T2_BN <= P) ? exp_pass(std::integral_constant<int, T2_POLY>(), &m_tile)
+                                   : exp_pass(std::integral_constant<int, 0>(), &m_tile);
+      const bool grow = m_tile > m_used + TC_RESCALE_LOG2;
+      if (__any_sync(0xffffffffu, grow)) {
+        tmem_wait_st();                               // the first pass's P stores land before they are redone
+        const float m_new = grow ? m_tile : m_used;
+        rescale_o(grow ? ex2_approx(m_used - m_new) : 1.f);
+        m_used = m_new;
+        lt = exp_pass(std::integral_constant<int, 0>(), &m_tile);
       }
-      l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+      l += lt;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.bar_pready[t]);
@@ -434,7 +521,7 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const size_t munit = (((size_t)layer * g.n_req + r) * g.Hkv + kvh) * p.mtiles + mt;
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
-      const bool live = node < nn;
+      const bool live = node < nn && DDT_IN_RANGE(node, 0, g.n);
       if (p.splits == 1) {
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
         __nv_bfloat16* orow =

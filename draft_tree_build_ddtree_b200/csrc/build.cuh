@@ -778,6 +778,7 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
       for (int k = b0 + wrp; k < b1; k += BUILD_THREADS / 32) {
         const int i = order[k];
         const int pi = sm.nd_parent[i];
+        if (!DDT_IN_RANGE(pi, 0, i)) continue;
         for (int w = lane; w < W; w += 32)
           rows[(size_t)i * W + w] = rows[(size_t)pi * W + w] | ((i >> 5) == w ? (1u << (i & 31)) : 0u);
       }
@@ -796,7 +797,10 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
     }
   }
   for (int i = tid; i < n; i += BUILD_THREADS) {
-    const bool live = i < nn;
+    bool live = i < nn;
+    if (live && i > 0)   // a live node's parent precedes it, its depth is a block position, its rank a top-K rank
+      live = DDT_IN_RANGE(sm.nd_parent[i], 0, i) && DDT_IN_RANGE(sm.nd_depth[i], 1, L + 1) &&
+             DDT_IN_RANGE(sm.nd_rank[i], 0, kc);
     const int d = live ? sm.nd_depth[i] : -1;
     const int rk = live ? sm.nd_rank[i] : -1;
     if (node_token) node_token[ro + i] = !live ? -1 : (i == 0 ? root_token[r] : idr[(size_t)(d - 1) * K + rk]);

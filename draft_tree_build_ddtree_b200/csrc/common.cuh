@@ -30,6 +30,21 @@ __device__ unsigned int g_status;
 
 __device__ __forceinline__ void flag_status(unsigned int bits) { atomicOr(&g_status, bits); }
 
+// Debug builds (-DDDTREE_DEBUG, libddtree_debug.so): internal indices are
+// checked before they address memory; a violation sets
+// DDTREE_STATUS_BOUNDS and the access is skipped, never a trap.  In release
+// builds the check is `true`.
+#ifdef DDTREE_DEBUG
+__device__ __forceinline__ bool ddt_in_range(long long i, long long lo, long long hi) {
+  if (i >= lo && i < hi) return true;
+  flag_status(DDTREE_STATUS_BOUNDS);
+  return false;
+}
+#define DDT_IN_RANGE(i, lo, hi) ddt::ddt_in_range((long long)(i), (long long)(lo), (long long)(hi))
+#else
+#define DDT_IN_RANGE(i, lo, hi) true
+#endif
+
 // ---------------------------------------------------------------------------
 // Order-preserving integer keys: a > b as reals  <=>  key(a) > key(b).
 // -0.0 maps to the key of +0.0; -inf is the smallest key of a real value.

@@ -63,6 +63,8 @@ typedef enum {
 #define DDTREE_STATUS_TIMEOUT   0x2u
 #define DDTREE_STATUS_CAPACITY  0x4u
 #define DDTREE_STATUS_SETUP     0x8u   /* a kernel could not set up (misaligned shared memory) and did nothing */
+#define DDTREE_STATUS_BOUNDS    0x10u  /* debug build (DDTREE_DEBUG) only: an internal index left its range;
+                                          the access was skipped */
 
 typedef enum { DDTREE_BF16 = 0, DDTREE_F32 = 1 } ddtree_dtype;
 

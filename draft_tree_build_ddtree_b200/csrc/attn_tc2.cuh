@@ -167,7 +167,6 @@ struct T2Params {
   float* ws_o;         // partials per (M-tile unit, split), as for the combine kernel
   float2* ws_ml;
   int lpt;
-  int light_last;      // 1: the one-M-tile pairs (odd M-tile count) are dispatched last
   uint64_t wait_ns;
   int stop_tile;
 };
@@ -189,20 +188,12 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   const int warp = tid >> 5, lane = tid & 31;
 
   // ---- which unit ----
-  // With an odd number of M-tiles the last pair of every (layer, request,
-  // KV head) holds one M-tile and costs about half: those units come last,
-  // so the final wave is made of them.
+  // The units of one (layer, request, KV head) are adjacent in launch order,
+  // so they run close together in time and share its K/V through L2.
   const int split = blockIdx.x % p.splits;
   int u = blockIdx.x / p.splits;
-  int mp;
-  if (p.light_last) {
-    const int nh = p.mpairs - 1;
-    const int heavy = (p.units / p.mpairs) * nh;
-    if (u < heavy) { mp = u % nh; u /= nh; } else { mp = nh; u -= heavy; }
-  } else {
-    mp = u % p.mpairs;
-    u /= p.mpairs;
-  }
+  const int mp = u % p.mpairs;
+  u /= p.mpairs;
   const int kvh = u % g.Hkv; u /= g.Hkv;
   int r = u % g.n_req; u /= g.n_req;
   const int layer = u;
@@ -656,7 +647,6 @@ inline int attn_tc_launch(const void* q, const void* kc, const void* vc, const i
   p.ws_o = nullptr;
   p.ws_ml = nullptr;
   p.lpt = (d.splits == 1 && g.n_req > 1 && g.n_req <= TC_LPT_MAX_REQ) ? 1 : 0;
-  p.light_last = (d.mtiles % 2 == 1) ? 1 : 0;
   p.wait_ns = wait_ns > 0 ? wait_ns : TC_WAIT_NS;
   p.stop_tile = stop_tile;
   const size_t slots = (size_t)g.layers * g.n_req * g.Hkv * d.mtiles * d.splits;

@@ -78,8 +78,14 @@ def parse(argv=None):
 # is reported only while the sources are unchanged (summaries under profiles/).
 CSRC = os.path.join(ROOT, "draft_tree_build_ddtree_b200", "csrc")
 TRAFFIC = {
-    ("b64_p2k", "topk"): (5069568, ("topk.cuh", "common.cuh", "exp64_table.h"), "4c480e2f4cca5119"),
-    ("b256_p8k_48l", "attn"): (1057939712, ("attn_tc.cuh", "attn_simt.cuh", "common.cuh"), "673c3d78fa774a8f"),
+    # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu
+    # captures summarised in profiles/ (keyed to a digest of the kernel's sources)
+    ("b64_p2k", "topk"): (5069056, ("topk.cuh", "common.cuh", "exp64_table.h"), "d3143192fdffa02b"),
+    ("batch32_ragged_paged", "topk"): (161091072, ("topk.cuh", "common.cuh", "exp64_table.h"), "d3143192fdffa02b"),
+    # captured at 8 of the 48 layers (172,030,208 B) and scaled by 6: each
+    # layer's units read that layer's K/V and write its outputs only
+    ("b256_p8k_48l", "attn"): (1032181248, ("attn_tc2.cuh", "attn_tc.cuh", "common.cuh", "exp2_poly.h"),
+                               "4a965ba898324b26"),
 }
 
 

@@ -33,7 +33,15 @@
 
 namespace ddt {
 
-constexpr int BUILD_THREADS = 256;
+// Threads of the build CTA: the enumeration's level passes, scans and sorts
+// scale with the block; the heap fallback uses one warp either way.
+// Measured (one request, L = 16): 256 threads are faster at B = 64 (8.2 vs
+// 8.8 us), 512 at B = 256 (27.9 vs 36.1 us) and B = 1024 (110 vs 142 us);
+// 1024 threads were slower than 512 at every B.
+constexpr int BUILD_THREADS_SMALL = 256;
+constexpr int BUILD_THREADS_LARGE = 512;
+constexpr int BUILD_LARGE_FROM_B = 129;
+inline int build_threads(int B) { return B >= BUILD_LARGE_FROM_B ? BUILD_THREADS_LARGE : BUILD_THREADS_SMALL; }
 
 // Entry metadata: parent node (11 bits), depth (6 bits), rank (15 bits).
 __device__ __forceinline__ uint32_t pack_meta(int parent, int depth, int rank) {
@@ -367,9 +375,10 @@ __device__ __forceinline__ bool e_before(int a, int b, const EnumSmem& es) {
 }
 
 // In-place exclusive scan of v[0..m) by the whole block; returns the total.
+template <int NT>
 __device__ __forceinline__ int block_exclusive_scan(int* v, int m, int* warp_tot) {
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int per = (m + BUILD_THREADS - 1) / BUILD_THREADS;
+  const int per = (m + NT - 1) / NT;
   const int b0 = tid * per, b1 = min(m, b0 + per);
   int sum = 0;
   for (int i = b0; i < b1; ++i) sum += v[i];
@@ -383,7 +392,7 @@ __device__ __forceinline__ int block_exclusive_scan(int* v, int m, int* warp_tot
   __syncthreads();
   int wbase = 0, total = 0;
 #pragma unroll
-  for (int w = 0; w < BUILD_THREADS / 32; ++w) {
+  for (int w = 0; w < NT / 32; ++w) {
     const int t = warp_tot[w];
     if (w < wid) wbase += t;
     total += t;
@@ -402,6 +411,7 @@ __device__ __forceinline__ int block_exclusive_scan(int* v, int m, int* warp_tot
 // Block-uniform.  Fills sm.nd_* for nodes 1..pops.
 // kfloor > 0 raises the score threshold: only prefixes whose score key is
 // at least kfloor are listed (the adaptive budget's floor).
+template <int NT>
 __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B, int kc, TieCode tc,
                           uint32_t* hist, int* bcast, int* warp_tot, float* chain, int* s_lev, uint32_t kfloor) {
   const int tid = threadIdx.x;
@@ -428,12 +438,12 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
       kmin = __reduce_min_sync(0xffffffffu, kmin);
       if (tid == 0) bcast[0] = (int)kmin;
     }
-    for (int i = tid; i < 256; i += BUILD_THREADS) hist[i] = 0;
+    for (int i = tid; i < 256; i += NT) hist[i] = 0;
     __syncthreads();
     const uint32_t kmin = (uint32_t)bcast[0];
     int shift = 0;
     while (((kmax - kmin) >> shift) >= 256u) ++shift;
-    for (int i = tid; i < L * kc; i += BUILD_THREADS) {
+    for (int i = tid; i < L * kc; i += NT) {
       const int d = i / kc;
       const uint32_t key = score_key(__fadd_rn(chain[d], sm.lp[i]));
       atomicAdd(&hist[(key - kmin) >> shift], 1u);
@@ -484,7 +494,7 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
   __syncthreads();
   if (s_lev[2]) return -1;
   int ls = 0, le = s_lev[1];
-  for (int r = tid; r < le; r += BUILD_THREADS) {
+  for (int r = tid; r < le; r += NT) {
     const float sc = __fadd_rn(0.f, sm.lp[r]);
     es.score[r] = sc;
     es.meta[r] = e_pack(ENUM_ROOT, 1, r);
@@ -495,7 +505,7 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
   for (int d = 1; d < L && le > ls; ++d) {        // parents at depth d, children at depth d+1
     const int m = le - ls;
     const float* lpd = sm.lp + d * kc;
-    for (int i = tid; i < m; i += BUILD_THREADS) {
+    for (int i = tid; i < m; i += NT) {
       const float ps = es.score[ls + i];
       int lo = 0, hi = kc;
       while (lo < hi) {
@@ -505,12 +515,12 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
       es.off[i] = lo;
     }
     __syncthreads();
-    const int T = block_exclusive_scan(es.off, m, warp_tot);
+    const int T = block_exclusive_scan<NT>(es.off, m, warp_tot);
     if (le + T > ENUM_CAP) return -1;             // block-uniform
     if (tid == 0) es.off[m] = T;
     __syncthreads();
     const uint32_t unit = tc.unit(d + 1);
-    for (int j = tid; j < T; j += BUILD_THREADS) {
+    for (int j = tid; j < T; j += NT) {
       int lo = 0, hi = m;                         // last parent with off <= j
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -532,10 +542,10 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
   // ---- 3. order: position of every entry among the enumerated set ----
   const int total = le;
   const int npop = total < B ? total : B;
-  if (total <= BUILD_THREADS) {
+  if (total <= NT) {
     // rank by counting; g threads share one entry
     int g = 32;
-    while (g > 1 && total * g > BUILD_THREADS) g >>= 1;
+    while (g > 1 && total * g > NT) g >>= 1;
     const int q = tid / g, part = tid - q * g;
     int rank = 0;
     if (q < total) {
@@ -564,18 +574,18 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
   } else {
     int P = 1;
     while (P < total) P <<= 1;
-    for (int i = tid; i < P; i += BUILD_THREADS) es.ord[i] = (uint16_t)(i < total ? i : 0xFFFFu);
+    for (int i = tid; i < P; i += NT) es.ord[i] = (uint16_t)(i < total ? i : 0xFFFFu);
     __syncthreads();
     for (int size = 2; size <= P; size <<= 1) {
       for (int stride = size >> 1; stride > 0; stride >>= 1) {
         // up to four compare-exchanges per thread, their loads issued together
-        for (int i0 = tid; i0 < P / 2; i0 += 4 * BUILD_THREADS) {
+        for (int i0 = tid; i0 < P / 2; i0 += 4 * NT) {
           int lo[4], hi[4];
           uint16_t a[4], b[4];
           unsigned long long ka[4], kb[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * BUILD_THREADS;
+            const int i = i0 + u * NT;
             lo[u] = 2 * stride * (i / stride) + (i % stride);
             hi[u] = lo[u] + stride;
             const bool in = i < P / 2;
@@ -589,7 +599,7 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
           }
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            if (i0 + u * BUILD_THREADS >= P / 2) continue;
+            if (i0 + u * NT >= P / 2) continue;
             const bool up = (lo[u] & size) == 0;   // this run sorts in pop order
             // b before a (pads last)
             bool b_first;
@@ -603,13 +613,13 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
         __syncthreads();
       }
     }
-    for (int i = tid; i < total; i += BUILD_THREADS) es.pos[i] = 0;
+    for (int i = tid; i < total; i += NT) es.pos[i] = 0;
     __syncthreads();
-    for (int i = tid; i < npop; i += BUILD_THREADS) es.pos[es.ord[i]] = (uint16_t)(i + 1);
+    for (int i = tid; i < npop; i += NT) es.pos[es.ord[i]] = (uint16_t)(i + 1);
   }
   __syncthreads();
   // ---- nodes 1..npop in pop order ----
-  for (int e = tid; e < total; e += BUILD_THREADS) {
+  for (int e = tid; e < total; e += NT) {
     const int node = es.pos[e];
     if (node == 0) continue;
     const uint32_t mt = es.meta[e];
@@ -622,7 +632,8 @@ __device__ int enum_build(const BuildSmem& sm, const EnumSmem& es, int L, int B,
   return npop;
 }
 
-__global__ void __launch_bounds__(BUILD_THREADS, 1)
+template <int NT>
+__global__ void __launch_bounds__(NT, 1)
 build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
              const int32_t* __restrict__ root_token, int L, int K, int B, int kc, TieCode tc, int use_enum,
              const float* __restrict__ gain_floor, int32_t* __restrict__ node_token, int32_t* __restrict__ parent,
@@ -662,7 +673,7 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
   __shared__ int s_pops;
   __shared__ uint32_t s_hist[256];
   __shared__ int s_bcast[4];
-  __shared__ int s_warp_tot[BUILD_THREADS / 32];
+  __shared__ int s_warp_tot[NT / 32];
   __shared__ float s_chain[64];
   __shared__ int s_lev[3];
 
@@ -671,22 +682,22 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
   if ((kc & 3) == 0 && (K & 3) == 0 && ((uintptr_t)lpr & 15) == 0) {
     // 16-byte loads, all of a thread's issued before any is stored
     const int q4 = kc >> 2, total4 = L * q4;
-    for (int i0 = tid; i0 < total4; i0 += 4 * BUILD_THREADS) {
+    for (int i0 = tid; i0 < total4; i0 += 4 * NT) {
       float4 v[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int i = i0 + u * BUILD_THREADS;
+        const int i = i0 + u * NT;
         const int d = i / q4, k4 = i - d * q4;
         if (i < total4) v[u] = *reinterpret_cast<const float4*>(lpr + (size_t)d * K + 4 * k4);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int i = i0 + u * BUILD_THREADS;
+        const int i = i0 + u * NT;
         if (i < total4) reinterpret_cast<float4*>(sm.lp)[i] = v[u];
       }
     }
   } else {
-    for (int i = tid; i < L * kc; i += BUILD_THREADS) {
+    for (int i = tid; i < L * kc; i += NT) {
       const int d = i / kc, k = i - d * kc;
       sm.lp[i] = lpr[(size_t)d * K + k];
     }
@@ -713,7 +724,7 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
   const uint32_t kfloor = !has_floor ? 0u : (floor_v == INFINITY ? 0xFFFFFFFFu : score_key(floor_v) + 1u);
   int epops = -1, how = 0;
   if (use_enum && B > 0)
-    epops = enum_build(sm, es, L, B, kc, tc, s_hist, s_bcast, s_warp_tot, s_chain, s_lev, kfloor);
+    epops = enum_build<NT>(sm, es, L, B, kc, tc, s_hist, s_bcast, s_warp_tot, s_chain, s_lev, kfloor);
   if (epops >= 0) {
     if (tid == 0) s_pops = epops;
   } else if (B > 0) {
@@ -737,7 +748,7 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
     __syncthreads();
     const int pops = s_pops;
     int keep = 0;
-    for (int i = 1 + tid; i <= pops; i += BUILD_THREADS) keep += score_key(sm.nd_score[i]) >= kfloor ? 1 : 0;
+    for (int i = 1 + tid; i <= pops; i += NT) keep += score_key(sm.nd_score[i]) >= kfloor ? 1 : 0;
     keep = __reduce_add_sync(0xffffffffu, keep);
     if ((tid & 31) == 0 && keep) atomicAdd(&s_keep, keep);
     __syncthreads();
@@ -759,14 +770,14 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
     uint32_t* rows = reinterpret_cast<uint32_t*>(smem_raw + (size_t)n * 16);   // [n][W]
     int* order = reinterpret_cast<int*>(rows + (size_t)n * W);                  // [n] nodes sorted by depth
     __shared__ int s_dcnt[66];
-    for (int i = tid; i < 66; i += BUILD_THREADS) s_dcnt[i] = 0;
+    for (int i = tid; i < 66; i += NT) s_dcnt[i] = 0;
     __syncthreads();
-    for (int i = tid; i < nn; i += BUILD_THREADS) atomicAdd(&s_dcnt[sm.nd_depth[i] + 1], 1);
+    for (int i = tid; i < nn; i += NT) atomicAdd(&s_dcnt[sm.nd_depth[i] + 1], 1);
     __syncthreads();
     if (tid == 0)
       for (int d = 1; d < 66; ++d) s_dcnt[d] += s_dcnt[d - 1];   // s_dcnt[d]: first slot of depth d
     __syncthreads();
-    for (int i = tid; i < nn; i += BUILD_THREADS) order[atomicAdd(&s_dcnt[sm.nd_depth[i]], 1)] = i;
+    for (int i = tid; i < nn; i += NT) order[atomicAdd(&s_dcnt[sm.nd_depth[i]], 1)] = i;
     __syncthreads();
     // after the scatter s_dcnt[d] is the end of depth d: depth d spans [s_dcnt[d-1], s_dcnt[d])
     const int lane = tid & 31, wrp = tid >> 5;
@@ -775,7 +786,7 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
     for (int d = 1; d <= L; ++d) {
       const int b0 = s_dcnt[d - 1], b1 = s_dcnt[d];
       if (b0 >= b1) break;
-      for (int k = b0 + wrp; k < b1; k += BUILD_THREADS / 32) {
+      for (int k = b0 + wrp; k < b1; k += NT / 32) {
         const int i = order[k];
         const int pi = sm.nd_parent[i];
         if (!DDT_IN_RANGE(pi, 0, i)) continue;
@@ -784,19 +795,19 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
       }
       __syncthreads();
     }
-    for (int i = nn * W + tid; i < n * W; i += BUILD_THREADS) rows[i] = 0u;   // absent nodes
+    for (int i = nn * W + tid; i < n * W; i += NT) rows[i] = 0u;   // absent nodes
     __syncthreads();
     uint32_t* arow0 = anc + ro * W;
     const int words = n * W;
     if (((uintptr_t)arow0 & 15) == 0) {
-      for (int i = tid; i < words / 4; i += BUILD_THREADS)
+      for (int i = tid; i < words / 4; i += NT)
         reinterpret_cast<uint4*>(arow0)[i] = reinterpret_cast<const uint4*>(rows)[i];
-      for (int i = (words & ~3) + tid; i < words; i += BUILD_THREADS) arow0[i] = rows[i];
+      for (int i = (words & ~3) + tid; i < words; i += NT) arow0[i] = rows[i];
     } else {
-      for (int i = tid; i < words; i += BUILD_THREADS) arow0[i] = rows[i];
+      for (int i = tid; i < words; i += NT) arow0[i] = rows[i];
     }
   }
-  for (int i = tid; i < n; i += BUILD_THREADS) {
+  for (int i = tid; i < n; i += NT) {
     bool live = i < nn;
     if (live && i > 0)   // a live node's parent precedes it, its depth is a block position, its rank a top-K rank
       live = DDT_IN_RANGE(sm.nd_parent[i], 0, i) && DDT_IN_RANGE(sm.nd_depth[i], 1, L + 1) &&

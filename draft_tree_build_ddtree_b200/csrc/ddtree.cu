@@ -172,15 +172,17 @@ int build_launch(const int32_t* ids, const float* lp, const int32_t* root_token,
   if (flags & ~DDTREE_BUILD_FORCE_HEAP) return DDTREE_ERR_INVALID_ARG;
   const int kc = B < K ? B : K;
   // the threshold enumeration when its arrays fit beside the heap's
+  const int nt = build_threads(B);
+  auto kern = nt == BUILD_THREADS_LARGE ? build_kernel<BUILD_THREADS_LARGE> : build_kernel<BUILD_THREADS_SMALL>;
   cudaFuncAttributes attr;
-  if (cudaFuncGetAttributes(&attr, build_kernel) != cudaSuccess) return DDTREE_ERR_CUDA;
+  if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return DDTREE_ERR_CUDA;
   const size_t smem_enum = build_smem_bytes_enum(L, kc, B);
   const int use_enum =
       (!(flags & DDTREE_BUILD_FORCE_HEAP) && smem_enum + attr.sharedSizeBytes <= (size_t)max_smem_optin()) ? 1 : 0;
   const size_t smem = use_enum ? smem_enum : build_smem_bytes(L, kc, B);
-  int st = set_smem(build_kernel, smem);
+  int st = set_smem(kern, smem);
   if (st) return st;
-  build_kernel<<<n_req, BUILD_THREADS, smem, s>>>(ids, lp, root_token, L, K, B, kc, tie_code(kc, L), use_enum,
+  kern<<<n_req, nt, smem, s>>>(ids, lp, root_token, L, K, B, kc, tie_code(kc, L), use_enum,
                                                    gain_floor, node_token, parent, depth, node_rank, score, anc,
                                                    n_nodes, build_path);
   return launch_status();

@@ -451,6 +451,32 @@ def measure(w, a, device, steps, warmup, shard=None, world=1, rank=0, clocks=Non
     ms_max = max_over_ranks(ms, device)
     status = dd.device_status()
 
+    # the spread of single rounds (each bracketed by its own events), and
+    # rounds launched eagerly instead of from CUDA graphs
+    n_each = min(steps, 200)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_each)]
+    for i, (a0, a1) in enumerate(evs):
+        a0.record(stream)
+        step(i)
+        a1.record(stream)
+    torch.cuda.synchronize()
+    each_us = sorted(a0.elapsed_time(a1) * 1e3 for a0, a1 in evs)
+    pct = lambda q: each_us[min(len(each_us) - 1, int(round(q * (len(each_us) - 1))))]
+    round_us = {"p10": round(pct(0.1), 3), "median": round(pct(0.5), 3), "p90": round(pct(0.9), 3),
+                "rounds": n_each}
+    eager_rps = None
+    if use_graph and not gather:
+        n_eager = min(steps, 50)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(n_eager):
+            rb = sets[i % R]
+            dd.ddtree_round(rb, rb._args)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        eager_rps = n_eager / (t0.elapsed_time(t1) / 1e3)
+
     # per-stage times with cold caches as in the rounds: a graph of (L2 flush,
     # stage on set k) for every set, minus the same graph of flushes alone
     flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
@@ -494,7 +520,7 @@ def measure(w, a, device, steps, warmup, shard=None, world=1, rank=0, clocks=Non
         stage_l2[name] = "L2 flushed before each launch"
     del flush_buf
     return dict(w=w_run, sets=sets, R=R, per_set=per_set, ms=ms_max, steps=steps, status=status,
-                stage_ms=stage_ms, stage_l2=stage_l2, work=work, use_graph=use_graph, host0=host0,
+                stage_ms=stage_ms, stage_l2=stage_l2, work=work, round_us=round_us, eager_rps=eager_rps, use_graph=use_graph, host0=host0,
                 launches=dd.ddtree_round_launch_count(sets[0], sets[0]._args),
                 accept_len_mean=float(torch.cat([rb.acc.accept_len.float() for rb in sets]).mean().item()))
 
@@ -598,6 +624,8 @@ def run_ours(a):
                                        else f"replicas x{world}"),
                        "l2": f"{m['R']} rotating input sets of {m['per_set'] / 1e6:.1f} MB (> 2x L2)",
                        "launch": "cuda graph per round" if m["use_graph"] else "eager"},
+            "round_us": m["round_us"],
+            "eager_rounds_per_s": m["eager_rps"],
             "stages_us": {k: round(v["us"], 3) for k, v in stages.items()},
             "stages_l2": m["stage_l2"],
             "stages": stages,
@@ -699,8 +727,21 @@ def cpu_baseline(w, h, budget_s=15.0):
             secs.append(s)
             n += 1
     per_round = statistics.median(secs)
-    return {"value": 1.0 / per_round, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n} timed oracle rounds ({desc}); numpy/BLAS limited to 1 thread"}
+    out = {"value": 1.0 / per_round, "unit": UNIT, "cores": 1, "kind": "oracle",
+           "sample": f"{n} timed oracle rounds ({desc}); numpy/BLAS limited to 1 thread"}
+    # the same sample with numpy's BLAS on every host core (its dense
+    # attention products are the part that runs in parallel)
+    cores = os.cpu_count() or 1
+    if cores > 1:
+        secs_all = []
+        with threadpool_limits(limits=cores):
+            t_end = time.perf_counter() + budget_s / 2
+            while not secs_all or (time.perf_counter() < t_end and len(secs_all) < 10):
+                s, _, _ = oracle_round(w, h, sample)
+                secs_all.append(s)
+        out["all_cores"] = {"value": 1.0 / statistics.median(secs_all), "cores": cores,
+                            "sample": f"{len(secs_all)} timed oracle rounds, numpy/BLAS on {cores} threads"}
+    return out
 
 
 def run_reference(a):

@@ -48,6 +48,7 @@ UNIT = "rounds/s"
 L2_BYTES = 126 * 1024 * 1024
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_HBM_GBS = 8000.0   # the workload statement's nominal HBM bandwidth (context, not the denominator)
 DEFAULT_CONFIG = 3
 PER_CONFIG = ((2, {}), (4, {}), (5, {"B": 64, "sigma": 4.0}), (5, {"B": 256, "sigma": 4.0}))
 SUSTAINED_AFTER_S = 1.0      # a timed region at least this long is graded against the sustained peak
@@ -382,6 +383,7 @@ def stage_report(w, work, stage_ms, peaks, long_region: bool):
         wk = work[name]
         d = {"us": t * 1e3, "bytes": wk["bytes"], "flops": wk["flops"], "gbs": wk["bytes"] / (t * 1e-3) / 1e9}
         d["hbm_frac"] = d["gbs"] / hbm
+        d["hbm_frac_nominal"] = d["gbs"] / NOMINAL_HBM_GBS
         if wk["flops"]:
             d["tflops"] = wk["flops"] / (t * 1e-3) / 1e12
             d["tensor_frac_burst"] = d["tflops"] / burst
@@ -603,7 +605,7 @@ def run_ours(a):
                 "ms_per_round": mc["ms"] / mc["steps"], "steps": mc["steps"], "device_status": mc["status"],
                 "stages_us": {k: round(v["us"], 3) for k, v in st_c.items()},
                 "stages_l2": mc["stage_l2"],
-                "roof": {k: {kk: v[kk] for kk in ("bound", "frac", "hbm_frac", "tensor_frac_burst",
+                "roof": {k: {kk: v[kk] for kk in ("bound", "frac", "hbm_frac", "hbm_frac_nominal", "tensor_frac_burst",
                                                   "tensor_frac_sustained", "gbs", "tflops") if kk in v}
                          for k, v in st_c.items()},
                 "accept_len_mean": mc["accept_len_mean"]}

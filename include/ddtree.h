@@ -443,7 +443,9 @@ int ddtree_round_launch_count(const ddtree_round_args* a);
  *      buffer of `dev`.
  * The call returns once everything is enqueued; synchronise `stream` before
  * reading the host outputs.  Host pointers left NULL are not copied (an
- * input then keeps whatever the device buffer holds).
+ * input then keeps whatever the device buffer holds).  Calls on different
+ * streams with disjoint `dev` buffers and workspaces may run at the same
+ * time: one round's copies then overlap another round's kernels.
  */
 typedef struct {
   /* inputs (host) */

@@ -72,6 +72,40 @@ def test_round_from_host_buffers(cfg):
     assert host.h2d_bytes == expect_h2d
 
 
+def test_round_from_host_concurrent_streams():
+    """Two host-buffer rounds with disjoint device buffers, issued on two
+    streams so that one round's copies overlap the other's kernels, give the
+    same outputs, bit for bit, as the same rounds run one after the other."""
+    w = datagen.workload(2)
+    pairs = []
+    for rep in (0, 1):
+        z, ids, lp32, lse32, root, trees, st = tree_inputs(w, rep)
+        prefix = datagen.prefix_lengths(w, rep)
+        cache = datagen.kv_cache(w, prefix, rep)
+        q = datagen.queries(w, rep)
+        tgt = datagen.target_logits(w, z, torch.from_numpy(st["depth"]), torch.from_numpy(st["n_nodes"]), rep)
+        rb = _round_buffers(w, z, root, q, cache, prefix, tgt)
+        pairs.append((rb, host_api.make_host_round(rb)))
+    ref = []
+    for rb, host in pairs:
+        host_api.round_from_host(rb, host, rb.args())
+        torch.cuda.synchronize()
+        ref.append({k: v.clone() for k, v in host.outputs.items()})
+    for _, host in pairs:
+        for v in host.outputs.values():
+            v.zero_()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for _ in range(4):
+        for (rb, host), s in zip(pairs, streams):
+            with torch.cuda.stream(s):
+                host_api.round_from_host(rb, host, rb.args())
+    torch.cuda.synchronize()
+    assert dd.device_status() == 0
+    for (_, host), r in zip(pairs, ref):
+        for k, v in r.items():
+            assert torch.equal(host.outputs[k].view(torch.uint8), v.view(torch.uint8)), k
+
+
 def test_round_from_host_rejects_paged_tree_rows():
     w = datagen.workload(4, N=2)
     z, ids, lp32, lse32, root, trees, st = tree_inputs(w)

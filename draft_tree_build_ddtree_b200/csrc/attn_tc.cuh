@@ -16,12 +16,16 @@
 // 128B-swizzled shared memory, fp32 accumulator in TMEM), then the softmax
 // warps read S from TMEM (one thread per row = TMEM lane), apply the
 // ancestor mask only on tiles that reach the tree slots, update the running
-// max/sum, write P = exp2(S*scale*log2e - m) as bf16 into shared memory
-// (K-major, swizzled like a TMA tile), and O += P V (V as an MN-major
-// operand) accumulates in TMEM.  O is rescaled only when the running max
-// grows by more than 2^8, which keeps every P <= 256 and leaves the final
-// O / l exact.  K and V tiles are double buffered; the QK^T of the next tile
-// overlaps the softmax of the current one.
+// max/sum, write P = exp2(S*scale*log2e - m) as packed bf16 pairs into
+// tensor-memory columns of its own, and O += P V (tcgen05.mma with the A
+// operand in TMEM, V as an MN-major operand from shared memory) accumulates
+// in TMEM.  O is rescaled only when the running max grows by more than 2^8,
+// which keeps every P <= 256 and leaves the final O / l exact.  K and V tiles
+// are double buffered; S is released as soon as the softmax has loaded it,
+// so the QK^T of the next tile overlaps the softmax of the current one.
+// (P in tensor memory instead of shared memory: b64_p2k attention 15.1 vs
+// 15.5 us, and 1.92 vs 2.05 ms when this kernel runs the 48-layer B = 256
+// workload.)
 //
 // Warp roles (192 threads): warps 0-3 softmax + epilogue (warp w reads TMEM
 // lanes 32w..32w+31), warp 4 the TMA producer, warp 5 TMEM allocation and
@@ -59,11 +63,13 @@ template <int BN>
 struct TcCfg {
   static constexpr int KATOM = BN * 64 * 2;     // one [BN keys][64 dims] bf16 atom
   static constexpr int KTILE = 2 * KATOM;       // a K or V tile [BN keys][128 dims]
-  static constexpr int PTILE = TC_BM * BN * 2;  // P [128 rows][BN keys] bf16
   static constexpr int CTAS = BN == 64 ? 2 : 1; // CTAs per SM
+  // tensor memory: S [0, BN), O [BN, BN+128), P [BN+128, BN+128+BN/2)
+  // (bf16 pairs); 224 of 256 columns at BN = 64 (two CTAs per SM), 320 of 512
+  // at BN = 128
+  static constexpr uint32_t TMEM_COLS = BN == 64 ? 256 : 512;
 };
 constexpr int TC_STAGES = 2;
-constexpr uint32_t TC_TMEM_COLS = 256;      // S: cols [0,64), O: cols [64,192); two CTAs per SM
 constexpr float TC_RESCALE_LOG2 = 8.0f;
 
 inline bool tc_attn_supported(int group) { return group >= 1 && group <= TC_BM && (TC_BM % group) == 0; }
@@ -176,6 +182,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+// D[tmem] (+)= A[tmem] * B[smem]: kind::f16 with the A operand in tensor memory.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
@@ -226,7 +241,6 @@ struct TcSmem {
   unsigned char q[TC_TILE];
   unsigned char k[TC_STAGES][TcCfg<BN>::KTILE];
   unsigned char v[TC_STAGES][TcCfg<BN>::KTILE];
-  unsigned char p[TcCfg<BN>::PTILE];
   uint64_t bar_q, bar_kf[TC_STAGES], bar_ke[TC_STAGES], bar_vf[TC_STAGES], bar_ve[TC_STAGES];
   uint64_t bar_sfull, bar_sfree, bar_pfull, bar_pvdone;
   uint32_t tmem_base;
@@ -330,15 +344,16 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   }
   if (warp == 5) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
-                 "r"(TC_TMEM_COLS));
+                 "r"(TcCfg<BN>::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t tmem_s = tmem;              // cols [0,64)
+  const uint32_t tmem_s = tmem;              // cols [0, BN)
   const uint32_t tmem_o = tmem + TC_BN;      // cols [BN, BN+128)
+  const uint32_t tmem_p = tmem + TC_BN + TC_D;   // cols [BN+128, BN+128+BN/2): P as bf16 pairs
   volatile int* abort = &sm.abort;
   const float sl2 = g.scale * 1.4426950408889634f;   // scale * log2(e)
 
@@ -402,7 +417,7 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (lane == 0 && nt > 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(TC_BM, TC_BN, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(TC_BM, TC_D, false, true);
-      const uint32_t q_addr = smem_u32(sm.q), p_addr = smem_u32(sm.p);
+      const uint32_t q_addr = smem_u32(sm.q);
       bool ok = mbar_wait(&sm.bar_q, 0, abort, p.wait_ns);
       int committed_pv = 0, committed_qk = 0;
       for (int jj = 0; ok && jj <= nt; ++jj) {
@@ -431,11 +446,9 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           tc_fence_after();
           const uint32_t v_addr = smem_u32(sm.v[st]);
 #pragma unroll
-          for (int kk = 0; kk < TC_BN / 16; ++kk) {
-            const uint32_t a_off = (kk >> 2) * TC_ATOM + (kk & 3) * 32;   // P: 64-key atoms
-            umma_f16(tmem_o, smem_desc_sw128(p_addr + a_off, 16, 1024),
-                     smem_desc_sw128(v_addr + kk * 16 * 128, TC_KATOM, 1024), IDESC_PV, (pj > 0 || kk > 0));
-          }
+          for (int kk = 0; kk < TC_BN / 16; ++kk)       // P from tensor memory: 16 keys = 8 columns per step
+            umma_f16_ts(tmem_o, tmem_p + kk * 8, smem_desc_sw128(v_addr + kk * 16 * 128, TC_KATOM, 1024), IDESC_PV,
+                        (pj > 0 || kk > 0));
           umma_commit(&sm.bar_pvdone);
           umma_commit(&sm.bar_ve[st]);
           committed_pv = jj;
@@ -548,15 +561,10 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (rescale) m_used = m_new;
       }
       l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
-      // into the swizzled K-major P tile
-      unsigned char* prow = sm.p + row * 128;
+      // P into its tensor-memory columns (this thread's lane), the PV product's A operand
 #pragma unroll
-      for (int ch = 0; ch < TC_BN / 8; ++ch) {
-        const int atom = ch >> 3, c16 = ch & 7;
-        *reinterpret_cast<uint4*>(prow + atom * TC_ATOM + ((c16 ^ (row & 7)) << 4)) =
-            make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      for (int c = 0; c < TC_BN / 64; ++c) tmem_st32(tmem_p + lane_off + 32 * c, reinterpret_cast<const float*>(pk + 32 * c));
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.bar_pfull);
     }
@@ -617,7 +625,7 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   if (warp == 5) {
     __syncwarp();
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_TMEM_COLS));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TcCfg<BN>::TMEM_COLS));
   }
 }
 

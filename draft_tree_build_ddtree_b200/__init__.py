@@ -107,6 +107,7 @@ _SIGS = {
     "ddtree_last_error": (ctypes.c_char_p, []),
     "ddtree_topk_static_ws": (_i, [_vp, _i, _i, _i, _ll, _i, _vp, _vp, _vp, _vp]),
     "ddtree_debug_attn_timeout": (_i, [ctypes.c_ulonglong, _i]),
+    "ddtree_attn_plan": (_i, [ctypes.POINTER(KVDesc), _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     "ddtree_round_host": (_i, [ctypes.POINTER(RoundArgs), _vp, _vp]),
     "ddtree_round_host_bytes": (_i, [ctypes.POINTER(RoundArgs), _vp, ctypes.POINTER(ctypes.c_ulonglong),
                                      ctypes.POINTER(ctypes.c_ulonglong)]),
@@ -304,6 +305,18 @@ def ddtree_tree_attn(q, k_cache, v_cache, kv: KVDesc, prefix_len, anc, n_nodes, 
                                   _stream()),
            "ddtree_tree_attn")
     return out, out_lse
+
+
+ATTN_KERNELS = {0: "cuda_core", 1: "one_mtile", 2: "two_mtile"}
+
+
+def attn_plan(kv: KVDesc, B: int, dtype: int = BF16, num_sms: int = 0):
+    """(kernel name, key-range splits) that ddtree_tree_attn launches for this
+    geometry; host-only.  num_sms = 0 plans for the current device."""
+    k, sp = ctypes.c_int(-1), ctypes.c_int(-1)
+    _check(lib().ddtree_attn_plan(ctypes.byref(kv), B, dtype, num_sms, ctypes.byref(k), ctypes.byref(sp)),
+           "ddtree_attn_plan")
+    return ATTN_KERNELS[k.value], sp.value
 
 
 def ddtree_tree_kv_write(k_in, v_in, depth, n_nodes, prefix_len, kv: KVDesc, k_cache, v_cache, B,

@@ -695,6 +695,21 @@ int ddtree_round(const ddtree_round_args* a, cudaStream_t stream) {
   return round_stages(a, stream, (char*)a->ws, off_attn, off_acc, need, mk);
 }
 
+int ddtree_attn_plan(const ddtree_kv_desc* kv, int B, int dtype, int sms, int* kernel, int* splits) {
+  int st = kv_check(kv);
+  if (st) return st;
+  if (!dtype_ok(dtype) || B < 0 || B > MAX_B || sms < 0 || !kernel || !splits) return DDTREE_ERR_INVALID_ARG;
+  if (!use_tc_attn(dtype, kv)) {
+    *kernel = 0;
+    *splits = 1;
+    return DDTREE_OK;
+  }
+  const AttnDispatch d = attn_dispatch(geom_of(kv, B), sms > 0 ? sms : num_sms());
+  *kernel = d.v2 ? 2 : 1;
+  *splits = d.v2 ? d.splits : d.v1.splits;
+  return DDTREE_OK;
+}
+
 int ddtree_debug_attn_timeout(unsigned long long wait_ns, int withhold_tile) {
   if (withhold_tile < -1) return DDTREE_ERR_INVALID_ARG;
   g_attn_wait_ns = wait_ns;

@@ -542,6 +542,21 @@ int ddtree_device_status(cudaStream_t stream, unsigned int* bits);
  */
 int ddtree_debug_attn_timeout(unsigned long long wait_ns, int withhold_tile);
 
+/*
+ * Which attention kernel ddtree_tree_attn (and the round's attention stage)
+ * launches for this cache geometry and tree budget B (no counterpart in the
+ * paper; host-only, no device work).  dtype as in ddtree_tree_attn;
+ * num_sms: the SM count to plan for (0: the current device's).  On
+ * DDTREE_OK, *kernel is
+ *   0  CUDA-core kernel (fp32, or a head grouping the tensor cores do not take),
+ *   1  one M-tile of 128 rows per CTA (short key ranges),
+ *   2  two M-tiles per CTA sharing each key tile (long key ranges; D = 64 always),
+ * and *splits the number of key-range splits (1: no combine launch).
+ * Returns DDTREE_ERR_INVALID_ARG / DDTREE_ERR_UNSUPPORTED as ddtree_tree_attn
+ * would for the geometry, or for null outputs.
+ */
+int ddtree_attn_plan(const ddtree_kv_desc* kv, int B, int dtype, int num_sms, int* kernel, int* splits);
+
 /* The call and the CUDA runtime's message behind the last DDTREE_ERR_CUDA
  * return of a host-side launch or set-up step (empty before any). */
 const char* ddtree_last_error(void);

@@ -217,7 +217,8 @@ def test_attention_paged_batched_sampled():
     w = datagen.workload(4)
     st, prefix, cache, q = _attn_case(w)
     out, lse = _gpu_attn(w, st, prefix, cache, q)
-    _check_attn(w, st, prefix, cache, q, out, lse, reqs=[0, 13, 31], nodes=[0, 1, 5, 33, 64],
+    # nodes 20 and 50 sit in M-tiles 1 and 3: the second M-tile of a two-M-tile CTA
+    _check_attn(w, st, prefix, cache, q, out, lse, reqs=[0, 13, 31], nodes=[0, 1, 5, 20, 33, 50, 64],
                 heads=[0, 7, 8, 31])
 
 
@@ -234,6 +235,58 @@ def test_attention_long_prefix_b1024_sampled():
     st, prefix, cache, q = _attn_case(w)
     out, lse = _gpu_attn(w, st, prefix, cache, q)
     _check_attn(w, st, prefix, cache, q, out, lse, nodes=[0, 1, 511, 1000, 1024], heads=[0, 31])
+
+
+def _plan(w, cache):
+    kv = dd.kv_desc_for(cache.k, w.N, w.Hq, cache.block_table)
+    return dd.attn_plan(kv, w.B, dd.BF16 if w.dtype == "bf16" else dd.F32)
+
+
+def test_attention_two_mtile_every_row():
+    """The two-M-tile kernel on 4 layers of the B = 256 tree over a
+    1000-token prefix (a ragged last key tile; 17 M-tiles, so the last CTA's
+    second M-tile has no rows): every node and head of two layers against
+    the oracle."""
+    w = datagen.workload(3, layers=4, P=1000)
+    st, prefix, cache, q = _attn_case(w)
+    assert _plan(w, cache) == ("two_mtile", 1)
+    out, lse = _gpu_attn(w, st, prefix, cache, q)
+    _check_attn(w, st, prefix, cache, q, out, lse, layers=[0, 3])
+
+
+def test_attention_two_mtile_split():
+    """The two-M-tile kernel split twelve ways over a 32k prefix (B = 64),
+    merged by the combine kernel: every node at four heads."""
+    w = datagen.workload(5)
+    st, prefix, cache, q = _attn_case(w)
+    assert _plan(w, cache) == ("two_mtile", 12)
+    out, lse = _gpu_attn(w, st, prefix, cache, q)
+    _check_attn(w, st, prefix, cache, q, out, lse, heads=[0, 7, 8, 31])
+
+
+def test_attention_two_mtile_wait_timeout_reports_and_recovers():
+    """The two-M-tile kernel's bounded waits: the producer withholds key
+    tile 1, the MMA issuer's wait for it runs out after 200 us, every role
+    leaves its loop, waits for its copies and products, frees the tensor
+    memory and returns; the next call matches the oracle."""
+    w = datagen.workload(3, layers=4, P=1000)
+    st, prefix, cache, q = _attn_case(w)
+    assert _plan(w, cache) == ("two_mtile", 1)
+    lib = dd.lib()
+    try:
+        assert lib.ddtree_debug_attn_timeout(200_000, 1) == 0
+        dev = _to_dev_cache(cache)
+        kv = dd.kv_desc_for(dev.k, w.N, w.Hq, dev.block_table)
+        dd.ddtree_tree_attn(q.to(CUDA), dev.k, dev.v, kv, _dev(prefix), _dev(st["anc"]), _dev(st["n_nodes"]), w.B)
+        torch.cuda.synchronize()
+        bits = dd.device_status()
+        assert bits & dd.STATUS_TIMEOUT, bits
+        assert not bits & dd.STATUS_SETUP
+        assert dd.device_status() == 0
+    finally:
+        assert lib.ddtree_debug_attn_timeout(0, -1) == 0
+    out, lse = _gpu_attn(w, st, prefix, cache, q)
+    _check_attn(w, st, prefix, cache, q, out, lse, layers=[1], nodes=[0, 1, 100, 255, 256])
 
 
 def test_attention_budget_zero_is_decode():

@@ -137,22 +137,28 @@ def test_launch_plans_from_sizes(lib):
     slots = 20 * 7
     assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv2), 64) == \
         _align256(slots * 128 * 128 * 4) + _align256(slots * 128 * 8)
+    assert dd.attn_plan(kv2, 64, num_sms=148) == ("one_mtile", 7)
     # sweep_p32k at B = 64: the two-M-tile kernel, 4 KV heads x 3 M-tile pairs
     # split 12 ways; partials per (M-tile, split): 4 x 5 x 12
     kv5 = dd.kv_desc(1, 1, 32, 4, 128, s_max=32896)
+    assert dd.attn_plan(kv5, 64, num_sms=148) == ("two_mtile", 12)
     slots = 4 * 5 * 12
     assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv5), 64) == \
         _align256(slots * 128 * 128 * 4) + _align256(slots * 128 * 8)
     # bf16 with D = 64 always takes the two-M-tile kernel: b64_p2k's shape
     # with D = 64 splits its 12 M-tile pairs twice (8 key tiles each at least)
     kv64 = dd.kv_desc(1, 1, 32, 4, 64, s_max=2176)
+    assert dd.attn_plan(kv64, 64, num_sms=148) == ("two_mtile", 2)
     slots = 4 * 5 * 2
     assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv64), 64) == \
         _align256(slots * 128 * 64 * 4) + _align256(slots * 128 * 8)
     kv3 = dd.kv_desc(48, 1, 32, 4, 128, s_max=8512)
     assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv3), 256) == 0
+    assert dd.attn_plan(kv3, 256, num_sms=148) == ("two_mtile", 1)
+    assert dd.attn_plan(kv3, 256, dd.F32, num_sms=148) == ("cuda_core", 1)
     kv4 = dd.kv_desc(1, 32, 32, 4, 128, paged=True, num_blocks=4096, max_blocks=258)
     assert lib.ddtree_attn_workspace_bytes(ctypes.byref(kv4), 64) == 0
+    assert dd.attn_plan(kv4, 64, num_sms=148) == ("two_mtile", 1)
     # accept: composite slots, argmax, one ticket per request
     n = 65
     assert lib.ddtree_accept_workspace_bytes(32, 64, V) == \

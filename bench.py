@@ -83,10 +83,10 @@ TRAFFIC = {
     # captures summarised in profiles/ (keyed to a digest of the kernel's sources)
     ("b64_p2k", "topk"): (5069056, ("topk.cuh", "common.cuh", "exp64_table.h"), "d3143192fdffa02b"),
     ("batch32_ragged_paged", "topk"): (161091072, ("topk.cuh", "common.cuh", "exp64_table.h"), "d3143192fdffa02b"),
-    # captured at 8 of the 48 layers (168,194,304 B) and scaled by 6: each
+    # captured at 8 of the 48 layers (171,388,672 B) and scaled by 6: each
     # layer's units read that layer's K/V and write its outputs only
-    ("b256_p8k_48l", "attn"): (1009165824, ("attn_tc2.cuh", "attn_tc.cuh", "common.cuh", "exp2_poly.h"),
-                               "2f4a5e4073f1a1a4"),
+    ("b256_p8k_48l", "attn"): (1028332032, ("attn_tc2.cuh", "attn_tc.cuh", "common.cuh", "exp2_poly.h"),
+                               "d4a7b7dfbb6995d9"),
 }
 
 

@@ -322,23 +322,25 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(TC_BM, D, false, true);
       bool ok = mbar_wait(&sm.bar_q, 0, abort, wlim);
       bool any_commit = false;
+      // descriptors advance by (byte offset >> 4) in their 14-bit address field
+      const uint64_t qd0 = smem_desc_sw128(smem_u32(sm.q[0]), 16, 1024);
+      const uint64_t kd0 = smem_desc_sw128(smem_u32(sm.k[0]), 16, 1024);
+      const uint64_t vd0 = smem_desc_sw128(smem_u32(sm.v[0]), T2_KATOM, 1024);
       auto issue_s = [&](int t, int st) {      // S_t = Q_t K^T over the 128 head dims
-        const uint32_t q_addr = smem_u32(sm.q[t]), k_addr = smem_u32(sm.k[st]);
+        const uint64_t qd = qd0 + (uint64_t)((t * Smem::QTILE) >> 4);
+        const uint64_t kd = kd0 + (uint64_t)((st * Smem::KTILE) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * TC_ATOM + (kk & 3) * 32;
-          const uint32_t koff = (kk >> 2) * T2_KATOM + (kk & 3) * 32;
-          umma_f16(tmem + 128 * t, smem_desc_sw128(q_addr + off, 16, 1024),
-                   smem_desc_sw128(k_addr + koff, 16, 1024), IDESC_QK, kk > 0);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_f16(tmem + 128 * t, qd + (uint64_t)(((kk >> 2) * TC_ATOM + (kk & 3) * 32) >> 4),
+                   kd + (uint64_t)(((kk >> 2) * T2_KATOM + (kk & 3) * 32) >> 4), IDESC_QK, kk > 0);
         umma_commit(&sm.bar_sfull[t]);
       };
       auto issue_pv = [&](int t, int st, int jj) {   // O_t += P_t V over the 128 keys
-        const uint32_t v_addr = smem_u32(sm.v[st]);
+        const uint64_t vd = vd0 + (uint64_t)((st * Smem::KTILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < T2_BN / 16; ++kk)
-          umma_f16_ts(tmem + 256 + 128 * t, tmem + 128 * t + kk * 8,
-                      smem_desc_sw128(v_addr + kk * 16 * 128, T2_KATOM, 1024), IDESC_PV, (jj > 0 || kk > 0));
+          umma_f16_ts(tmem + 256 + 128 * t, tmem + 128 * t + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), IDESC_PV,
+                      (jj > 0 || kk > 0));
       };
       if (ok && mbar_wait(&sm.bar_kf[0], 0, abort, wlim)) {
         tc_fence_after();

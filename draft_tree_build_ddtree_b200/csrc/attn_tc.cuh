@@ -233,6 +233,7 @@ struct TcParams {
   int lpt;             // 1: requests taken longest key range first (unsplit only)
   uint64_t wait_ns;    // limit of the pipeline's bounded waits
   int stop_tile;       // >= 0: the producer issues no key tile from this one on (timeout-path diagnostics)
+  int early;           // 1: launched while the tree is still being built (see the kernel)
 };
 
 template <int BN>
@@ -300,10 +301,17 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   }
   const int nodes_per_tile = TC_BM / p.G;
   const int node0 = mt * nodes_per_tile;
-  const int nn = p.n_nodes[r];
-  if (node0 >= nn) return;                       // this M-tile holds no live node
   const int P = p.prefix_len[r];
   const long long cap = g.paged ? (long long)g.max_blocks * DDTREE_PAGE : (long long)g.s_max;
+  // Early start (inside a round, contiguous cache): the build of this round's
+  // tree may still be running.  The CTA tiles over the budget's node bound
+  // g.n (keys >= P + n_nodes are masked anyway) and its softmax warps wait for
+  // the build only before the first tile holding tree slots and before the
+  // epilogue, which are the only readers of the tree.  Otherwise it waits here.
+  const bool early = p.early && P >= 0 && (long long)P + g.n <= cap;
+  if (!early) griddep_wait();
+  const int nn = early ? g.n : p.n_nodes[r];     // node bound of the tiling
+  if (node0 >= nn) return;                       // this M-tile holds no live node
   if (P < 0 || (long long)P + nn > cap) {
     if (tid == 0 && mt == 0 && kvh == 0 && split == 0) flag_status(DDTREE_STATUS_CAPACITY);
     return;
@@ -468,6 +476,15 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int hq = kvh * p.G + row % p.G;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const uint32_t* arow = p.anc + ((size_t)r * g.n + min(node, g.n - 1)) * g.W;
+    int nn_act = nn;                                      // the tree's node count, once the build is seen done
+    bool tree_seen = !early;
+    auto see_tree = [&]() {
+      if (!tree_seen) {
+        griddep_wait();
+        nn_act = p.n_nodes[r];
+        tree_seen = true;
+      }
+    };
     float m_used = -INFINITY;      // running max (log2 units) the accumulation uses
     float l = 0.f;
     bool ok = true;
@@ -486,6 +503,7 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       // mask: keys >= P are tree slots (visible iff an ancestor), keys >= T absent.
       // Four 32-key visibility words per tile, built from the node's ancestor row.
       if (k0 + TC_BN > P) {
+        see_tree();
         uint32_t mw[TC_BN / 32];
 #pragma unroll
         for (int w = 0; w < TC_BN / 32; ++w) {
@@ -495,11 +513,11 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           if (j0 <= -32) {
             word = 0xffffffffu;                        // all prefix keys
           } else if (j0 < 0) {
-            word = (node < nn ? (arow[0] << (-j0)) : 0u) | ((1u << (-j0)) - 1u);
+            word = (node < nn_act ? (arow[0] << (-j0)) : 0u) | ((1u << (-j0)) - 1u);
           } else {
             const int wi = j0 >> 5, sh = j0 & 31;
-            const uint32_t lo = (node < nn && wi < g.W) ? arow[wi] : 0u;
-            const uint32_t hi = (node < nn && wi + 1 < g.W) ? arow[wi + 1] : 0u;
+            const uint32_t lo = (node < nn_act && wi < g.W) ? arow[wi] : 0u;
+            const uint32_t hi = (node < nn_act && wi + 1 < g.W) ? arow[wi + 1] : 0u;
             word = __funnelshift_r(lo, hi, sh);
           }
           mw[w] = word;
@@ -569,11 +587,12 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       mbar_arrive(&sm.bar_pfull);
     }
     // ---- epilogue ----
+    see_tree();
     bool fin = ok && nt > 0;
     if (fin) fin = mbar_wait(&sm.bar_pvdone, (nt - 1) & 1, abort, p.wait_ns);
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
-      const bool live = node < nn;
+      const bool live = node < nn_act;
       if (p.splits == 1) {
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
         __nv_bfloat16* orow =
@@ -782,7 +801,7 @@ inline bool make_map_4d(CUtensorMap* m, const void* base, uint64_t d1, uint64_t 
 inline int tc_attn_launch(const void* q, const void* kc, const void* vc, const int32_t* block_table,
                           const int32_t* prefix_len, const uint32_t* anc, const int32_t* n_nodes, const AttnGeom& g,
                           void* out, float* out_lse, void* ws, int num_sms, cudaStream_t stream,
-                          uint64_t wait_ns = 0, int stop_tile = -1) {
+                          uint64_t wait_ns = 0, int stop_tile = -1, int early = 0) {
   TcPlan pl = tc_plan(g, num_sms);
   TcParams p;
   p.g = g;
@@ -801,6 +820,7 @@ inline int tc_attn_launch(const void* q, const void* kc, const void* vc, const i
   p.lpt = (pl.splits == 1 && g.n_req > 1 && g.n_req <= TC_LPT_MAX_REQ) ? 1 : 0;
   p.wait_ns = wait_ns > 0 ? wait_ns : TC_WAIT_NS;
   p.stop_tile = stop_tile;
+  p.early = (early && !g.paged && !p.lpt) ? 1 : 0;   // start during the build (see the kernel)
   if (pl.splits > 1) {
     const size_t slots = (size_t)pl.units * pl.splits;
     p.ws_o = (float*)ws;
@@ -830,11 +850,12 @@ inline int tc_attn_launch(const void* q, const void* kc, const void* vc, const i
   }
   const long long grid = (long long)pl.units * pl.splits;
   if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
-  if (pl.bn == 64)
-    tree_attn_tc_kernel<64><<<(unsigned)grid, TC_THREADS, tc_smem_bytes<64>(), stream>>>(mq, mk, mv, p);
-  else
-    tree_attn_tc_kernel<128><<<(unsigned)grid, TC_THREADS, tc_smem_bytes<128>(), stream>>>(mq, mk, mv, p);
-  if (cudaGetLastError() != cudaSuccess) return DDTREE_ERR_CUDA;
+  const cudaError_t le =
+      pl.bn == 64 ? launch_maybe_pdl(tree_attn_tc_kernel<64>, dim3((unsigned)grid), dim3(TC_THREADS),
+                                     tc_smem_bytes<64>(), stream, p.early != 0, mq, mk, mv, p)
+                  : launch_maybe_pdl(tree_attn_tc_kernel<128>, dim3((unsigned)grid), dim3(TC_THREADS),
+                                     tc_smem_bytes<128>(), stream, p.early != 0, mq, mk, mv, p);
+  if (le != cudaSuccess || cudaGetLastError() != cudaSuccess) return DDTREE_ERR_CUDA;
   if (pl.splits > 1) {
     if (pl.splits <= 8)
       tree_attn_combine_kernel<8><<<pl.units * (TC_D / 8), TC_BM, 0, stream>>>(p);

@@ -645,6 +645,9 @@ build_kernel(const int32_t* __restrict__ ids, const float* __restrict__ lp,
   const int tid = threadIdx.x;
   const int n = B + 1;
   const int W = (n + 31) >> 5;
+  // the round's attention may start its prefix tiles now (it waits for this
+  // grid before reading the tree)
+  griddep_launch_dependents();
 
   BuildSmem sm;
   {

@@ -3,6 +3,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <utility>
 #include <stdint.h>
 #include <stdio.h>
 
@@ -29,6 +30,36 @@ inline int cuda_fail_msg(const char* where) {
 __device__ unsigned int g_status;
 
 __device__ __forceinline__ void flag_status(unsigned int bits) { atomicOr(&g_status, bits); }
+
+// Programmatic dependent launch: a grid launched with programmatic stream
+// serialization may start while the grid before it still runs; it must pass
+// griddep_wait (which returns once that grid has completed and its writes are
+// visible, and at once for a grid launched without the attribute) before it
+// reads anything that grid writes.  griddep_launch_dependents lets such a
+// dependent start as soon as every CTA of this grid has executed it.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launch with programmatic stream serialization when `pdl` (the kernel then
+// starts while the preceding kernel in the stream runs and must griddep_wait
+// before reading its outputs); a plain launch otherwise.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_maybe_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                    bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Debug builds (-DDDTREE_DEBUG, libddtree_debug.so): internal indices are
 // checked before they address memory; a violation sets

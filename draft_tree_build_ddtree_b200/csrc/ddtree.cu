@@ -236,7 +236,7 @@ size_t attn_ws(const ddtree_kv_desc* kv, int B, int dtype) {
 int attn_launch(const void* q, const void* k_cache, const void* v_cache, int dtype, const ddtree_kv_desc* kv,
                 const int32_t* block_table, const int32_t* prefix_len, const uint32_t* anc,
                 const int32_t* n_nodes, int B, void* out, float* out_lse, void* ws, size_t ws_bytes,
-                cudaStream_t s) {
+                cudaStream_t s, int early = 0) {
   int st = kv_check(kv);
   if (st) return st;
   if (!dtype_ok(dtype) || B < 0 || B > MAX_B) return DDTREE_ERR_INVALID_ARG;
@@ -249,7 +249,7 @@ int attn_launch(const void* q, const void* k_cache, const void* v_cache, int dty
     const size_t need = attn_tc_ws_bytes(g, num_sms());
     if (need && (!ws || !aligned16(ws) || ws_bytes < need)) return DDTREE_ERR_INVALID_ARG;
     return attn_tc_launch(q, k_cache, v_cache, block_table, prefix_len, anc, n_nodes, g, out, out_lse, ws,
-                          num_sms(), s, g_attn_wait_ns, g_attn_stop_tile);
+                          num_sms(), s, g_attn_wait_ns, g_attn_stop_tile, early);
   }
   const long long grid =
       (long long)g.layers * g.n_req * g.n * ((g.Hq + ATTN_SIMT_WARPS - 1) / ATTN_SIMT_WARPS);
@@ -656,8 +656,12 @@ static int round_stages(const ddtree_round_args* a, cudaStream_t stream, char* w
     if (st) return st;
   }
   if ((st = mk.next("ddtree_tree_attn"))) return st;
+  // Directly after the build (no RoPE write in between), the attention starts
+  // while the build runs: its prefix tiles need no tree (the kernels wait for
+  // the build before the tree tiles and the epilogue).
   st = attn_launch(a->q, a->k_cache, a->v_cache, a->dtype, &a->kv, a->block_table, a->prefix_len, a->anc,
-                   a->n_nodes, a->B, a->attn_out, a->attn_lse, ws + off_attn, off_acc - off_attn, stream);
+                   a->n_nodes, a->B, a->attn_out, a->attn_lse, ws + off_attn, off_acc - off_attn, stream,
+                   a->tree_k_in == nullptr ? 1 : 0);
   if (st) return st;
   if ((st = mk.next("ddtree_accept"))) return st;
   if (a->target_hidden != nullptr) {   // the target's argmax from its LM head, logits never written

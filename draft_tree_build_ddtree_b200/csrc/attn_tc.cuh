@@ -476,13 +476,12 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int hq = kvh * p.G + row % p.G;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const uint32_t* arow = p.anc + ((size_t)r * g.n + min(node, g.n - 1)) * g.W;
-    int nn_act = nn;                                      // the tree's node count, once the build is seen done
-    bool tree_seen = !early;
+    // this row's node exists (1) or not (0); -1 until the build is seen done
+    int row_live = early ? -1 : (node < nn ? 1 : 0);
     auto see_tree = [&]() {
-      if (!tree_seen) {
+      if (row_live < 0) {
         griddep_wait();
-        nn_act = p.n_nodes[r];
-        tree_seen = true;
+        row_live = node < p.n_nodes[r] ? 1 : 0;
       }
     };
     float m_used = -INFINITY;      // running max (log2 units) the accumulation uses
@@ -513,11 +512,11 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           if (j0 <= -32) {
             word = 0xffffffffu;                        // all prefix keys
           } else if (j0 < 0) {
-            word = (node < nn_act ? (arow[0] << (-j0)) : 0u) | ((1u << (-j0)) - 1u);
+            word = (row_live ? (arow[0] << (-j0)) : 0u) | ((1u << (-j0)) - 1u);
           } else {
             const int wi = j0 >> 5, sh = j0 & 31;
-            const uint32_t lo = (node < nn_act && wi < g.W) ? arow[wi] : 0u;
-            const uint32_t hi = (node < nn_act && wi + 1 < g.W) ? arow[wi + 1] : 0u;
+            const uint32_t lo = (row_live && wi < g.W) ? arow[wi] : 0u;
+            const uint32_t hi = (row_live && wi + 1 < g.W) ? arow[wi + 1] : 0u;
             word = __funnelshift_r(lo, hi, sh);
           }
           mw[w] = word;
@@ -592,7 +591,7 @@ tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (fin) fin = mbar_wait(&sm.bar_pvdone, (nt - 1) & 1, abort, p.wait_ns);
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
-      const bool live = node < nn_act;
+      const bool live = row_live != 0;
       if (p.splits == 1) {
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
         __nv_bfloat16* orow =

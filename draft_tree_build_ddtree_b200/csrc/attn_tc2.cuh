@@ -161,7 +161,6 @@ struct T2Params {
   int lpt;
   uint64_t wait_ns;
   int stop_tile;
-  int early;           // 1: launched while the tree is still being built (see the kernel)
 };
 
 template <int D>
@@ -206,20 +205,13 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   }
   const int nodes_per_tile = TC_BM / p.G;
   const int mt0 = mp * p.nq;                          // first M-tile of this CTA
-  const int P = p.prefix_len[r];
-  const long long cap = g.paged ? (long long)g.max_blocks * DDTREE_PAGE : (long long)g.s_max;
-  // Early start (inside a round, contiguous cache): the build of this round's
-  // tree may still be running.  The CTA tiles over the budget's node bound
-  // g.n (keys >= P + n_nodes are masked anyway) and its softmax warps wait for
-  // the build only before the first tile holding tree slots and before the
-  // epilogue, which are the only readers of the tree.  Otherwise it waits here.
-  const bool early = p.early && P >= 0 && (long long)P + g.n <= cap;
-  if (!early) griddep_wait();
-  const int nn = early ? g.n : p.n_nodes[r];          // node bound of the tiling
+  const int nn = p.n_nodes[r];
   const int node_base = mt0 * nodes_per_tile;
   if (node_base >= nn) return;                        // no live node in this CTA's M-tiles
   // M-tiles of this CTA holding a live node (1 or 2)
   const int ntl = (p.nq == 2 && node_base + nodes_per_tile < nn && mt0 + 1 < p.mtiles) ? 2 : 1;
+  const int P = p.prefix_len[r];
+  const long long cap = g.paged ? (long long)g.max_blocks * DDTREE_PAGE : (long long)g.s_max;
   if (P < 0 || (long long)P + nn > cap) {
     if (tid == 0 && mp == 0 && kvh == 0 && split == 0) flag_status(DDTREE_STATUS_CAPACITY);
     return;
@@ -401,15 +393,6 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t tm_s = tmem + 128 * t + lane_off;
     const uint32_t tm_o = tmem + 256 + 128 * t + lane_off;
     const uint32_t* arow = p.anc + ((size_t)r * g.n + min(node, g.n - 1)) * g.W;
-    int nn_act = nn;                                       // the tree's node count, once the build is seen done
-    bool tree_seen = !early;
-    auto see_tree = [&]() {
-      if (!tree_seen) {
-        griddep_wait();
-        nn_act = p.n_nodes[r];
-        tree_seen = true;
-      }
-    };
     float m_used = -INFINITY;
     float l = 0.f;
     bool ok = t < ntl;
@@ -423,7 +406,6 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       for (int c = 0; c < T2_BN / 32; ++c) tmem_ld32(tm_s + c * 32, s + 32 * c);
       tmem_wait_ld();
       if (k0 + T2_BN > P) {     // keys >= P are tree slots (visible iff an ancestor); keys >= T absent
-        see_tree();
 #pragma unroll
         for (int w = 0; w < T2_BN / 32; ++w) {
           const int j0 = k0 + 32 * w - P;              // tree index of the word's first key
@@ -431,11 +413,11 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           if (j0 <= -32) {
             word = 0xffffffffu;
           } else if (j0 < 0) {
-            word = (node < nn_act ? (arow[0] << (-j0)) : 0u) | ((1u << (-j0)) - 1u);
+            word = (node < nn ? (arow[0] << (-j0)) : 0u) | ((1u << (-j0)) - 1u);
           } else {
             const int wi = j0 >> 5, sh = j0 & 31;
-            const uint32_t lo = (node < nn_act && wi < g.W) ? arow[wi] : 0u;
-            const uint32_t hi = (node < nn_act && wi + 1 < g.W) ? arow[wi + 1] : 0u;
+            const uint32_t lo = (node < nn && wi < g.W) ? arow[wi] : 0u;
+            const uint32_t hi = (node < nn && wi + 1 < g.W) ? arow[wi + 1] : 0u;
             word = __funnelshift_r(lo, hi, sh);
           }
 #pragma unroll
@@ -530,14 +512,13 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       mbar_arrive(&sm.bar_pready[t]);
     }
     // ---- epilogue ----
-    see_tree();
     bool fin = ok && nt > 0;
     if (fin) fin = mbar_wait(&sm.bar_odone, 0, abort, wlim);
     const int mt = mt0 + t;
     const size_t munit = (((size_t)layer * g.n_req + r) * g.Hkv + kvh) * p.mtiles + mt;
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
-      const bool live = node < nn_act && DDT_IN_RANGE(node, 0, g.n);
+      const bool live = node < nn && DDT_IN_RANGE(node, 0, g.n);
       if (p.splits == 1) {
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
         __nv_bfloat16* orow =
@@ -639,6 +620,10 @@ inline int attn_tc_launch(const void* q, const void* kc, const void* vc, const i
                           const int32_t* prefix_len, const uint32_t* anc, const int32_t* n_nodes, const AttnGeom& g,
                           void* out, float* out_lse, void* ws, int num_sms, cudaStream_t stream,
                           uint64_t wait_ns = 0, int stop_tile = -1, int early = 0) {
+  // early: inside a round, directly after the build.  The single-M-tile
+  // kernel then starts while the tree is built; this kernel's 168-register
+  // softmax has no room for the late wait that needs (its spills grew from 24
+  // to 52 bytes and its launches were 2-4% slower), so it launches plainly.
   const AttnDispatch d = attn_dispatch(g, num_sms);
   if (!d.v2)
     return tc_attn_launch(q, kc, vc, block_table, prefix_len, anc, n_nodes, g, out, out_lse, ws, num_sms, stream,
@@ -662,7 +647,6 @@ inline int attn_tc_launch(const void* q, const void* kc, const void* vc, const i
   p.lpt = (d.splits == 1 && g.n_req > 1 && g.n_req <= TC_LPT_MAX_REQ) ? 1 : 0;
   p.wait_ns = wait_ns > 0 ? wait_ns : TC_WAIT_NS;
   p.stop_tile = stop_tile;
-  p.early = (early && !g.paged && !p.lpt) ? 1 : 0;   // start during the build (see the kernel)
   const size_t slots = (size_t)g.layers * g.n_req * g.Hkv * d.mtiles * d.splits;
   if (d.splits > 1) {
     p.ws_o = (float*)ws;
@@ -694,12 +678,12 @@ inline int attn_tc_launch(const void* q, const void* kc, const void* vc, const i
   }
   const long long grid = (long long)d.units2 * d.splits;
   if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
+  if (g.D == 64)
+    tree_attn_tc2_kernel<64><<<(unsigned)grid, T2_THREADS, t2_smem_bytes<64>(), stream>>>(mq, mk, mv, p);
+  else
+    tree_attn_tc2_kernel<128><<<(unsigned)grid, T2_THREADS, t2_smem_bytes<128>(), stream>>>(mq, mk, mv, p);
   {
-    cudaError_t e = g.D == 64 ? launch_maybe_pdl(tree_attn_tc2_kernel<64>, dim3((unsigned)grid), dim3(T2_THREADS),
-                                                 t2_smem_bytes<64>(), stream, p.early != 0, mq, mk, mv, p)
-                              : launch_maybe_pdl(tree_attn_tc2_kernel<128>, dim3((unsigned)grid), dim3(T2_THREADS),
-                                                 t2_smem_bytes<128>(), stream, p.early != 0, mq, mk, mv, p);
-    if (e == cudaSuccess) e = cudaGetLastError();
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "tree attention (two M-tiles): launch");
   }
   if (d.splits > 1) {

@@ -522,7 +522,8 @@ def measure(w, a, device, steps, warmup, shard=None, world=1, rank=0, clocks=Non
         stage_l2[name] = "L2 flushed before each launch"
     del flush_buf
     return dict(w=w_run, sets=sets, R=R, per_set=per_set, ms=ms_max, steps=steps, status=status,
-                stage_ms=stage_ms, stage_l2=stage_l2, work=work, round_us=round_us, eager_rps=eager_rps, use_graph=use_graph, host0=host0,
+                stage_ms=stage_ms, stage_l2=stage_l2, work=work, round_us=round_us, eager_rps=eager_rps,
+                use_graph=use_graph, host0=host0,
                 launches=dd.ddtree_round_launch_count(sets[0], sets[0]._args),
                 accept_len_mean=float(torch.cat([rb.acc.accept_len.float() for rb in sets]).mean().item()))
 

@@ -161,9 +161,12 @@ struct T2Params {
   int lpt;
   uint64_t wait_ns;
   int stop_tile;
+  int early;           // 1: launched (EARLY instance) while the tree is still being built
 };
 
-template <int D>
+// EARLY: the instance a round launches for a split key range directly after
+// the build (see the host side); the plain instance reads the tree at once.
+template <int D, bool EARLY>
 __global__ void __launch_bounds__(T2_THREADS, 1)
 tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const T2Params p) {
@@ -205,7 +208,24 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   }
   const int nodes_per_tile = TC_BM / p.G;
   const int mt0 = mp * p.nq;                          // first M-tile of this CTA
-  const int nn = p.n_nodes[r];
+  // EARLY: the build of this round's tree may still be running.  The CTA
+  // tiles over the budget's node bound g.n (keys >= P + n_nodes are masked
+  // anyway); its softmax warps wait for the build before their first tile if
+  // the CTA's key range reaches the tree slots, else before the epilogue, the
+  // only readers of the tree, so splits holding prefix tiles only run while
+  // the tree is built.  Without room in the tiling (P + g.n beyond the
+  // cache) it waits here.
+  bool early = false;
+  int nn;
+  if constexpr (EARLY) {
+    const int Pe = p.prefix_len[r];
+    const long long cape = g.paged ? (long long)g.max_blocks * DDTREE_PAGE : (long long)g.s_max;
+    early = p.early && Pe >= 0 && (long long)Pe + g.n <= cape;
+    if (!early) griddep_wait();
+    nn = early ? g.n : p.n_nodes[r];
+  } else {
+    nn = p.n_nodes[r];
+  }
   const int node_base = mt0 * nodes_per_tile;
   if (node_base >= nn) return;                        // no live node in this CTA's M-tiles
   // M-tiles of this CTA holding a live node (1 or 2)
@@ -396,6 +416,15 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     float m_used = -INFINITY;
     float l = 0.f;
     bool ok = t < ntl;
+    int nn_r = nn;                                         // the request's node count once the tree is read
+    [[maybe_unused]] bool tree_seen = !early;
+    if constexpr (EARLY) {
+      if (!tree_seen && (long long)t_end * T2_BN > P) {   // this key range reaches the tree slots
+        griddep_wait();
+        nn_r = p.n_nodes[r];
+        tree_seen = true;
+      }
+    }
     for (int jj = 0; ok && jj < nt; ++jj) {
       const int k0 = (t_begin + jj) * T2_BN;
       // tcgen05.ld/st are warp-collective: every exit and branch around them is warp-uniform
@@ -413,11 +442,11 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           if (j0 <= -32) {
             word = 0xffffffffu;
           } else if (j0 < 0) {
-            word = (node < nn ? (arow[0] << (-j0)) : 0u) | ((1u << (-j0)) - 1u);
+            word = (node < nn_r ? (arow[0] << (-j0)) : 0u) | ((1u << (-j0)) - 1u);
           } else {
             const int wi = j0 >> 5, sh = j0 & 31;
-            const uint32_t lo = (node < nn && wi < g.W) ? arow[wi] : 0u;
-            const uint32_t hi = (node < nn && wi + 1 < g.W) ? arow[wi + 1] : 0u;
+            const uint32_t lo = (node < nn_r && wi < g.W) ? arow[wi] : 0u;
+            const uint32_t hi = (node < nn_r && wi + 1 < g.W) ? arow[wi + 1] : 0u;
             word = __funnelshift_r(lo, hi, sh);
           }
 #pragma unroll
@@ -512,13 +541,20 @@ tree_attn_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       mbar_arrive(&sm.bar_pready[t]);
     }
     // ---- epilogue ----
+    if constexpr (EARLY) {
+      if (!tree_seen) {
+        griddep_wait();
+        nn_r = p.n_nodes[r];
+        tree_seen = true;
+      }
+    }
     bool fin = ok && nt > 0;
     if (fin) fin = mbar_wait(&sm.bar_odone, 0, abort, wlim);
     const int mt = mt0 + t;
     const size_t munit = (((size_t)layer * g.n_req + r) * g.Hkv + kvh) * p.mtiles + mt;
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
-      const bool live = node < nn && DDT_IN_RANGE(node, 0, g.n);
+      const bool live = node < nn_r && DDT_IN_RANGE(node, 0, g.n);
       if (p.splits == 1) {
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
         __nv_bfloat16* orow =
@@ -621,9 +657,10 @@ inline int attn_tc_launch(const void* q, const void* kc, const void* vc, const i
                           void* out, float* out_lse, void* ws, int num_sms, cudaStream_t stream,
                           uint64_t wait_ns = 0, int stop_tile = -1, int early = 0) {
   // early: inside a round, directly after the build.  The single-M-tile
-  // kernel then starts while the tree is built; this kernel's 168-register
-  // softmax has no room for the late wait that needs (its spills grew from 24
-  // to 52 bytes and its launches were 2-4% slower), so it launches plainly.
+  // kernel then starts while the tree is built; so does this kernel's EARLY
+  // instance for a split key range.  Unsplit units reach the tree slots at
+  // once, and the late wait costs the 168-register softmax spills, so they
+  // take the plain instance and launch plainly.
   const AttnDispatch d = attn_dispatch(g, num_sms);
   if (!d.v2)
     return tc_attn_launch(q, kc, vc, block_table, prefix_len, anc, n_nodes, g, out, out_lse, ws, num_sms, stream,
@@ -647,6 +684,7 @@ inline int attn_tc_launch(const void* q, const void* kc, const void* vc, const i
   p.lpt = (d.splits == 1 && g.n_req > 1 && g.n_req <= TC_LPT_MAX_REQ) ? 1 : 0;
   p.wait_ns = wait_ns > 0 ? wait_ns : TC_WAIT_NS;
   p.stop_tile = stop_tile;
+  p.early = (early && !g.paged && !p.lpt && d.splits > 1) ? 1 : 0;
   const size_t slots = (size_t)g.layers * g.n_req * g.Hkv * d.mtiles * d.splits;
   if (d.splits > 1) {
     p.ws_o = (float*)ws;
@@ -668,22 +706,35 @@ inline int attn_tc_launch(const void* q, const void* kc, const void* vc, const i
   }
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tree_attn_tc2_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)t2_smem_bytes<128>());
+    cudaError_t e = cudaFuncSetAttribute(tree_attn_tc2_kernel<128, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)t2_smem_bytes<128>());
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(tree_attn_tc2_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(tree_attn_tc2_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)t2_smem_bytes<64>());
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tree_attn_tc2_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)t2_smem_bytes<128>());
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tree_attn_tc2_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)t2_smem_bytes<64>());
     if (e != cudaSuccess) return cuda_fail(e, "tree attention (two M-tiles): shared-memory attribute");
     attr_set = true;
   }
   const long long grid = (long long)d.units2 * d.splits;
   if (grid > 0x7fffffffLL) return DDTREE_ERR_UNSUPPORTED;
-  if (g.D == 64)
-    tree_attn_tc2_kernel<64><<<(unsigned)grid, T2_THREADS, t2_smem_bytes<64>(), stream>>>(mq, mk, mv, p);
-  else
-    tree_attn_tc2_kernel<128><<<(unsigned)grid, T2_THREADS, t2_smem_bytes<128>(), stream>>>(mq, mk, mv, p);
   {
-    cudaError_t e = cudaGetLastError();
+    const dim3 gd((unsigned)grid), bd(T2_THREADS);
+    cudaError_t e;
+    if (p.early)
+      e = g.D == 64 ? launch_maybe_pdl(tree_attn_tc2_kernel<64, true>, gd, bd, t2_smem_bytes<64>(), stream, true, mq,
+                                       mk, mv, p)
+                    : launch_maybe_pdl(tree_attn_tc2_kernel<128, true>, gd, bd, t2_smem_bytes<128>(), stream, true,
+                                       mq, mk, mv, p);
+    else if (g.D == 64)
+      tree_attn_tc2_kernel<64, false><<<gd, bd, t2_smem_bytes<64>(), stream>>>(mq, mk, mv, p);
+    else
+      tree_attn_tc2_kernel<128, false><<<gd, bd, t2_smem_bytes<128>(), stream>>>(mq, mk, mv, p);
+    if (!p.early || e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "tree attention (two M-tiles): launch");
   }
   if (d.splits > 1) {

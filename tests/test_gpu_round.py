@@ -115,6 +115,26 @@ def test_round_p32k_b1024(sigma):
     check_round(w, rb, h, nodes=[0, 1, 17, 512, 1023, 1024], heads=[0, 13, 31])
 
 
+@pytest.mark.parametrize("floor_node", [None, 20])
+def test_round_p32k_b64_split(floor_node):
+    """sweep_p32k at B = 64 end to end: the two-M-tile attention split twelve
+    ways inside the round, the splits holding prefix tiles only started while
+    the tree is built; with a gain floor the tree stops short of the budget,
+    so the attention tiles over more nodes than the tree has."""
+    w = datagen.workload(5)
+    assert dd.attn_plan(dd.kv_desc(1, 1, w.Hq, w.Hkv, w.D, s_max=32896), w.B) == ("two_mtile", 12)
+    floor = None
+    if floor_node is not None:
+        z, ids, lp32, lse32, root, trees, st = tree_inputs(w)
+        floor = np.array([float(st["score"][0, floor_node])], np.float32)
+    rb, h = make_round(w, gain_floor=floor)
+    dd.ddtree_round(rb)
+    torch.cuda.synchronize()
+    if floor_node is not None:
+        assert int(rb.tree.n_nodes[0]) < w.n
+    check_round(w, rb, h, nodes=[0, 1, 7, 15, 20] + ([] if floor_node else [40, 64]), heads=[0, 13, 31])
+
+
 def test_round_batched_paged_sampled():
     w = datagen.workload(4)
     rb, h = make_round(w)
